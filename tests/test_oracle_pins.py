@@ -1,0 +1,357 @@
+"""Pins of the fp64 oracle to facts outside itself (closed forms, the pages'
+printed numbers, textbook special cases, invariants, hand-worked cases)."""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import kv_budget as kb
+from oracle import mla_oracle as om
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_table(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name), encoding="utf-8") as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+# ---------------------------------------------------------------- mscale / scale
+
+def test_mscale_closed_form():
+    # ln 64 = 6 ln 2, so 0.1 ln 64 + 1 = 1.41588830833597 (YaRN section 3.4 with s = 64).
+    assert om.yarn_get_mscale(64.0, 1.0) == pytest.approx(1.4158883083359671, abs=1e-15)
+    assert om.yarn_get_mscale(1.0, 1.0) == 1.0          # no extension, no correction
+    assert om.yarn_get_mscale(0.5, 1.0) == 1.0
+    assert om.yarn_get_mscale(64.0, 0.0) == 1.0         # mscale 0 switches the log term off
+
+
+def test_softmax_scale_closed_form():
+    cfg = om.YarnConfig()
+    # (1 + 0.6 ln 2)^2 / sqrt(192), evaluated with 40-digit decimal arithmetic
+    assert om.softmax_scale(cfg) == pytest.approx(0.14467962580268923172, rel=1e-14)
+    assert om.cos_sin_factor(cfg) == 1.0                # mscale == mscale_all_dim
+    plain = om.YarnConfig(factor=1.0)
+    assert om.softmax_scale(plain) == pytest.approx(1.0 / math.sqrt(192.0), rel=1e-15)
+
+
+# ---------------------------------------------------------------- YaRN table
+
+def test_factor_one_is_textbook_rope():
+    for theta in (1e4, 1e7):
+        f = om.yarn_inv_freq(om.YarnConfig(rope_theta=theta, factor=1.0))
+        # textbook RoPE: a geometric progression starting at 1 with ratio theta^(-2/64)
+        assert f[0] == 1.0
+        ratios = f[1:] / f[:-1]
+        assert np.allclose(ratios, theta ** (-1.0 / 32.0), rtol=1e-13, atol=0)
+
+
+def _rotations_over_original_context(cfg):
+    i = np.arange(cfg.rotary_dim // 2)
+    base = 1.0 / np.power(cfg.rope_theta, i / (cfg.rotary_dim / 2.0))
+    return base, cfg.original_max_position_embeddings * base / (2.0 * math.pi)
+
+
+@pytest.mark.parametrize("theta", [1e4, 1e7])
+def test_yarn_by_parts_behaviour(theta):
+    """YaRN section 3.2: pairs that turn more than beta_fast times over the original
+    context keep their frequency; pairs that turn fewer than beta_slow times are
+    divided by the scale factor; the band between is blended (strictly between)."""
+    cfg = om.YarnConfig(rope_theta=theta)
+    f = om.yarn_inv_freq(cfg)
+    base, rot = _rotations_over_original_context(cfg)
+    keep = rot > cfg.beta_fast
+    interp = rot < cfg.beta_slow
+    assert keep.any() and interp.any()
+    assert np.allclose(f[keep], base[keep], rtol=1e-15, atol=0)
+    assert np.allclose(f[interp], base[interp] / cfg.factor, rtol=1e-15, atol=0)
+    # rounding the band edges outward may keep/interpolate one extra pair at each edge,
+    # but every pair lies within [base/factor, base] and frequencies stay decreasing
+    assert np.all(f <= base * (1 + 1e-15)) and np.all(f >= base / cfg.factor * (1 - 1e-15))
+    assert np.all(np.diff(f) < 0)
+
+
+def test_yarn_band_edges_at_theta_1e4():
+    # Pair 10 turns 36.7 times (> 32) over 4096 positions and pair 11 27.5 times;
+    # pair 22 turns 1.16 times (> 1) and pair 23 0.87 times: the band is pairs 11..22.
+    cfg = om.YarnConfig()
+    base, rot = _rotations_over_original_context(cfg)
+    assert rot[10] > 32 > rot[11] and rot[22] > 1 > rot[23]
+    f = om.yarn_inv_freq(cfg)
+    assert f[10] == pytest.approx(base[10], rel=1e-15)
+    assert f[23] == pytest.approx(base[23] / 64, rel=1e-15)
+    assert base[11] / 64 < f[11] < base[11]
+    assert base[22] / 64 < f[22] < base[22]
+
+
+# ---------------------------------------------------------------- RoPE
+
+def test_rope_matches_complex_rotation():
+    """Rotate-half RoPE is multiplication of z_i = x_i + i x_{i+32} by exp(i p f_i)."""
+    rng = np.random.default_rng(0)
+    cfg = om.YarnConfig()
+    x = rng.standard_normal((5, 64))
+    pos = np.array([0, 1, 4095, 262143, 524287])
+    y = om.rope(x, pos, cfg)
+    z = (x[:, :32] + 1j * x[:, 32:]) * np.exp(1j * pos[:, None] * om.yarn_inv_freq(cfg)[None, :])
+    assert np.allclose(y[:, :32], z.real, atol=1e-12)
+    assert np.allclose(y[:, 32:], z.imag, atol=1e-12)
+    assert np.array_equal(om.rope(x[:1], np.array([0]), cfg), x[:1])   # position 0 is identity
+
+
+def test_rope_preserves_norm_and_is_relative():
+    rng = np.random.default_rng(1)
+    cfg = om.YarnConfig()
+    q = rng.standard_normal(64)
+    k = rng.standard_normal(64)
+    for m, n in [(5, 3), (4095, 17), (262143, 262000), (524287, 1)]:
+        qm = om.rope(q, np.array(m), cfg)
+        kn = om.rope(k, np.array(n), cfg)
+        assert np.linalg.norm(qm) == pytest.approx(np.linalg.norm(q), rel=1e-13)
+        shift = 1000
+        d0 = qm @ kn
+        d1 = om.rope(q, np.array(m - shift), cfg) @ om.rope(k, np.array(n - shift), cfg)
+        assert d0 == pytest.approx(d1, abs=1e-9)
+
+
+# ---------------------------------------------------------------- attention
+
+def _rand_case(rng, N, q_len, H, scale_w=512 ** -0.5):
+    q = rng.standard_normal((q_len, H, 192))
+    c = rng.standard_normal((N, 512))
+    kp = rng.standard_normal((N, 64))
+    wk = rng.standard_normal((H, 128, 512)) * scale_w
+    wv = rng.standard_normal((H, 512, 128)) * scale_w
+    return q, c, kp, wk, wv
+
+
+@pytest.mark.parametrize("N,q_len,H", [(1, 1, 2), (7, 1, 2), (64, 1, 32), (129, 4, 4), (300, 3, 32)])
+def test_absorbed_equals_expanded(N, q_len, H):
+    rng = np.random.default_rng(N * 10 + q_len)
+    cfg = om.YarnConfig()
+    q, c, kp, wk, wv = _rand_case(rng, N, q_len, H)
+    ref = om.mla_attention_expanded(q, c, kp, wk, wv, cfg)
+    kp_rot = om.rope(kp, np.arange(N), cfg)
+    got = om.mla_attention_absorbed(q, c, kp_rot, wk, wv, cfg)
+    assert np.max(np.abs(got - ref)) <= 1e-10 * max(1.0, np.max(np.abs(ref)))
+
+
+def test_absorbed_equals_expanded_4k_context():
+    """The 4K-context decode shape (32 heads, 4096 tokens) in both forms."""
+    rng = np.random.default_rng(4096)
+    cfg = om.YarnConfig()
+    q, c, kp, wk, wv = _rand_case(rng, 4096, 1, 32)
+    ref = om.mla_attention_expanded(q, c, kp, wk, wv, cfg)
+    got = om.mla_attention_absorbed(q, c, om.rope(kp, np.arange(4096), cfg), wk, wv, cfg)
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel <= 1e-10
+
+
+def test_probabilities_sum_to_one_and_respect_causality():
+    rng = np.random.default_rng(2)
+    cfg = om.YarnConfig()
+    q, c, kp, wk, _ = _rand_case(rng, 40, 4, 3)
+    P = om.mla_attention_probs(q, c, kp, wk, cfg)
+    assert np.allclose(P.sum(axis=-1), 1.0, atol=1e-13)
+    for j in range(4):                       # query j sits at position 36 + j
+        assert np.all(P[j, :, 36 + j + 1:] == 0.0)
+        assert np.all(P[j, :, :36 + j + 1] > 0.0)
+
+
+def _zeros(N, H):
+    return (np.zeros((1, H, 192)), np.zeros((N, 512)), np.zeros((N, 64)),
+            np.zeros((H, 128, 512)), np.zeros((H, 512, 128)))
+
+
+def test_hand_single_token_returns_its_value():
+    # N = 1: softmax over one token is 1, so out[h] = W_UV[h]^T c.
+    q, c, kp, wk, wv = _zeros(1, 2)
+    q[0, 0, 0] = 3.0
+    kp[0, 5] = 1.0
+    c[0, 3] = 2.0
+    wv[0, 3, 5] = 0.5      # head 0: out[5] = 2.0 * 0.5 = 1.0
+    wv[1, 3, 7] = -1.5     # head 1: out[7] = 2.0 * -1.5 = -3.0
+    out = om.mla_attention_expanded(q, c, kp, wk, wv, om.YarnConfig())
+    want = np.zeros((1, 2, 128))
+    want[0, 0, 5] = 1.0
+    want[0, 1, 7] = -3.0
+    assert np.array_equal(out, want)
+
+
+def test_hand_designed_scores():
+    # One head, two tokens.  W_UK maps latent dim 0 onto nope dim 0 and q_nope[0] = a, so the
+    # logits are scale*a*c[t,0] = (ln 3, 0): P = (3/4, 1/4).  V reads latent dim 1 = (4, 8):
+    # out = 0.75*4 + 0.25*8 = 5.
+    cfg = om.YarnConfig()
+    q, c, kp, wk, wv = _zeros(2, 1)
+    wk[0, 0, 0] = 1.0
+    q[0, 0, 0] = math.log(3.0) / om.softmax_scale(cfg)
+    c[0, 0], c[1, 0] = 1.0, 0.0
+    c[0, 1], c[1, 1] = 4.0, 8.0
+    wv[0, 1, 0] = 1.0
+    P = om.mla_attention_probs(q, c, kp, wk, cfg)
+    assert np.allclose(P[0, 0], [0.75, 0.25], atol=1e-15)
+    out = om.mla_attention_expanded(q, c, kp, wk, wv, cfg)
+    assert out[0, 0, 0] == pytest.approx(5.0, abs=1e-14)
+    assert np.count_nonzero(out) == 1
+
+
+def test_hand_rope_term():
+    # Plain RoPE (factor 1).  The query (position 1) has q_pe = e_0; token 0 has k_pe = 2 e_32 and
+    # token 1 has k_pe = 3 e_0.  Pair 0 turns 1 rad per position, so the rope dot products are
+    # (cos 1, sin 1).(0, 2) = 2 sin 1 for token 0 and 3 (cos^2 1 + sin^2 1) = 3 for token 1.
+    cfg = om.YarnConfig(factor=1.0)
+    s = om.softmax_scale(cfg)
+    q, c, kp, wk, wv = _zeros(2, 1)
+    q[0, 0, 128] = 1.0
+    kp[0, 32] = 2.0
+    kp[1, 0] = 3.0
+    c[0, 0], c[1, 0] = 1.0, 0.0
+    wv[0, 0, 0] = 1.0                       # V_t[0] = c[t, 0] = (1, 0): out = P_0
+    z0, z1 = s * 2.0 * math.sin(1.0), s * 3.0
+    p0 = math.exp(z0) / (math.exp(z0) + math.exp(z1))
+    out = om.mla_attention_expanded(q, c, kp, wk, wv, cfg)
+    assert out[0, 0, 0] == pytest.approx(p0, abs=1e-14)
+
+
+def test_hand_causal_two_queries():
+    # q_len = 2 over N = 3 with all logits 0: query 0 (position 1) averages tokens 0, 1 and
+    # query 1 (position 2) averages tokens 0, 1, 2.  V_t[0] = c[t, 0] = (3, 6, 30).
+    q, c, kp, wk, wv = _zeros(3, 1)
+    q = np.zeros((2, 1, 192))
+    c[:, 0] = [3.0, 6.0, 30.0]
+    wv[0, 0, 0] = 1.0
+    out = om.mla_attention_expanded(q, c, kp, wk, wv, om.YarnConfig())
+    assert out[0, 0, 0] == pytest.approx(4.5, abs=1e-14)
+    assert out[1, 0, 0] == pytest.approx(13.0, abs=1e-14)
+
+
+def test_constant_latent_returns_constant_value():
+    rng = np.random.default_rng(3)
+    cfg = om.YarnConfig()
+    q, _, kp, wk, wv = _rand_case(rng, 50, 2, 4)
+    cvec = rng.standard_normal(512)
+    c = np.tile(cvec, (50, 1))
+    out = om.mla_attention_expanded(q, c, kp, wk, wv, cfg)
+    want = np.einsum("c,hcv->hv", cvec, wv)
+    assert np.allclose(out, np.broadcast_to(want, out.shape), atol=1e-12)
+
+
+def _build_pool(rng, seqlens, perm_seed, pad_value=None):
+    cfg = om.YarnConfig()
+    nblk = sum((n + 63) // 64 for n in seqlens)
+    perm = np.random.default_rng(perm_seed).permutation(nblk)
+    mb = max((n + 63) // 64 for n in seqlens)
+    bt = np.full((len(seqlens), mb), -1, dtype=np.int64)
+    pool = np.full((nblk, 64, 576), np.nan if pad_value is None else pad_value)
+    rows = []
+    k = 0
+    for s, n in enumerate(seqlens):
+        nb = (n + 63) // 64
+        bt[s, :nb] = perm[k:k + nb]
+        k += nb
+        c = rng.standard_normal((n, 512))
+        kp = om.rope(rng.standard_normal((n, 64)), np.arange(n), cfg)
+        rows.append(np.concatenate([c, kp], axis=1))
+        for t in range(n):
+            pool[bt[s, t // 64], t % 64] = rows[-1][t]
+    return pool, bt, rows
+
+
+def test_page_permutation_and_padding_leave_output_unchanged():
+    cfg = om.YarnConfig()
+    seqlens = [130, 64, 1]
+    rng_a = np.random.default_rng(11)
+    rng_b = np.random.default_rng(11)
+    pool_a, bt_a, rows_a = _build_pool(rng_a, seqlens, perm_seed=1, pad_value=0.0)
+    pool_b, bt_b, rows_b = _build_pool(rng_b, seqlens, perm_seed=2, pad_value=1e30)
+    assert not np.array_equal(bt_a, bt_b)
+    rng = np.random.default_rng(12)
+    q = rng.standard_normal((3, 1, 4, 192))
+    wk = rng.standard_normal((4, 128, 512)) * 512 ** -0.5
+    wv = rng.standard_normal((4, 512, 128)) * 512 ** -0.5
+    out_a = om.mla_decode_from_pool(q, pool_a, bt_a, np.array(seqlens), wk, wv, cfg)
+    out_b = om.mla_decode_from_pool(q, pool_b, bt_b, np.array(seqlens), wk, wv, cfg)
+    assert np.array_equal(out_a, out_b)
+    # and the pooled absorbed form agrees with the per-sequence expanded definition
+    for s, n in enumerate(seqlens):
+        c = rows_a[s][:, :512]
+        ref = om.mla_attention_absorbed(q[s], c, rows_a[s][:, 512:], wk, wv, cfg)
+        assert np.array_equal(out_a[s], ref)
+
+
+def test_oracle_cache_append_roundtrip():
+    rng = np.random.default_rng(5)
+    seqlens = [70, 3]
+    nblk = 3
+    bt = np.array([[2, 0], [1, -1]])
+    pool = np.zeros((nblk, 64, 576), dtype=np.uint16)
+    T = sum(seqlens)
+    c = rng.integers(0, 65536, size=(T, 512), dtype=np.uint16)
+    k = rng.integers(0, 65536, size=(T, 64), dtype=np.uint16)
+    sid = np.array([0] * 70 + [1] * 3)
+    pos = np.concatenate([np.arange(70), np.arange(3)])
+    om.cache_append(pool, bt, sid, pos, c, k)
+    g0 = om.gather_sequence(pool, bt[0], 70)
+    g1 = om.gather_sequence(pool, bt[1], 3)
+    assert np.array_equal(g0, np.concatenate([c[:70], k[:70]], axis=1))
+    assert np.array_equal(g1, np.concatenate([c[70:], k[70:]], axis=1))
+    assert np.array_equal(pool[2, 5, :512], c[5])      # token 5 of seq 0 -> block 2 row 5
+    assert np.array_equal(pool[0, 69 - 64, 512:], k[69])
+
+
+# ---------------------------------------------------------------- cache ledger
+
+def test_page1_per_token_scalars():
+    want = {r[0]: float(r[1]) for r in _read_table("p1_scalars.txt")}
+    per_layer = kb.kv_bytes_per_token(kb.mla_elems_page_estimate(), 1)
+    per_token = kb.kv_bytes_per_token(kb.mla_elems_page_estimate(), 40)
+    assert per_layer == want["mla_bytes_per_token_layer"]
+    assert per_token == want["mla_bytes_per_token_40l"]
+    mha = kb.kv_bytes_per_token(kb.mha_elems(), 40)
+    assert round(mha / per_token) == want["mha_over_mla_ratio"]
+    toks = kb.tokens_fitting(want["kv_budget_gb"] * kb.GB, per_token)
+    assert round(toks / 1000) == want["kv_budget_tokens_k"]
+    full = kb.as_units(kb.cache_bytes(262144, per_token), kb.GiB, 1)
+    assert kb.round_half_up(full / 2, 1) == want["q8_cache_256k_gb"]
+
+
+def test_page1_ledger_table():
+    mla = kb.kv_bytes_per_token(kb.mla_elems_page_estimate(), 40)
+    mha = kb.kv_bytes_per_token(kb.mha_elems(), 40)
+    for label, mla_gb, mha_gb in _read_table("p1_kv_ledger.txt"):
+        k = int(label[:-1])
+        got_mla = kb.as_units(kb.cache_bytes(k * 1024, mla), kb.GiB, 1)
+        assert got_mla == float(mla_gb), label
+        mha_tokens = k * 1000 if k <= 128 else k * 1024
+        digits = 1 if "." in mha_gb else 0
+        got_mha = kb.as_units(kb.cache_bytes(mha_tokens, mha), kb.GiB, digits)
+        assert got_mha == float(mha_gb), label
+
+
+def test_other_pages_ledgers():
+    p2 = kb.kv_bytes_per_token(kb.gqa_elems(4, 256), 16)
+    p3 = kb.kv_bytes_per_token(kb.gqa_elems(4, 256), 18)
+    assert p2 == 64 * 1024 and p3 == 72 * 1024
+    for page, tokens, printed in _read_table("p2_p3_kv_ledgers.txt"):
+        n = int(tokens)
+        if page == "P2":
+            assert kb.as_units(n * p2, kb.GiB, 1) == float(printed)
+        else:
+            gb = n * p3 / kb.GB
+            digits = 1 if "." in printed else 0
+            assert math.floor(gb * 10 ** digits) / 10 ** digits == float(printed)
+
+
+def test_repository_cache_row_is_576_elements():
+    # [c_kv 512 | k_pe 64] bf16 = 1152 B per token and layer; 45 KiB over 40 layers.
+    per_token = kb.kv_bytes_per_token(kb.mla_elems_latent_rope(), 40)
+    assert kb.kv_bytes_per_token(kb.mla_elems_latent_rope(), 1) == 1152
+    assert per_token == 45 * 1024
+    assert kb.cache_bytes(262144, per_token) / kb.GiB == 11.25
