@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""MLA decode throughput on B200: latent-KV HBM GB/s and attended tokens/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl xmla|reference]
+
+A step is one decode step of the whole hot path over every layer of the
+workload: RoPE on the queries and on the q_len new tokens, the append of those
+tokens to the paged latent cache, and xmla_decode (q absorb, split-K latent
+attention, LSE combine with W_UV).  The default workload is a single 256K
+context (batch 1, q_len 1, 64-token pages in a shuffled order).
+
+Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
+events on the launching stream; the L2 is flushed (256 MiB write) before every
+step, outside the events.  The K steps are bracketed by a barrier and a device
+synchronise; the reported time is the max over ranks.  Under torchrun every
+rank runs its own replica of the workload (independent sequences, no
+collective on the data path): weak scaling.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode: latent-KV HBM GB/s (% of B200 peak) and attended tokens/s"
+ROW_BYTES = 1152  # one cache row: [c_kv 512 | k_pe 64] bf16
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_256k")
+    ap.add_argument("--impl", default="xmla", choices=["xmla", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_config(wl, world):
+    return {
+        "workload": wl.name,
+        "batch_per_gpu": wl.batch,
+        "q_len": wl.q_len,
+        "context": wl.seqlens[0] if len(set(wl.seqlens)) == 1 else f"U[8192,65536] mean {sum(wl.seqlens) / len(wl.seqlens):.0f}",
+        "layers": wl.layers,
+        "heads": 32,
+        "cache_row": "[c_kv 512 | k_pe 64] bf16",
+        "paging": "64-token blocks, contiguous" if wl.contiguous else "64-token blocks, shuffled",
+        "l2": "flushed before every timed step (256 MiB write)",
+        "parallelism": f"dp{world} (independent replicas)",
+    }
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+
+def oracle_sample(wl, seconds: float):
+    """Time the fp64 expanded oracle on the first S tokens of sequence 0 (one
+    query at position S-1, 32 heads), S chosen for about `seconds` of work."""
+    import numpy as np
+    import torch
+
+    from mla_latent_kv_yarn_b200 import workloads
+    from oracle import mla_oracle as om
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([t.get("num_threads", 1) for t in threadpool_info()
+                     if t.get("user_api") == "blas"] or [os.cpu_count() or 1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    n_max = wl.seqlens[0]
+    one = workloads.custom(1, 1, [n_max], seed=wl.seed, name=wl.name)
+    inp = workloads.layer_inputs(one, 0, "cpu")
+    c = inp.c_kv.double().numpy()
+    kp = inp.k_pe.double().numpy()
+    wk, wv = inp.W_UK.double().numpy(), inp.W_UV.double().numpy()
+    q = inp.q[0].double().numpy()
+    cfg = om.YarnConfig()
+
+    def run(n):
+        t0 = time.perf_counter()
+        om.mla_attention_expanded(q, c[:n], kp[:n], wk, wv, cfg)
+        return time.perf_counter() - t0
+
+    probe_n = min(n_max, 4096)
+    t_probe = run(probe_n)
+    n = int(min(n_max, max(probe_n, probe_n * seconds / max(t_probe, 1e-6))))
+    n = max(64, n // 64 * 64)
+    return n, run, cores
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, wl):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    per_step = max(1.0, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    n, run, cores = oracle_sample(wl, per_step)
+    for _ in range(args.warmup):
+        run(n)
+    times = [run(n) for _ in range(args.steps)]
+    total = sum(times)
+    gbs = n * ROW_BYTES * args.steps / total / 1e9
+    sample = (f"fp64 expanded oracle (numpy), sequence 0 of {wl.name}, first {n} tokens, "
+              f"32 heads, q_len 1, one layer per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 6), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, world),
+        "attended_tokens_per_s": round(n * args.steps / total, 3),
+        "cpu_baseline": {"value": round(gbs, 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(gbs, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def traffic_record(kernel_src_sha: str, name: str):
+    """DRAM bytes per launch of the split-K kernel from a committed ncu summary,
+    valid only while the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", f"mla_decode_kernel_{name}_dram.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("kernel_source_sha256") == kernel_src_sha:
+            return float(d["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def run_xmla(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    from mla_latent_kv_yarn_b200 import build, session, workloads, xmla
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    build.build()
+    cfg = xmla.xmla_yarn_default()
+    scale = xmla.xmla_softmax_scale(cfg, 192)
+
+    # ---- set up every layer's cache and step inputs on this GPU
+    layers = []
+    for layer in range(wl.layers):
+        inp = workloads.layer_inputs(wl, layer, dev)
+        prefix, new = session.split_prefix(wl, inp)
+        st = session.build_layer(cfg, wl, prefix, dev)
+        layers.append({"st": st, "q": inp.q.clone(), "k_raw": new.k_pe.clone(),
+                       "c_new": new.c_kv.clone(), "pos": new.positions.clone(),
+                       "sid": new.seq_ids.clone(), "k": torch.empty_like(new.k_pe),
+                       "out": torch.empty((wl.batch, wl.q_len, 32, 128), dtype=torch.bfloat16,
+                                          device=dev)})
+        del inp, prefix, new
+    torch.cuda.synchronize()
+    dec = session.Decoder(wl.batch, wl.q_len, wl.max_seqlen, dev)
+    ev_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in layers]
+    for a, b in ev_attn:          # materialise the events before capture
+        a.record()
+        b.record()
+    torch.cuda.synchronize()
+
+    def step(events=True):
+        for L, ev in zip(layers, ev_attn):
+            L["k"].copy_(L["k_raw"])   # the new tokens' rope keys are rotated in place
+            dec.step(cfg, L["st"], L["q"], L["c_new"], L["k"], L["pos"], L["sid"], scale,
+                     out=L["out"], events=ev if events else None)
+
+    # eager warm-up (loads modules), then capture the whole step in a CUDA graph
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+    if dec.check_status() != 0:
+        raise RuntimeError(f"device status {dec.check_status()} after warm-up")
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        graph.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    step_ms, attn_ms = [], []
+    for i in range(args.steps):
+        flush.fill_((i + 1) & 0xFF)
+        e0[i].record(stream)
+        graph.replay()
+        e1[i].record(stream)
+        e1[i].synchronize()
+        step_ms.append(e0[i].elapsed_time(e1[i]))
+        attn_ms.extend(a.elapsed_time(b) for a, b in ev_attn)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    status = dec.check_status()
+
+    # ---- end to end through the API: pinned host inputs in, result out, every step
+    h_in = [{k: L[k].cpu().pin_memory() for k in ("q", "k_raw", "c_new", "pos", "sid")}
+            for L in layers]
+    h_out = [torch.empty_like(L["out"], device="cpu").pin_memory() for L in layers]
+    h2d = sum(t.numel() * t.element_size() for d in h_in for t in d.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    ee0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ee1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e2e_ms = []
+    for i in range(args.steps):
+        flush.fill_((i + 7) & 0xFF)
+        ee0[i].record(stream)
+        for L, h in zip(layers, h_in):
+            for k, v in h.items():
+                L[k].copy_(v, non_blocking=True)
+        graph.replay()
+        for L, h in zip(layers, h_out):
+            h.copy_(L["out"], non_blocking=True)
+        ee1[i].record(stream)
+        ee1[i].synchronize()
+        e2e_ms.append(ee0[i].elapsed_time(ee1[i]))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+
+    cache_bytes_layer = sum(wl.seqlens) * ROW_BYTES
+    tokens_step = sum(wl.seqlens) * wl.layers * world
+    bytes_step = cache_bytes_layer * wl.layers * world
+    gbs = bytes_step * args.steps / (total_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    attn_mean_ms = statistics.mean(attn_ms)
+    achieved = cache_bytes_layer / (attn_mean_ms * 1e-3) / 1e9
+    ksha = hashlib.sha256(open(os.path.join(ROOT, "mla_latent_kv_yarn_b200", "csrc",
+                                            "mla_decode.cu"), "rb").read()).hexdigest()
+    traffic = traffic_record(ksha, wl.name)
+    launches = 5 * wl.layers * args.steps
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(gbs, 3), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(wl, world),
+            "attended_tokens_per_s": round(tokens_step * args.steps / (total_ms * 1e-3), 1),
+            "pct_of_hbm_peak": round(100.0 * gbs / (peak * world), 2),
+            "roofline": {"bound": "hbm", "kernel": f"mla_decode_kernel<{32 if wl.q_len == 1 else 64}>",
+                         "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "algorithmic_bytes_per_launch": cache_bytes_layer,
+                         "kernel_ms": round(attn_mean_ms, 5), "peak_source": peak_kind},
+            "e2e": {"value": round(bytes_step * args.steps / (e2e_total * 1e-3) / 1e9, 3),
+                    "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "splits": dec.splits,
+            "device_status": status,
+        }
+        if clk is not None:
+            line["clocks"] = clk
+        if world == 1 and not args.no_cpu_baseline:
+            n, run, cores = oracle_sample(wl, args.cpu_seconds)
+            t = run(n)
+            line["cpu_baseline"] = {
+                "value": round(n * ROW_BYTES / t / 1e9, 6), "unit": "GB/s", "cores": cores,
+                "kind": "oracle",
+                "sample": f"fp64 expanded oracle (numpy), sequence 0 of {wl.name}, first {n} "
+                          f"tokens, 32 heads, q_len 1, one layer ({t:.1f} s)"}
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    from mla_latent_kv_yarn_b200 import workloads
+    wl = workloads.workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_xmla(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

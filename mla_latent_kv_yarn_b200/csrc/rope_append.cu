@@ -1,0 +1,143 @@
+// YaRN rotary embedding (in place, bf16) and the paged latent-cache append.
+//
+// [P1] "256K 长上下文真能本地用：Xing4.0 原生长上下文的工程代价拆解", section 一:
+//      rope_scaling yarn (frequency table in yarn.cuh).
+// [P5] "mHC+MLA+MTP 是什么？拆开给 Agent 用的百亿 MoE", section "MLA：256K 上下文的
+//      '内存革命'": the cache holds the 512-dim latent and the 64-dim rope key.
+#include <cmath>
+#include <cstdint>
+
+#include "xmla_device.cuh"
+#include "yarn.cuh"
+
+namespace xmla {
+
+// ---------------------------------------------------------------- device: RoPE
+
+// One thread per (vector, pair).  Angle formed in float64 from the exact
+// integer position; the rotated pair is rounded once to bf16.
+__global__ void __launch_bounds__(256) rope_yarn_kernel(__nv_bfloat16* __restrict__ x, int64_t rows,
+                                                        int32_t n_heads, int64_t head_stride,
+                                                        int64_t row_stride, int32_t offset,
+                                                        const int64_t* __restrict__ positions,
+                                                        const RopeTable tab) {
+  const int64_t total = rows * (int64_t)n_heads * (kDRope / 2);
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int i = (int)(idx % (kDRope / 2));
+    const int64_t rh = idx / (kDRope / 2);
+    const int64_t h = rh % n_heads;
+    const int64_t r = rh / n_heads;
+    __nv_bfloat16* v = x + r * row_stride + h * head_stride + offset;
+    double y1, y2;
+    rope_pair((double)__bfloat162float(v[i]), (double)__bfloat162float(v[i + kDRope / 2]),
+              positions[r], i, tab, &y1, &y2);
+    v[i] = __double2bfloat16(y1);
+    v[i + kDRope / 2] = __double2bfloat16(y2);
+  }
+}
+
+// ---------------------------------------------------------------- device: append
+
+// One thread per 16-byte piece of a cache row (64 pieces of latent, 8 of rope key).
+__global__ void __launch_bounds__(256) cache_append_kernel(
+    uint4* __restrict__ pool, int64_t num_blocks, const int32_t* __restrict__ block_table,
+    int32_t max_blocks, int32_t batch, const int32_t* __restrict__ seq_ids,
+    const int64_t* __restrict__ positions, const uint4* __restrict__ c_kv,
+    const uint4* __restrict__ k_pe, int64_t T, int32_t* status) {
+  constexpr int kLatPieces = kDLatent * 2 / 16;  // 64
+  constexpr int kRopePieces = kDRope * 2 / 16;   // 8
+  constexpr int kRowPieces = kLatPieces + kRopePieces;
+  const int64_t total = T * kRowPieces;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = idx / kRowPieces;
+    const int piece = (int)(idx % kRowPieces);
+    const int32_t s = seq_ids[t];
+    const int64_t pos = positions[t];
+    if (s < 0 || s >= batch || pos < 0 || pos >= (int64_t)max_blocks * kPage) {
+      record_status(status, XMLA_ERR_DEVICE_OOB);
+      continue;
+    }
+    const int32_t blk = block_table[(int64_t)s * max_blocks + pos / kPage];
+    if (blk < 0 || (int64_t)blk >= num_blocks) {
+      record_status(status, XMLA_ERR_DEVICE_OOB);
+      continue;
+    }
+    const uint4 val = piece < kLatPieces ? c_kv[t * kLatPieces + piece]
+                                         : k_pe[t * kRopePieces + (piece - kLatPieces)];
+    pool[((int64_t)blk * kPage + pos % kPage) * kRowPieces + piece] = val;
+  }
+}
+
+static int grid_for(int64_t work, int threads) {
+  int64_t g = (work + threads - 1) / threads;
+  if (g > (1 << 20)) g = 1 << 20;
+  return (int)(g < 1 ? 1 : g);
+}
+
+}  // namespace xmla
+
+using namespace xmla;
+
+extern "C" void xmla_yarn_default(xmla_yarn_cfg* cfg) {
+  if (cfg == nullptr) return;
+  cfg->rope_theta = 10000.0;
+  cfg->factor = 64.0;
+  cfg->original_max_position_embeddings = 4096;
+  cfg->beta_fast = 32.0;
+  cfg->beta_slow = 1.0;
+  cfg->mscale = 1.0;
+  cfg->mscale_all_dim = 1.0;
+  cfg->rotary_dim = kDRope;
+}
+
+extern "C" xmla_status xmla_yarn_inv_freq(const xmla_yarn_cfg* cfg, double* inv_freq_out) {
+  if (!yarn_cfg_ok(cfg) || inv_freq_out == nullptr) return XMLA_ERR_INVALID_ARG;
+  if (cfg->rotary_dim != kDRope) return XMLA_ERR_SHAPE;
+  yarn_table(cfg, inv_freq_out);
+  return XMLA_OK;
+}
+
+extern "C" double xmla_softmax_scale(const xmla_yarn_cfg* cfg, int32_t qk_head_dim) {
+  if (cfg == nullptr || qk_head_dim <= 0) return 0.0;
+  const double m = mscale_of(cfg->factor, cfg->mscale_all_dim);
+  return m * m / std::sqrt((double)qk_head_dim);
+}
+
+extern "C" xmla_status xmla_rope_yarn(const xmla_yarn_cfg* cfg, void* x, int64_t rows,
+                                      int32_t n_heads, int64_t head_stride_elems,
+                                      int64_t row_stride_elems, int32_t rope_offset_elems,
+                                      const int64_t* positions, void* stream) {
+  if (!yarn_cfg_ok(cfg)) return XMLA_ERR_INVALID_ARG;
+  if (cfg->rotary_dim != kDRope || n_heads < 1 || rows < 0) return XMLA_ERR_SHAPE;
+  if (rows == 0) return XMLA_OK;
+  if (x == nullptr || positions == nullptr || head_stride_elems < 0 || row_stride_elems < 0 ||
+      rope_offset_elems < 0)
+    return XMLA_ERR_INVALID_ARG;
+  const RopeTable tab = make_rope_table(cfg);
+  const int64_t work = rows * n_heads * (kDRope / 2);
+  rope_yarn_kernel<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(
+      (__nv_bfloat16*)x, rows, n_heads, head_stride_elems, row_stride_elems, rope_offset_elems,
+      positions, tab);
+  return cudaGetLastError() == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+}
+
+extern "C" xmla_status xmla_cache_append(void* pool, int64_t num_blocks, const int32_t* block_table,
+                                         int32_t max_blocks, int32_t batch, const int32_t* seq_ids,
+                                         const int64_t* positions, const void* c_kv,
+                                         const void* k_pe_rot, int64_t T, int32_t* status_dev,
+                                         void* stream) {
+  if (T < 0 || num_blocks < 1 || max_blocks < 1 || batch < 1) return XMLA_ERR_SHAPE;
+  if (T == 0) return XMLA_OK;
+  if (pool == nullptr || block_table == nullptr || seq_ids == nullptr || positions == nullptr ||
+      c_kv == nullptr || k_pe_rot == nullptr)
+    return XMLA_ERR_INVALID_ARG;
+  if ((((uintptr_t)pool) | ((uintptr_t)c_kv) | ((uintptr_t)k_pe_rot)) & 15u)
+    return XMLA_ERR_INVALID_ARG;
+  const int64_t work = T * 72;
+  cache_append_kernel<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(
+      (uint4*)pool, num_blocks, block_table, max_blocks, batch, seq_ids, positions,
+      (const uint4*)c_kv, (const uint4*)k_pe_rot, T, status_dev);
+  return cudaGetLastError() == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+}

@@ -1,0 +1,187 @@
+"""ctypes binding of libxmla (include/xmla.h), same names as the C ABI.
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+Tensors are torch tensors on the current CUDA device; the stream defaults to
+torch's current stream.  A non-OK status raises XmlaError.  Loading fails
+loudly when the shared library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libxmla.so")
+
+XMLA_OK = 0
+STATUS_NAMES = {
+    0: "XMLA_OK", 1: "XMLA_ERR_INVALID_ARG", 2: "XMLA_ERR_SHAPE", 3: "XMLA_ERR_WORKSPACE",
+    4: "XMLA_ERR_CUDA", 5: "XMLA_ERR_DEVICE_OOB", 6: "XMLA_ERR_TIMEOUT", 7: "XMLA_ERR_UNSUPPORTED",
+}
+
+# Every symbol include/xmla.h declares.
+EXPORTS = [
+    "xmla_yarn_default", "xmla_yarn_inv_freq", "xmla_softmax_scale", "xmla_rope_yarn",
+    "xmla_cache_append", "xmla_decode_workspace_size", "xmla_decode_num_splits", "xmla_decode",
+    "xmla_decode_profiled", "xmla_selftest_wait_timeout", "xmla_status_string",
+]
+
+
+class XmlaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({xmla_status_string(status)})")
+        self.status = status
+
+
+class xmla_yarn_cfg(ctypes.Structure):
+    _fields_ = [
+        ("rope_theta", ctypes.c_double),
+        ("factor", ctypes.c_double),
+        ("original_max_position_embeddings", ctypes.c_int64),
+        ("beta_fast", ctypes.c_double),
+        ("beta_slow", ctypes.c_double),
+        ("mscale", ctypes.c_double),
+        ("mscale_all_dim", ctypes.c_double),
+        ("rotary_dim", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libxmla.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libxmla.so not built at {LIB_PATH}; run mla_latent_kv_yarn_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f32, f64, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                                      ctypes.c_float, ctypes.c_double, ctypes.c_size_t)
+        cfgp = ctypes.POINTER(xmla_yarn_cfg)
+        L.xmla_yarn_default.argtypes = [cfgp]
+        L.xmla_yarn_default.restype = None
+        L.xmla_yarn_inv_freq.argtypes = [cfgp, ctypes.POINTER(ctypes.c_double)]
+        L.xmla_yarn_inv_freq.restype = ctypes.c_int
+        L.xmla_softmax_scale.argtypes = [cfgp, i32]
+        L.xmla_softmax_scale.restype = f64
+        L.xmla_rope_yarn.argtypes = [cfgp, vp, i64, i32, i64, i64, i32, vp, vp]
+        L.xmla_rope_yarn.restype = ctypes.c_int
+        L.xmla_cache_append.argtypes = [vp, i64, vp, i32, i32, vp, vp, vp, vp, i64, vp, vp]
+        L.xmla_cache_append.restype = ctypes.c_int
+        L.xmla_decode_workspace_size.argtypes = [i32, i32, i64, i32, i32]
+        L.xmla_decode_workspace_size.restype = sz
+        L.xmla_decode_num_splits.argtypes = [i32, i32, i64, i32, i32]
+        L.xmla_decode_num_splits.restype = i32
+        L.xmla_decode.argtypes = [cfgp, vp, vp, vp, vp, i64, vp, i32, vp, i32, i32, i64, f32, i32,
+                                  vp, sz, vp, vp, vp]
+        L.xmla_decode.restype = ctypes.c_int
+        L.xmla_decode_profiled.argtypes = L.xmla_decode.argtypes + [vp, vp]
+        L.xmla_decode_profiled.restype = ctypes.c_int
+        L.xmla_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
+        L.xmla_selftest_wait_timeout.restype = ctypes.c_int
+        L.xmla_status_string.argtypes = [ctypes.c_int]
+        L.xmla_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != XMLA_OK:
+        raise XmlaError(status, what)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def xmla_status_string(status: int) -> str:
+    return lib().xmla_status_string(int(status)).decode()
+
+
+def xmla_yarn_default() -> xmla_yarn_cfg:
+    cfg = xmla_yarn_cfg()
+    lib().xmla_yarn_default(ctypes.byref(cfg))
+    return cfg
+
+
+def xmla_yarn_inv_freq(cfg: xmla_yarn_cfg) -> list[float]:
+    out = (ctypes.c_double * (cfg.rotary_dim // 2))()
+    _check(lib().xmla_yarn_inv_freq(ctypes.byref(cfg), out), "xmla_yarn_inv_freq")
+    return list(out)
+
+
+def xmla_softmax_scale(cfg: xmla_yarn_cfg, qk_head_dim: int = 192) -> float:
+    return float(lib().xmla_softmax_scale(ctypes.byref(cfg), int(qk_head_dim)))
+
+
+def xmla_rope_yarn(cfg: xmla_yarn_cfg, x: torch.Tensor, rows: int, n_heads: int,
+                   head_stride_elems: int, row_stride_elems: int, rope_offset_elems: int,
+                   positions: torch.Tensor, stream=None) -> None:
+    _check(lib().xmla_rope_yarn(ctypes.byref(cfg), _ptr(x), int(rows), int(n_heads),
+                                int(head_stride_elems), int(row_stride_elems),
+                                int(rope_offset_elems), _ptr(positions), _stream(stream)),
+           "xmla_rope_yarn")
+
+
+def xmla_cache_append(pool: torch.Tensor, num_blocks: int, block_table: torch.Tensor,
+                      max_blocks: int, batch: int, seq_ids: torch.Tensor, positions: torch.Tensor,
+                      c_kv: torch.Tensor, k_pe_rot: torch.Tensor, T: int,
+                      status: torch.Tensor | None = None, stream=None) -> None:
+    _check(lib().xmla_cache_append(_ptr(pool), int(num_blocks), _ptr(block_table),
+                                   int(max_blocks), int(batch), _ptr(seq_ids), _ptr(positions),
+                                   _ptr(c_kv), _ptr(k_pe_rot), int(T), _ptr(status),
+                                   _stream(stream)),
+           "xmla_cache_append")
+
+
+def xmla_decode_workspace_size(batch: int, q_len: int, max_seqlen: int, num_sms: int,
+                               num_splits: int = 0) -> int:
+    return int(lib().xmla_decode_workspace_size(int(batch), int(q_len), int(max_seqlen),
+                                                int(num_sms), int(num_splits)))
+
+
+def xmla_decode_num_splits(batch: int, q_len: int, max_seqlen: int, num_sms: int,
+                           num_splits: int = 0) -> int:
+    return int(lib().xmla_decode_num_splits(int(batch), int(q_len), int(max_seqlen),
+                                            int(num_sms), int(num_splits)))
+
+
+def xmla_decode(cfg: xmla_yarn_cfg, q: torch.Tensor, W_UK: torch.Tensor, W_UV: torch.Tensor, pool: torch.Tensor,
+                num_blocks: int, block_table: torch.Tensor, max_blocks: int,
+                seqlens: torch.Tensor, batch: int, q_len: int, max_seqlen: int,
+                softmax_scale: float, num_splits: int, workspace: torch.Tensor,
+                workspace_bytes: int, status: torch.Tensor | None, out: torch.Tensor,
+                stream=None) -> None:
+    _check(lib().xmla_decode(ctypes.byref(cfg), _ptr(q), _ptr(W_UK), _ptr(W_UV), _ptr(pool), int(num_blocks),
+                             _ptr(block_table), int(max_blocks), _ptr(seqlens), int(batch),
+                             int(q_len), int(max_seqlen), float(softmax_scale), int(num_splits),
+                             _ptr(workspace), int(workspace_bytes), _ptr(status), _ptr(out),
+                             _stream(stream)),
+           "xmla_decode")
+
+
+def xmla_decode_profiled(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens, batch,
+                         q_len, max_seqlen, softmax_scale, num_splits, workspace, workspace_bytes,
+                         status, out, stream=None, attn_start=None, attn_stop=None) -> None:
+    ev = [None if e is None else (e.cuda_event if hasattr(e, "cuda_event") else int(e))
+          for e in (attn_start, attn_stop)]
+    _check(lib().xmla_decode_profiled(ctypes.byref(cfg), _ptr(q), _ptr(W_UK), _ptr(W_UV), _ptr(pool), int(num_blocks),
+                                      _ptr(block_table), int(max_blocks), _ptr(seqlens), int(batch),
+                                      int(q_len), int(max_seqlen), float(softmax_scale),
+                                      int(num_splits), _ptr(workspace), int(workspace_bytes),
+                                      _ptr(status), _ptr(out), _stream(stream), ev[0], ev[1]),
+           "xmla_decode_profiled")
+
+
+def xmla_selftest_wait_timeout(status: torch.Tensor, timeout_ns: int, stream=None) -> None:
+    _check(lib().xmla_selftest_wait_timeout(_ptr(status), int(timeout_ns), _stream(stream)),
+           "xmla_selftest_wait_timeout")

@@ -1,0 +1,252 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from mla_latent_kv_yarn_b200 import session, workloads, xmla
+from oracle import mla_oracle as om
+
+import gpu_cases as gc
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from mla_latent_kv_yarn_b200 import build
+    build.build()
+    torch.cuda.init()
+
+
+# ------------------------------------------------------------------ RoPE
+
+def _half_ulp_bf16(v: np.ndarray) -> np.ndarray:
+    a = np.maximum(np.abs(v), 1e-30)
+    return np.exp2(np.floor(np.log2(a)) - 8.0)
+
+
+@pytest.mark.parametrize("theta,factor", [(1e4, 64.0), (1e7, 64.0), (1e4, 1.0)])
+def test_rope_within_half_ulp_of_oracle(theta, factor):
+    cfg, ocfg = gc.cfgs(theta)
+    cfg.factor = factor
+    ocfg = om.YarnConfig(rope_theta=theta, factor=factor)
+    g = torch.Generator().manual_seed(5)
+    R, H = 37, 32
+    q = torch.randn((R, H, 192), generator=g).to(torch.bfloat16)
+    k = torch.randn((R, 64), generator=g).to(torch.bfloat16)
+    pos = torch.tensor([0, 1, 63, 64, 4095, 4096, 262143, 262144, 524287] +
+                       torch.randint(0, 524288, (R - 9,), generator=g).tolist(), dtype=torch.int64)
+    qd, kd, pd = q.cuda(), k.cuda(), pos.cuda()
+    session.rope_rows(cfg, qd, pd)
+    session.rope_rows(cfg, kd, pd)
+    torch.cuda.synchronize()
+    want_q = om.rope(gc.f64(q)[..., 128:], pos.numpy()[:, None], ocfg)
+    want_k = om.rope(gc.f64(k), pos.numpy(), ocfg)
+    got_q, got_k = gc.f64(qd), gc.f64(kd)
+    assert np.array_equal(got_q[..., :128], gc.f64(q)[..., :128])   # nope part untouched
+    assert np.all(np.abs(got_q[..., 128:] - want_q) <= _half_ulp_bf16(want_q) * (1 + 1e-6))
+    assert np.all(np.abs(got_k - want_k) <= _half_ulp_bf16(want_k) * (1 + 1e-6))
+
+
+# ------------------------------------------------------------------ cache append
+
+def test_cache_append_is_a_bit_exact_scatter():
+    wl = workloads.custom(3, 1, [130, 64, 7], seed=3)
+    bt = workloads.block_table(wl, 0)
+    sid, pos, _ = workloads.token_index(wl)
+    T = wl.tokens
+    g = torch.Generator().manual_seed(9)
+    c_bits = torch.randint(-32768, 32767, (T, 512), generator=g, dtype=torch.int16)
+    k_bits = torch.randint(-32768, 32767, (T, 64), generator=g, dtype=torch.int16)
+    pool0 = torch.randint(-32768, 32767, (wl.num_blocks + 2, 64, 576), generator=g, dtype=torch.int16)
+    pool = pool0.cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    xmla.xmla_cache_append(pool, pool.shape[0], bt.cuda(), bt.shape[1], 3, sid.cuda(), pos.cuda(),
+                           c_bits.cuda(), k_bits.cuda(), T, status)
+    torch.cuda.synchronize()
+    want = pool0.numpy().view(np.uint16).copy()
+    om.cache_append(want, bt.numpy(), sid.numpy(), pos.numpy(), c_bits.numpy().view(np.uint16),
+                    k_bits.numpy().view(np.uint16))
+    assert np.array_equal(pool.cpu().numpy().view(np.uint16), want)
+    assert int(status.item()) == 0
+
+
+def test_cache_append_skips_out_of_range_rows():
+    bt = torch.tensor([[1, 0], [2, 5]], dtype=torch.int32)          # block 5 is outside a 3-block pool
+    sid = torch.tensor([0, 1, 1, 2, 0], dtype=torch.int32)         # seq 2 does not exist
+    pos = torch.tensor([3, 10, 70, 0, 200], dtype=torch.int64)      # 200 is past max_blocks*64
+    c = torch.ones((5, 512), dtype=torch.bfloat16)
+    k = torch.ones((5, 64), dtype=torch.bfloat16)
+    pool = torch.zeros((3, 64, 576), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    xmla.xmla_cache_append(pool, 3, bt.cuda(), 2, 2, sid.cuda(), pos.cuda(), c.cuda(), k.cuda(), 5,
+                           status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 5
+    p = pool.cpu().float()
+    assert torch.all(p[1, 3] == 1) and torch.all(p[2, 10] == 1)    # the two valid rows landed
+    assert float(p.sum()) == 2 * 576
+
+
+# ------------------------------------------------------------------ decode, small cases
+
+SMALL = [
+    # batch, q_len, seqlens, num_splits
+    (1, 1, [1], 0),
+    (1, 1, [64], 0),
+    (1, 1, [65], 0),
+    (4, 1, [8, 16, 24, 40], 0),
+    (2, 1, [1000, 130], 0),
+    (3, 1, [777, 64, 2049], 3),
+    (1, 1, [5000], 1),
+    (1, 1, [300], 16),
+    (2, 2, [129, 70], 0),
+    (2, 3, [500, 63], 2),
+    (2, 4, [1000, 257], 0),
+    (1, 8, [2000], 0),
+    (1, 4, [4], 0),
+]
+
+
+@pytest.mark.parametrize("batch,q_len,seqlens,splits", SMALL)
+def test_decode_matches_expanded_oracle(batch, q_len, seqlens, splits):
+    wl = workloads.custom(batch, q_len, seqlens, seed=sum(seqlens) + q_len)
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg, num_splits=splits)
+    assert dec.check_status() == 0
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg), f"{batch}x{q_len} {seqlens} s={splits}")
+
+
+def test_decode_ignores_garbage_past_sequence_end():
+    """Cache rows past a sequence's end (inside its last block) hold NaN here."""
+    wl = workloads.custom(2, 1, [100, 130], seed=21)
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg, pool_fill=float("nan"))
+    assert dec.check_status() == 0
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg), "nan tail")
+
+
+def test_decode_theta_1e7():
+    wl = workloads.custom(1, 2, [3000], seed=22)
+    cfg, ocfg = gc.cfgs(1e7)
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    out, _, _ = gc.gpu_step(wl, inp, cfg)
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg), "theta 1e7")
+
+
+def test_decode_is_deterministic_and_split_count_only_changes_rounding():
+    wl = workloads.custom(1, 1, [9000], seed=23)
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    a, dec, st = gc.gpu_step(wl, inp, cfg)
+    q = inp.q.cuda().clone()
+    b = dec.decode(cfg, st, q, xmla.xmla_softmax_scale(cfg)).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)                                   # same split plan: bit-identical
+    ref = gc.oracle_out(wl, inp, ocfg)
+    for s in (1, 2, 7, 70):
+        d = session.Decoder(1, 1, 9000, "cuda", s)
+        gc.assert_close(d.decode(cfg, st, q, xmla.xmla_softmax_scale(cfg)), ref, f"splits={s}")
+
+
+# ------------------------------------------------------------------ device-detected errors
+
+def test_bad_block_id_is_reported_not_faulted():
+    wl = workloads.custom(1, 1, [200], seed=24)
+    cfg, _ = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    _, dec, st = gc.gpu_step(wl, inp, cfg)
+    st.block_table[0, 1] = st.num_blocks + 7          # points outside the pool
+    dec.status.zero_()
+    q = inp.q.cuda().clone()
+    out = dec.decode(cfg, st, q, 0.1)
+    torch.cuda.synchronize()
+    assert dec.check_status() == 5
+    assert torch.isfinite(out.float()).all()
+
+
+def test_sequence_longer_than_max_seqlen_is_reported():
+    wl = workloads.custom(1, 1, [200], seed=25)
+    cfg, _ = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    _, dec, st = gc.gpu_step(wl, inp, cfg)
+    st.seqlens[0] = 10_000                            # > max_seqlen given to the plan (200)
+    dec.status.zero_()
+    dec.decode(cfg, st, inp.q.cuda().clone(), 0.1)
+    torch.cuda.synchronize()
+    assert dec.check_status() == 5
+
+
+def test_bounded_wait_gives_up_and_reports_timeout():
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    xmla.xmla_selftest_wait_timeout(status, 2_000_000)      # 2 ms
+    torch.cuda.synchronize()
+    assert int(status.item()) == 6
+    # the context is still usable
+    assert float(torch.ones(4, device="cuda").sum()) == 4.0
+
+
+def test_host_rejects_small_workspace():
+    wl = workloads.custom(1, 1, [256], seed=26)
+    cfg, _ = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    _, dec, st = gc.gpu_step(wl, inp, cfg)
+    with pytest.raises(xmla.XmlaError) as e:
+        xmla.xmla_decode(cfg, inp.q.cuda(), st.W_UK, st.W_UV, st.pool, st.num_blocks, st.block_table,
+                         st.max_blocks, st.seqlens, 1, 1, 256, 0.1, 0, dec.workspace,
+                         dec.ws_bytes - 1024, dec.status, dec.out)
+    assert e.value.status == 3
+
+
+# ------------------------------------------------------------------ the five seeded workloads
+
+def test_workload_decode_4k():
+    wl = workloads.workload("decode_4k")
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg)
+    assert dec.check_status() == 0
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, form="expanded"), "decode_4k", plain_max_abs=True)
+
+
+def test_workload_decode_256k():
+    wl = workloads.workload("decode_256k")
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cuda")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg)
+    assert dec.check_status() == 0
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, form="expanded"), "decode_256k", plain_max_abs=True)
+
+
+def test_workload_verify_q4_b8():
+    wl = workloads.workload("verify_q4_b8")
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cuda")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg)
+    assert dec.check_status() == 0
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, seqs=[0, 3, 7], form="absorbed"), "verify_q4_b8", plain_max_abs=True)
+
+
+def test_workload_decode_512k_b4():
+    wl = workloads.workload("decode_512k_b4")
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cuda")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg)
+    assert dec.check_status() == 0
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, seqs=[0, 3], form="absorbed"), "decode_512k_b4", plain_max_abs=True)
+
+
+@pytest.mark.parametrize("layer", [0, 39])
+def test_workload_step_40l_b32_sampled_layers(layer):
+    wl = workloads.workload("step_40l_b32")
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, layer, "cuda")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg)
+    assert dec.check_status() == 0
+    seqs = [int(np.argmax(wl.seqlens)), int(np.argmin(wl.seqlens)), 5, 17]
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, seqs=seqs, form="absorbed"),
+                    f"step_40l_b32 layer {layer}", plain_max_abs=True)
