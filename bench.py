@@ -10,8 +10,9 @@ attention, LSE combine with W_UV).  The default workload is a single 256K
 context (batch 1, q_len 1, 64-token pages in a shuffled order).
 
 Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
-events on the launching stream; the L2 is flushed (256 MiB write) before every
-step, outside the events.  The K steps are bracketed by a barrier and a device
+events on the launching stream; the L2 is flushed before every step, outside
+the events (a 256 MiB write, then a 256 MiB read so that no dirty lines are
+left for the timed step to write back).  The K steps are bracketed by a barrier and a device
 synchronise; the reported time is the max over ranks.  Under torchrun every
 rank runs its own replica of the workload (independent sequences, no
 collective on the data path): weak scaling.
@@ -26,7 +27,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -78,7 +78,7 @@ def workload_config(wl, world):
         "heads": 32,
         "cache_row": "[c_kv 512 | k_pe 64] bf16",
         "paging": "64-token blocks, contiguous" if wl.contiguous else "64-token blocks, shuffled",
-        "l2": "flushed before every timed step (256 MiB write)",
+        "l2": "flushed before every timed step (256 MiB write, then 256 MiB read so no dirty lines remain)",
         "parallelism": f"dp{world} (independent replicas)",
     }
 
@@ -86,53 +86,62 @@ def workload_config(wl, world):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Polls SM clock and clock-event (throttle) reasons through NVML every
+    millisecond from a background thread while the timed region runs."""
+
+    REASONS = {  # NVML clocks-event reason bits
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x4: "sw_power_cap",
+    }
 
     def __init__(self, gpu_index: int):
-        self.proc = None
         self.gpu = gpu_index
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.samples = []
+        self.reasons = set()
+        self.thread = None
+        self.max_mhz = None
 
     def start(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.gpu]) if vis and vis.split(",")[0].isdigit() else self.gpu
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nvml = pynvml
         except Exception:
-            self.proc = None
+            self.nvml = None
+            return
+        self.stop_flag = False
+
+        def loop():
+            get_r = getattr(self.nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(self.nvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            while not self.stop_flag:
+                try:
+                    self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                    r = get_r(self.h)
+                    for bit, name in self.REASONS.items():
+                        if r & bit:
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+                time.sleep(0.001)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx = float(parts[2])
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower().startswith("active"):
-                        reasons.add(n)
-        if not sm:
+        self.stop_flag = True
+        self.thread.join(timeout=2)
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm),
-                "reasons": sorted(reasons)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": sorted(self.reasons), "source": "nvml"}
 
 
 # ------------------------------------------------------------------ CPU oracle sample
@@ -278,10 +287,18 @@ def run_xmla(args, wl):
     if dec.check_status() != 0:
         raise RuntimeError(f"device status {dec.check_status()} after warm-up")
 
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def flush_l2(i):
+        # evict everything (write), then replace the now-dirty lines with clean
+        # ones (read) so the timed step does not pay for their write-back
+        flush_w.fill_(i & 0xFF)
+        flush_r.sum()
+
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         graph.replay()
     torch.cuda.synchronize()
 
@@ -294,7 +311,7 @@ def run_xmla(args, wl):
     e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     step_ms, attn_ms = [], []
     for i in range(args.steps):
-        flush.fill_((i + 1) & 0xFF)
+        flush_l2(i + 1)
         e0[i].record(stream)
         graph.replay()
         e1[i].record(stream)
@@ -322,7 +339,7 @@ def run_xmla(args, wl):
     ee1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     e2e_ms = []
     for i in range(args.steps):
-        flush.fill_((i + 7) & 0xFF)
+        flush_l2(i + 7)
         ee0[i].record(stream)
         for L, h in zip(layers, h_in):
             for k, v in h.items():

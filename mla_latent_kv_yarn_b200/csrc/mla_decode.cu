@@ -10,15 +10,20 @@
 //      cache, not the weights, is what long contexts pay for; reading it is the
 //      whole cost of a decode step.
 //
-// Three kernels per call:
+// Three kernels per call, chained with programmatic dependent launch:
 //   q_absorb   q_ext[b,j,h] = c * [W_UK[h]^T q_nope | rope(q_pe)]   (c = scale * log2 e)
 //   decode     one CTA per (sequence, row group, KV split): 64-token pages are
-//              streamed by TMA into shared memory; S^T = page . q_ext^T (M = 64
-//              tokens, N = rows, K = 576) and O^T += c_kv^T . P^T (M = 128 latent
-//              dims x 4, N = rows, K = 64 tokens) run on tcgen05 with fp32
-//              accumulators in tensor memory; the online softmax (base 2, lazy
-//              max update) runs in registers.  Writes per-split (m, l, O).
-//   combine    merges the splits by their log-sum-exp and applies W_UV[h].
+//              streamed by TMA into a shared-memory ring; S^T = page . q_ext^T
+//              (M = 64 tokens, N = rows, K = 576) and O^T += c_kv^T . P^T (M = 128
+//              latent dims x 4, N = rows, K = 64 tokens) run on tcgen05 with fp32
+//              accumulators in tensor memory; S is double-buffered so the QK of
+//              page i+1 runs while the softmax of page i does; the online softmax
+//              (base 2, lazy max update) runs in registers.  Writes per-split
+//              (m, l, O).
+//   combine    a cluster of 8 CTAs per (head, row chunk) merges the splits by their
+//              log-sum-exp over 64-dim slices of the latent and applies W_UV; the
+//              slices' partial outputs are summed through distributed shared memory.
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -29,6 +34,8 @@
 #include "xmla_device.cuh"
 #include "yarn.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace xmla {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -37,7 +44,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazyMax = 8.0f;
 constexpr int kMaxSplits = 1024;
 constexpr int kSoftmaxThreads = 128;
-constexpr int kDecodeThreads = 64 + kSoftmaxThreads;
+constexpr int kSoftmaxWarp0 = 3;  // warps: 0 TMA producer, 1 QK issuer, 2 PV issuer, 3-6 softmax
+constexpr int kDecodeThreads = 32 * kSoftmaxWarp0 + kSoftmaxThreads;
 
 // ---------------------------------------------------------------- shared-memory plan
 
@@ -47,7 +55,12 @@ struct DecodeLayout {
   static constexpr int kLatSlots = NR == 32 ? 9 : 7;   // 16 KB: latent dims 128m..128m+127 of a page
   static constexpr int kRopeSlots = NR == 32 ? 4 : 2;  // 8 KB: rope dims of a page
   static constexpr uint32_t kQChunk = NR * 128;        // one 64-column chunk of q_ext
-  static constexpr uint32_t kPBytes = NR * 128;        // P^T: NR rows x 64 tokens bf16
+  // P^T is stored MN-major: one row of NR bf16 per token, 64 B (64-byte swizzle)
+  // for 32 rows or 128 B (128-byte swizzle) for 64 rows.
+  static constexpr uint32_t kPRow = NR * 2;
+  static constexpr uint32_t kPBytes = 64 * kPRow;
+  static constexpr uint32_t kPSwizzle = NR == 32 ? kSwizzle64B : kSwizzle128B;
+  static constexpr uint32_t kPGroup = 8 * kPRow;       // 8 tokens: one swizzle atom
   static constexpr uint32_t kLatBytes = 16384;
   static constexpr uint32_t kRopeBytes = 8192;
   static constexpr uint32_t kOffQ = 0;
@@ -61,12 +74,12 @@ struct DecodeLayout {
   static constexpr int kBarLatEmpty = kBarLatFull + kLatSlots;
   static constexpr int kBarRopeFull = kBarLatEmpty + kLatSlots;
   static constexpr int kBarRopeEmpty = kBarRopeFull + kRopeSlots;
-  static constexpr int kBarSFull = kBarRopeEmpty + kRopeSlots;
-  static constexpr int kBarSFree = kBarSFull + 1;
-  static constexpr int kBarPFull = kBarSFree + 1;   // 2
-  static constexpr int kBarPvDone = kBarPFull + 2;  // 2
-  static constexpr int kBarDrain = kBarPvDone + 2;
-  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kBarSFull = kBarRopeEmpty + kRopeSlots;  // 2
+  static constexpr int kBarSFree = kBarSFull + 2;               // 2
+  static constexpr int kBarPFull = kBarSFree + 2;               // 2
+  static constexpr int kBarPvDone = kBarPFull + 2;              // 2
+  static constexpr int kBarDrain = kBarPvDone + 2;  // 2: QK issuer, PV issuer
+  static constexpr int kNumBars = kBarDrain + 2;
   static constexpr uint32_t kOffMUsed = (kOffBars + kNumBars * 8 + 15) & ~15u;
   static constexpr uint32_t kOffMNext = kOffMUsed + NR * 4;
   static constexpr uint32_t kOffAlpha = kOffMNext + NR * 4;
@@ -76,10 +89,11 @@ struct DecodeLayout {
   static constexpr uint32_t kBytes = kOffAbort + 12;
   static constexpr uint32_t kSmem = kBytes + 1024;  // slack for 1024-byte alignment
   static_assert(kSmem <= 232448, "shared memory per CTA");
-  // tensor memory columns: O^T at [0, 4 NR), S^T at [4 NR, 5 NR)
+  static_assert(kOffP % 1024 == 0 && kOffLat % 1024 == 0 && kOffRope % 1024 == 0, "alignment");
+  // tensor memory columns: O^T at [0, 4 NR), S^T buffers at [4 NR, 5 NR) and [5 NR, 6 NR)
   static constexpr uint32_t kColO = 0;
   static constexpr uint32_t kColS = 4 * NR;
-  static constexpr uint32_t kTmemCols = 5 * NR <= 256 ? 256 : 512;
+  static constexpr uint32_t kTmemCols = 6 * NR <= 256 ? 256 : 512;
 };
 
 struct DecodeParams {
@@ -113,6 +127,11 @@ __device__ __forceinline__ void xpose_reduce32(float (&v)[32], int lane) {
       v[k] = kMax ? fmaxf(keep, recv) : keep + recv;
     }
   }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 template <int NR>
@@ -156,7 +175,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int64_t p_end = min(npages, p_begin + pps);
   const int n_pages = (int)max((int64_t)0, p_end - p_begin);
 
-  // ---- setup
+  // ---- setup (independent of the previous kernel's results)
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kBarQ), 1);
     for (int i = 0; i < L::kLatSlots; ++i) {
@@ -167,13 +186,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       mbar_init(bar(L::kBarRopeFull + i), 1);
       mbar_init(bar(L::kBarRopeEmpty + i), 1);
     }
-    mbar_init(bar(L::kBarSFull), 1);
-    mbar_init(bar(L::kBarSFree), kSoftmaxThreads);
-    mbar_init(bar(L::kBarPFull + 0), kSoftmaxThreads);
-    mbar_init(bar(L::kBarPFull + 1), kSoftmaxThreads);
-    mbar_init(bar(L::kBarPvDone + 0), 1);
-    mbar_init(bar(L::kBarPvDone + 1), 1);
-    mbar_init(bar(L::kBarDrain), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::kBarSFull + i), 1);
+      mbar_init(bar(L::kBarSFree + i), kSoftmaxThreads);
+      mbar_init(bar(L::kBarPFull + i), kSoftmaxThreads);
+      mbar_init(bar(L::kBarPvDone + i), 1);
+    }
+    mbar_init(bar(L::kBarDrain + 0), 1);
+    mbar_init(bar(L::kBarDrain + 1), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -181,12 +201,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     tmem_alloc(base + L::kOffTmem, L::kTmemCols);
     tmem_relinquish();
   }
-  if (threadIdx.x >= 64 && threadIdx.x < 64 + NR) m_used[threadIdx.x - 64] = -INFINITY;
+  if (threadIdx.x >= 32 * kSoftmaxWarp0 && threadIdx.x < 32 * kSoftmaxWarp0 + NR)
+    m_used[threadIdx.x - 32 * kSoftmaxWarp0] = -INFINITY;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + L::kOffTmem);
   const int32_t qrow0 = (int32_t)(((int64_t)b * p.q_len + j0) * 32);
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ================================================================ TMA producer
@@ -194,15 +216,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       tma_prefetch_desc(&tmap_pool);
       tma_prefetch_desc(&tmap_q);
       const uint64_t stream_policy = policy_evict_first();
-      mbar_arrive_expect_tx(bar(L::kBarQ), 9u * L::kQChunk);
-      for (int c = 0; c < 9; ++c)
-        tma_load_2d(base + L::kOffQ + c * L::kQChunk, &tmap_q, c * 64, qrow0, bar(L::kBarQ));
       int li = 0, ri = 0;
       uint32_t lph = 0, rph = 0;
       int64_t lat_issued = 0, rope_issued = 0;
-      bool ok = true;
+      bool ok = true, q_issued = false;
+      // block ids are fetched four pages ahead so their load latency is hidden
+      const int32_t* bt = p.block_table + (int64_t)b * p.max_blocks + p_begin;
+      int32_t nb0 = bt[0];
+      int32_t nb1 = n_pages > 1 ? bt[1] : 0;
+      int32_t nb2 = n_pages > 2 ? bt[2] : 0;
+      int32_t nb3 = n_pages > 3 ? bt[3] : 0;
       for (int i = 0; i < n_pages && ok; ++i) {
-        int32_t blk = p.block_table[(int64_t)b * p.max_blocks + p_begin + i];
+        int32_t blk = nb0;
+        nb0 = nb1;
+        nb1 = nb2;
+        nb2 = nb3;
+        nb3 = i + 4 < n_pages ? bt[i + 4] : 0;
         if (blk < 0 || (int64_t)blk >= p.num_blocks) {
           record_status(p.status, XMLA_ERR_DEVICE_OOB);
           blk = (int32_t)p.num_blocks;  // past the end: the tensor copy reads zeros
@@ -233,10 +262,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                          bar(L::kBarRopeFull + ri), stream_policy);
         ++rope_issued;
         if (++ri == L::kRopeSlots) { ri = 0; rph ^= 1u; }
+        if (!q_issued) {
+          // q_ext is the previous kernel's output: wait for it only after the
+          // first page is on its way.
+          pdl_wait();
+          mbar_arrive_expect_tx(bar(L::kBarQ), 9u * L::kQChunk);
+          for (int c = 0; c < 9; ++c)
+            tma_load_2d(base + L::kOffQ + c * L::kQChunk, &tmap_q, c * 64, qrow0, bar(L::kBarQ));
+          q_issued = true;
+        }
       }
       // Every copy issued must land before the CTA may exit: wait for the last
       // phase armed on each slot (immediate when the consumer already saw it).
-      mbar_wait(bar(L::kBarQ), 0, nullptr, p.status, p.wait_limit_ns);
+      if (q_issued) mbar_wait(bar(L::kBarQ), 0, nullptr, p.status, p.wait_limit_ns);
       for (int s = 0; s < L::kLatSlots; ++s) {
         if (lat_issued > s) {
           const int64_t last = s + ((lat_issued - 1 - s) / L::kLatSlots) * L::kLatSlots;
@@ -252,113 +290,123 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ================================================================ tensor-core issuers
+    // Warp 1 issues QK (S^T[64 tok, NR] = page . q_ext^T into S buffer i & 1),
+    // running up to two pages ahead of the softmax; warp 2 issues PV
+    // (O^T[512, NR] += c_kv^T . P^T) as soon as a page's P is written.  Each
+    // blocks in mbarrier try_wait, which suspends the thread instead of
+    // spinning, so neither steals issue slots from the softmax warps.
     if (lane == 0 && n_pages > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(64, NR, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, NR, true, false);
-      const uint32_t t_s = tmem_base + L::kColS;
-      const uint32_t t_o = tmem_base + L::kColO;
-      bool ok = mbar_wait(bar(L::kBarQ), 0, abort_flag, p.status, p.wait_limit_ns);
-      tc_fence_after();
-      int li = 0, ri = 0;
-      uint32_t lph = 0, rph = 0;
-      for (int i = 0; i < n_pages && ok; ++i) {
-        if (i > 0) {
-          ok = mbar_wait(bar(L::kBarSFree), (uint32_t)((i - 1) & 1), abort_flag, p.status,
-                         p.wait_limit_ns);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        // S^T[64 tok, NR] = page[64, 576] . q_ext[NR, 576]^T
-        for (int m = 0; m < 4 && ok; ++m) {
-          int s = li + m;
-          uint32_t ph = lph;
-          if (s >= L::kLatSlots) { s -= L::kLatSlots; ph ^= 1u; }
-          ok = mbar_wait(bar(L::kBarLatFull + s), ph, abort_flag, p.status, p.wait_limit_ns);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t slot = base + L::kOffLat + s * L::kLatBytes;
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, NR, true, true);
+      // descriptor bases; operands are reached by adding (byte offset >> 4)
+      const uint64_t d_lat_k = smem_desc_sw128(base + L::kOffLat, 16, 1024);     // page, K-major
+      const uint64_t d_rope_k = smem_desc_sw128(base + L::kOffRope, 16, 1024);
+      const uint64_t d_q = smem_desc_sw128(base + L::kOffQ, 16, 1024);           // q_ext, K-major
+      const uint64_t d_lat_mn = smem_desc_sw128(base + L::kOffLat, 8192, 1024);  // c_kv^T, MN-major
+      const uint64_t d_p = smem_desc(base + L::kOffP, 8192, L::kPGroup, L::kPSwizzle);  // P^T, MN-major
+      auto wait = [&](int idx, uint32_t parity) {
+        return mbar_wait(bar(idx), parity, abort_flag, p.status, p.wait_limit_ns);
+      };
+      bool ok = true;
+      if (warp == 1) {
+        ok = wait(L::kBarQ, 0);
+        tc_fence_after();
+        for (int i = 0; i < n_pages && ok; ++i) {
+          const int sb = i & 1;
+          if (i >= 2) {
+            if (!(ok = wait(L::kBarSFree + sb, (uint32_t)(((i - 2) >> 1) & 1)))) break;
+            tc_fence_after();
+          }
+          const uint32_t t_s = tmem_base + L::kColS + sb * NR;
+          for (int m = 0; m < 4 && ok; ++m) {
+            const int f = 4 * i + m;
+            const int s = f % L::kLatSlots;
+            if (!(ok = wait(L::kBarLatFull + s, (uint32_t)((f / L::kLatSlots) & 1)))) break;
+            tc_fence_after();
+            const uint64_t a0 = d_lat_k + ((s * L::kLatBytes) >> 4);
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int c = 2 * m + half;
+            for (int half = 0; half < 2; ++half) {
+              const uint64_t bq = d_q + (((2 * m + half) * L::kQChunk) >> 4);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t a = smem_desc_sw128(slot + half * 8192 + k * 32, 16, 1024);
-              const uint64_t bq = smem_desc_sw128(base + L::kOffQ + c * L::kQChunk + k * 32, 16, 1024);
-              tc_mma_bf16(t_s, a, bq, idesc_qk, (c | k) != 0 ? 1u : 0u);
+              for (int k = 0; k < 4; ++k)
+                tc_mma_bf16(t_s, a0 + ((half * 8192 + k * 32) >> 4), bq + ((k * 32) >> 4), idesc_qk,
+                            (m | half | k) != 0 ? 1u : 0u);
             }
           }
-        }
-        if (!ok) break;
-        ok = mbar_wait(bar(L::kBarRopeFull + ri), rph, abort_flag, p.status, p.wait_limit_ns);
-        if (!ok) break;
-        tc_fence_after();
-        {
-          const uint32_t slot = base + L::kOffRope + ri * L::kRopeBytes;
+          if (!ok) break;
+          const int r = i % L::kRopeSlots;
+          if (!(ok = wait(L::kBarRopeFull + r, (uint32_t)((i / L::kRopeSlots) & 1)))) break;
+          tc_fence_after();
+          const uint64_t ar = d_rope_k + ((r * L::kRopeBytes) >> 4);
+          const uint64_t bq = d_q + ((8 * L::kQChunk) >> 4);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t a = smem_desc_sw128(slot + k * 32, 16, 1024);
-            const uint64_t bq = smem_desc_sw128(base + L::kOffQ + 8 * L::kQChunk + k * 32, 16, 1024);
-            tc_mma_bf16(t_s, a, bq, idesc_qk, 1u);
-          }
+          for (int k = 0; k < 4; ++k)
+            tc_mma_bf16(t_s, ar + ((k * 32) >> 4), bq + ((k * 32) >> 4), idesc_qk, 1u);
+          tc_commit(bar(L::kBarSFull + sb));
+          tc_commit(bar(L::kBarRopeEmpty + r));
         }
-        tc_commit(bar(L::kBarSFull));
-        tc_commit(bar(L::kBarRopeEmpty + ri));
-        if (++ri == L::kRopeSlots) { ri = 0; rph ^= 1u; }
-
-        // O^T[512, NR] += c_kv^T[512, 64 tok] . P^T[64 tok, NR]
-        ok = mbar_wait(bar(L::kBarPFull + (i & 1)), (uint32_t)((i >> 1) & 1), abort_flag, p.status,
-                       p.wait_limit_ns);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t pbuf = base + L::kOffP + (i & 1) * L::kPBytes;
-        for (int m = 0; m < 4; ++m) {
-          int s = li + m;
-          if (s >= L::kLatSlots) s -= L::kLatSlots;
-          const uint32_t slot = base + L::kOffLat + s * L::kLatBytes;
+      } else {
+        for (int i = 0; i < n_pages && ok; ++i) {
+          if (!(ok = wait(L::kBarPFull + (i & 1), (uint32_t)((i >> 1) & 1)))) break;
+          tc_fence_after();
+          const uint64_t bp = d_p + (((i & 1) * L::kPBytes) >> 4);
+#pragma unroll 1
+          for (int m = 0; m < 4; ++m) {
+            const int s = (4 * i + m) % L::kLatSlots;
+            const uint64_t a0 = d_lat_mn + ((s * L::kLatBytes) >> 4);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t a = smem_desc_sw128(slot + k * 2048, 8192, 1024);
-            const uint64_t bp = smem_desc_sw128(pbuf + k * 32, 16, 1024);
-            tc_mma_bf16(t_o + m * NR, a, bp, idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < 4; ++k)
+              tc_mma_bf16(tmem_base + L::kColO + m * NR, a0 + ((k * 2048) >> 4),
+                          bp + ((k * 2 * L::kPGroup) >> 4), idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
+            tc_commit(bar(L::kBarLatEmpty + s));
           }
-          tc_commit(bar(L::kBarLatEmpty + s));
+          tc_commit(bar(L::kBarPvDone + (i & 1)));
         }
-        tc_commit(bar(L::kBarPvDone + (i & 1)));
-        li += 4;
-        if (li >= L::kLatSlots) { li -= L::kLatSlots; lph ^= 1u; }
       }
-      // all issued tensor-core work must finish before tensor memory is freed
-      tc_commit(bar(L::kBarDrain));
-      mbar_wait(bar(L::kBarDrain), 0, nullptr, p.status, p.wait_limit_ns);
+      // all tensor-core work this thread issued must finish before tensor memory is freed
+      const int drain = L::kBarDrain + (warp - 1);
+      tc_commit(bar(drain));
+      mbar_wait(bar(drain), 0, nullptr, p.status, p.wait_limit_ns);
     }
   } else {
     // ================================================================ softmax / epilogue
-    const int tid = threadIdx.x - 64;
+    const int tid = threadIdx.x - 32 * kSoftmaxWarp0;
     const int quarter = warp & 3;            // tensor-memory lane quarter this warp may access
     const int tok = 16 * quarter + lane;     // token of the page held by this thread (lane < 16)
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quarter) << 16);
     float l_part[NR];
 #pragma unroll
     for (int n = 0; n < NR; ++n) l_part[n] = 0.f;
+    // running maxima: a register copy for 32 rows, shared memory for 64
+    constexpr bool kRegM = NR == 32;
+    float mr[kRegM ? NR : 1];
+#pragma unroll
+    for (int n = 0; n < (kRegM ? NR : 1); ++n) mr[n] = -INFINITY;
+    auto mu = [&](int n) -> float {
+      if constexpr (kRegM) return mr[n];
+      else return m_used[n];
+    };
     const int64_t qpos0 = seqlen - p.q_len + j0;  // position of this CTA's first query
     bool ok = true;
     for (int i = 0; i < n_pages; ++i) {
-      ok = mbar_wait(bar(L::kBarSFull), (uint32_t)(i & 1), abort_flag, p.status, p.wait_limit_ns);
+      const int sb = i & 1;
+      ok = mbar_wait(bar(L::kBarSFull + sb), (uint32_t)((i >> 1) & 1), abort_flag, p.status,
+                     p.wait_limit_ns);
       if (named_bar_or(1, kSoftmaxThreads, !ok)) { ok = false; break; }
       tc_fence_after();
       float sv[NR];
 #pragma unroll
       for (int c = 0; c < NR / 32; ++c) {
         float tmp[32];
-        tmem_ld32(t_lane + L::kColS + 32 * c, tmp);
+        tmem_ld32(t_lane + L::kColS + sb * NR + 32 * c, tmp);
 #pragma unroll
         for (int k = 0; k < 32; ++k) sv[32 * c + k] = tmp[k];
       }
       tc_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(L::kBarSFree));
+      mbar_arrive(bar(L::kBarSFree + sb));
 
       const int64_t tpos = (p_begin + i) * kPage + tok;
       bool exceed = false;
@@ -366,7 +414,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       for (int n = 0; n < NR; ++n) {
         const bool vis = lane < 16 && (n >> 5) < jn && tpos <= qpos0 + (n >> 5);
         sv[n] = vis ? sv[n] : -INFINITY;
-        exceed |= sv[n] > m_used[n] + kLazyMax;
+        exceed |= sv[n] > mu(n) + kLazyMax;
       }
       if (named_bar_or(1, kSoftmaxThreads, exceed)) {
 #pragma unroll
@@ -413,6 +461,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         for (int n = 0; n < NR; ++n) l_part[n] *= alpha_s[n];
         if (tid < NR) m_used[tid] = m_next[tid];
         named_bar_sync(1, kSoftmaxThreads);
+        if constexpr (kRegM) {
+#pragma unroll
+          for (int n = 0; n < NR; ++n) mr[n] = m_used[n];
+        }
       }
       if (i >= 2) {
         // P buffer (i & 1) is free once the PV of page i - 2 has completed
@@ -435,17 +487,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           dst[u] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      uint8_t* pbuf = smem + L::kOffP + (i & 1) * L::kPBytes;
+      // P^T row of this token: NR bf16, written as 16-byte units in the swizzled
+      // MN-major layout the PV descriptor reads.
+      uint8_t* prow = smem + L::kOffP + sb * L::kPBytes + tok * L::kPRow;
 #pragma unroll
-      for (int n = 0; n < NR; ++n) {
-        const float pr = sv[n] == -INFINITY ? 0.f : ex2(sv[n] - m_used[n]);
-        const __nv_bfloat16 hb = __float2bfloat16_rn(pr);
-        l_part[n] += __bfloat162float(hb);
-        if (lane < 16) *reinterpret_cast<__nv_bfloat16*>(pbuf + sw128_offset(n, tok)) = hb;
+      for (int u = 0; u < NR / 8; ++u) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int n0 = 8 * u + 2 * e;
+          const float p0 = sv[n0] == -INFINITY ? 0.f : ex2(sv[n0] - mu(n0));
+          const float p1 = sv[n0 + 1] == -INFINITY ? 0.f : ex2(sv[n0 + 1] - mu(n0 + 1));
+          w[e] = pack_bf16x2(p0, p1);
+          const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
+          l_part[n0] += __low2float(hb);
+          l_part[n0 + 1] += __high2float(hb);
+        }
+        const int phys = NR == 32 ? (u ^ ((tok >> 1) & 3)) : (u ^ (tok & 7));
+        if (lane < 16)
+          *reinterpret_cast<uint4*>(prow + phys * 16) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(L::kBarPFull + (i & 1)));
+      mbar_arrive(bar(L::kBarPFull + sb));
     }
 
     // ---- epilogue: unnormalised O, running max m and sum l of this split
@@ -507,9 +571,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
 // q_ext[r, h] = qscale * [W_UK[h]^T q_nope[r, h] | rope(q_pe[r, h], pos_r)], r = b*q_len + j,
 // with pos_r = seqlens[b] - q_len + j (the q_len new tokens are the last cache
-// entries).  grid (32 heads, 4 column blocks of 128); block 128 threads, one
-// latent column each; the column-block-0 CTAs also rotate the rope part.
-constexpr int kAbsorbRows = 32;
+// entries).  grid (32 heads, 8 blocks of 64 latent columns); 128 threads:
+// thread t owns 8 columns (t % 8) and 8 of the 128 nope dims (t / 8), holding
+// its 8 x 8 slice of W_UK in registers; partial sums meet in shared memory.
+// The column-block-0 CTAs also rotate the rope part.
+constexpr int kAbsorbRows = 8;
 
 __global__ void __launch_bounds__(128) q_absorb_kernel(const __nv_bfloat16* __restrict__ q,
                                                        const __nv_bfloat16* __restrict__ W_UK,
@@ -518,30 +584,56 @@ __global__ void __launch_bounds__(128) q_absorb_kernel(const __nv_bfloat16* __re
                                                        int q_len, float qscale,
                                                        const RopeTable tab) {
   __shared__ float sq[kAbsorbRows][kDNope];
+  __shared__ float part[16][kAbsorbRows][64];
+  pdl_launch_dependents();
   const int h = blockIdx.x;
-  const int col = blockIdx.y * 128 + threadIdx.x;
-  float w[kDNope];
+  const int cb = blockIdx.y;
+  const int t = threadIdx.x;
+  const int c8 = t & 7;
+  const int dg = t >> 3;
+  float w[8][8];
 #pragma unroll
-  for (int d = 0; d < kDNope; ++d)
-    w[d] = __bfloat162float(W_UK[((int64_t)h * kDNope + d) * kDLatent + col]);
+  for (int dd = 0; dd < 8; ++dd) {
+    const uint4 v = *reinterpret_cast<const uint4*>(
+        W_UK + ((int64_t)h * kDNope + dg * 8 + dd) * kDLatent + cb * 64 + c8 * 8);
+    const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      w[dd][2 * e] = __low2float(pv[e]);
+      w[dd][2 * e + 1] = __high2float(pv[e]);
+    }
+  }
   for (int r0 = 0; r0 < rows; r0 += kAbsorbRows) {
     const int nr = min(kAbsorbRows, rows - r0);
     __syncthreads();
-    for (int e = threadIdx.x; e < nr * kDNope; e += blockDim.x) {
+    for (int e = t; e < nr * kDNope; e += blockDim.x) {
       const int r = e / kDNope, d = e % kDNope;
       sq[r][d] = __bfloat162float(q[((int64_t)(r0 + r) * kHeads + h) * kDQ + d]);
     }
     __syncthreads();
     for (int r = 0; r < nr; ++r) {
-      float acc = 0.f;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int d = 0; d < kDNope; ++d) acc = fmaf(sq[r][d], w[d], acc);
-      q_ext[((int64_t)(r0 + r) * kHeads + h) * kDRow + col] = __float2bfloat16_rn(acc * qscale);
+      for (int dd = 0; dd < 8; ++dd) {
+        const float x = sq[r][dg * 8 + dd];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = fmaf(x, w[dd][k], acc[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) part[dg][r][c8 * 8 + k] = acc[k];
+    }
+    __syncthreads();
+    for (int o = t; o < nr * 64; o += blockDim.x) {
+      const int r = o / 64, col = o % 64;
+      float s = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) s += part[k][r][col];
+      q_ext[((int64_t)(r0 + r) * kHeads + h) * kDRow + cb * 64 + col] = __float2bfloat16_rn(s * qscale);
     }
   }
-  if (blockIdx.y == 0) {
+  if (cb == 0) {
     constexpr int kPairs = kDRope / 2;
-    for (int e = threadIdx.x; e < rows * kPairs; e += blockDim.x) {
+    for (int e = t; e < rows * kPairs; e += blockDim.x) {
       const int r = e / kPairs, i = e % kPairs;
       const int64_t pos = (int64_t)seqlens[r / q_len] - q_len + (r % q_len);
       const __nv_bfloat16* x = q + ((int64_t)r * kHeads + h) * kDQ + kDNope;
@@ -557,77 +649,127 @@ __global__ void __launch_bounds__(128) q_absorb_kernel(const __nv_bfloat16* __re
 
 // ---------------------------------------------------------------- combine + W_UV
 
-// One CTA (128 threads) per output row (b, j, h): merge the splits' partial
-// latent outputs by their log-sum-exp, then out = o_lat . W_UV[h].
-__global__ void __launch_bounds__(128) combine_uv_kernel(const float* __restrict__ part_o,
-                                                         const float* __restrict__ part_ml,
-                                                         const __nv_bfloat16* __restrict__ W_UV,
-                                                         __nv_bfloat16* __restrict__ out, int q_len,
-                                                         int groups, int nsplit, int rows_per_cta) {
-  __shared__ float w_s[kMaxSplits];
-  __shared__ float o_lat[kDLatent];
-  __shared__ float red_s[4];
-  const int row = blockIdx.x;  // (b*q_len + j)*32 + h
-  const int h = row % kHeads;
-  const int bj = row / kHeads;
-  const int j = bj % q_len;
-  const int b = bj / q_len;
-  const int r = j * kHeads + h;
-  const int g = r / rows_per_cta;
-  const int n = r % rows_per_cta;
-  const int64_t item0 = ((int64_t)b * groups + g) * nsplit;
+// Cluster of 8 CTAs per (head h, chunk of up to kCombineRows output rows).
+// CTA `slice` owns latent dims [64 slice, 64 slice + 64): for every row it
+// merges the splits' partial O by their log-sum-exp weights, normalises, and
+// multiplies by the matching 64 rows of W_UV[h]; the 8 partial outputs of a
+// row are summed through distributed shared memory by the cluster's CTA 0.
+constexpr int kSlices = 8;
+constexpr int kSliceDims = kDLatent / kSlices;  // 64
+constexpr int kCombineRows = 16;
+
+__global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(128)
+    combine_uv_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                      const __nv_bfloat16* __restrict__ W_UV, __nv_bfloat16* __restrict__ out,
+                      int rows, int q_len, int groups, int nsplit, int rows_per_cta) {
+  __shared__ __align__(16) __nv_bfloat16 w_s[kSliceDims][kDV];  // this slice's rows of W_UV[h]
+  __shared__ float wt_s[kMaxSplits];                             // split weights of one row
+  __shared__ __align__(16) float4 acc_s[8][kSliceDims / 4];
+  __shared__ float o_s[kCombineRows][kSliceDims];
+  __shared__ float out_s[kCombineRows][kDV];
+  __shared__ float red_s[8];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int slice = (int)cluster.block_rank();
+  const int cid = blockIdx.x / kSlices;
+  const int h = cid % kHeads;
+  const int chunk = cid / kHeads;
+  const int r0 = chunk * kCombineRows;
+  const int nr = min(kCombineRows, rows - r0);
   const int tid = threadIdx.x;
-
-  // global max over splits that saw any token
-  float mx = -INFINITY;
-  for (int s = tid; s < nsplit; s += blockDim.x) {
-    const float m = part_ml[((item0 + s) * rows_per_cta + n) * 2 + 0];
-    const float l = part_ml[((item0 + s) * rows_per_cta + n) * 2 + 1];
-    if (l > 0.f) mx = fmaxf(mx, m);
+  pdl_launch_dependents();
+  // W_UV does not depend on the decode kernel: stage it while that kernel finishes
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(W_UV + ((int64_t)h * kDLatent + slice * kSliceDims) * kDV);
+    uint4* dst = reinterpret_cast<uint4*>(&w_s[0][0]);
+#pragma unroll
+    for (int e = 0; e < kSliceDims * kDV / 8 / 128; ++e) dst[tid + 128 * e] = src[tid + 128 * e];
   }
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if ((tid & 31) == 0) red_s[tid >> 5] = mx;
-  __syncthreads();
-  mx = fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3]));
-  __syncthreads();
-  float lsum = 0.f;
-  for (int s = tid; s < nsplit; s += blockDim.x) {
-    const float m = part_ml[((item0 + s) * rows_per_cta + n) * 2 + 0];
-    const float l = part_ml[((item0 + s) * rows_per_cta + n) * 2 + 1];
-    const float wgt = l > 0.f ? ex2(m - mx) : 0.f;
-    w_s[s] = wgt;
-    lsum += wgt * l;
-  }
-  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  if ((tid & 31) == 0) red_s[tid >> 5] = lsum;
-  __syncthreads();
-  lsum = red_s[0] + red_s[1] + red_s[2] + red_s[3];
-  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+  pdl_wait();  // the split partials come from the decode kernel
 
-  // o_lat: thread handles 4 consecutive latent dims
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < nsplit; ++s) {
-    const float wgt = w_s[s];
-    if (wgt == 0.f) continue;
-    const float4 v = reinterpret_cast<const float4*>(
-        part_o + ((item0 + s) * rows_per_cta + n) * kDLatent)[tid];
-    acc.x = fmaf(wgt, v.x, acc.x);
-    acc.y = fmaf(wgt, v.y, acc.y);
-    acc.z = fmaf(wgt, v.z, acc.z);
-    acc.w = fmaf(wgt, v.w, acc.w);
+  for (int rr = 0; rr < nr; ++rr) {
+    const int r = r0 + rr;  // r = b*q_len + j
+    const int b = r / q_len, j = r % q_len;
+    const int ridx = j * kHeads + h;
+    const int g = ridx / rows_per_cta;
+    const int n = ridx % rows_per_cta;
+    const int64_t item0 = ((int64_t)b * groups + g) * nsplit;
+    const float2* ml = reinterpret_cast<const float2*>(part_ml) + item0 * rows_per_cta + n;
+    // max over the splits that saw any token
+    float mx = -INFINITY;
+    for (int s = tid; s < nsplit; s += 128) {
+      const float2 v = ml[(int64_t)s * rows_per_cta];
+      if (v.y > 0.f) mx = fmaxf(mx, v.x);
+    }
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((tid & 31) == 0) red_s[tid >> 5] = mx;
+    __syncthreads();
+    mx = fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3]));
+    float lsum = 0.f;
+    for (int s = tid; s < nsplit; s += 128) {
+      const float2 v = ml[(int64_t)s * rows_per_cta];
+      const float wgt = v.y > 0.f ? ex2(v.x - mx) : 0.f;
+      wt_s[s] = wgt;
+      lsum = fmaf(wgt, v.y, lsum);
+    }
+    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    if ((tid & 31) == 0) red_s[4 + (tid >> 5)] = lsum;
+    __syncthreads();
+    const float L = red_s[4] + red_s[5] + red_s[6] + red_s[7];
+    // this slice of the weighted sum: 16 threads x float4 cover the 64 dims of
+    // one split; the 8 thread groups take every 8th split
+    const int q4 = tid & 15;
+    const int grp = tid >> 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float* po = part_o + (item0 * rows_per_cta + n) * kDLatent + slice * kSliceDims + 4 * q4;
+#pragma unroll 4
+    for (int s = grp; s < nsplit; s += 8) {
+      const float wgt = wt_s[s];
+      const float4 v = *reinterpret_cast<const float4*>(po + (int64_t)s * rows_per_cta * kDLatent);
+      if (wgt != 0.f) {
+        acc.x = fmaf(wgt, v.x, acc.x);
+        acc.y = fmaf(wgt, v.y, acc.y);
+        acc.z = fmaf(wgt, v.z, acc.z);
+        acc.w = fmaf(wgt, v.w, acc.w);
+      }
+    }
+    acc_s[grp][q4] = acc;
+    __syncthreads();
+    if (tid < kSliceDims) {
+      const float* a = reinterpret_cast<const float*>(&acc_s[0][0]);
+      float t = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) t += a[k * kSliceDims + tid];
+      o_s[rr][tid] = L > 0.f ? t / L : 0.f;
+    }
+    __syncthreads();
   }
-  o_lat[4 * tid + 0] = acc.x * inv;
-  o_lat[4 * tid + 1] = acc.y * inv;
-  o_lat[4 * tid + 2] = acc.z * inv;
-  o_lat[4 * tid + 3] = acc.w * inv;
-  __syncthreads();
 
-  // out[v] = sum_c o_lat[c] W_UV[h][c][v], thread v
-  const __nv_bfloat16* wv = W_UV + (int64_t)h * kDLatent * kDV + tid;
-  float y = 0.f;
+  // partial out[r][v] = sum over this slice's 64 latent dims of o[r][c] W_UV[h][c][v]
+  {
+    const int v = tid;
+    float acc[kCombineRows];
+#pragma unroll
+    for (int rr = 0; rr < kCombineRows; ++rr) acc[rr] = 0.f;
 #pragma unroll 8
-  for (int c = 0; c < kDLatent; ++c) y = fmaf(o_lat[c], __bfloat162float(wv[(int64_t)c * kDV]), y);
-  out[(int64_t)row * kDV + tid] = __float2bfloat16_rn(y);
+    for (int c = 0; c < kSliceDims; ++c) {
+      const float wcv = __bfloat162float(w_s[c][v]);
+#pragma unroll
+      for (int rr = 0; rr < kCombineRows; ++rr) acc[rr] = fmaf(o_s[rr][c], wcv, acc[rr]);
+    }
+#pragma unroll
+    for (int rr = 0; rr < kCombineRows; ++rr) out_s[rr][v] = acc[rr];
+  }
+  cluster.sync();
+  if (slice == 0) {
+    for (int e = tid; e < nr * kDV; e += blockDim.x) {
+      const int rr = e / kDV, v = e % kDV;
+      float t = 0.f;
+#pragma unroll
+      for (int k = 0; k < kSlices; ++k) t += cluster.map_shared_rank(&out_s[0][0], k)[rr * kDV + v];
+      out[((int64_t)(r0 + rr) * kHeads + h) * kDV + v] = __float2bfloat16_rn(t);
+    }
+  }
+  cluster.sync();  // keep every CTA's shared memory alive until CTA 0 has read it
 }
 
 // ---------------------------------------------------------------- self-test kernel
@@ -726,8 +868,8 @@ static cudaError_t launch_decode(const CUtensorMap& tp, const CUtensorMap& tq, c
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  mla_decode_kernel<NR><<<(unsigned)items, kDecodeThreads, L::kSmem, st>>>(tp, tq, dp);
-  return cudaGetLastError();
+  return launch_pdl(mla_decode_kernel<NR>, dim3((unsigned)items), dim3(kDecodeThreads), L::kSmem,
+                    st, tp, tq, dp);
 }
 
 static bool device_ok(int* num_sms) {
@@ -803,7 +945,10 @@ extern "C" xmla_status xmla_decode_profiled(const xmla_yarn_cfg* cfg, const void
   if (!encode_rows576(&tmap_q, q_ext, (uint64_t)rows * kHeads, (uint32_t)P.nr)) return XMLA_ERR_CUDA;
 
   const float qscale = softmax_scale * kLog2e;
-  q_absorb_kernel<<<dim3(kHeads, kDLatent / 128), 128, 0, st>>>(
+  // q_absorb reads only the caller's inputs; it is an ordinary launch so that it
+  // (and hence the decode kernel chained to it) starts after every earlier
+  // write to the cache on this stream has landed.
+  q_absorb_kernel<<<dim3(kHeads, kDLatent / 64), 128, 0, st>>>(
       (const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext, rows, q_len, qscale,
       make_rope_table(cfg));
   if (cudaGetLastError() != cudaSuccess) return XMLA_ERR_CUDA;
@@ -828,11 +973,11 @@ extern "C" xmla_status xmla_decode_profiled(const xmla_yarn_cfg* cfg, const void
   if (e != cudaSuccess) return XMLA_ERR_CUDA;
   if (record_event(attn_stop, st) != cudaSuccess) return XMLA_ERR_CUDA;
 
-  combine_uv_kernel<<<rows * kHeads, 128, 0, st>>>(dp.part_o, dp.part_ml,
-                                                    (const __nv_bfloat16*)W_UV,
-                                                    (__nv_bfloat16*)out, q_len, P.groups,
-                                                    P.nsplit, P.nr);
-  return cudaGetLastError() == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+  const int chunks = (rows + kCombineRows - 1) / kCombineRows;
+  e = launch_pdl(combine_uv_kernel, dim3(kSlices * kHeads * chunks), dim3(128), 0, st,
+                 (const float*)dp.part_o, (const float*)dp.part_ml, (const __nv_bfloat16*)W_UV,
+                 (__nv_bfloat16*)out, rows, q_len, P.groups, P.nsplit, P.nr);
+  return e == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
 }
 
 extern "C" xmla_status xmla_decode(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -72,6 +73,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking probe: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -251,19 +265,31 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 
 // ---------------------------------------------------------------- UMMA descriptors
 
-// Shared-memory matrix descriptor (sm_100 format, version 1) for a tile stored
-// with the 128-byte swizzle.  Addresses and offsets are in bytes.
-//   K-major operand: rows of 128 B (64 bf16 along K), 8-row groups `sbo` apart.
-//   MN-major operand: 128-B rows are K indices holding 64 consecutive M/N
-//   elements; 8-row K groups `sbo` apart, 64-element M/N groups `lbo` apart.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor (sm_100 format, version 1).  Addresses and
+// offsets are in bytes; `swizzle` is the layout code (2 = 128-byte swizzle,
+// 4 = 64-byte swizzle).
+//   K-major operand, 128-B swizzle: rows of 128 B (64 bf16 along K), 8-row
+//   groups `sbo` apart.
+//   MN-major operand: each row of the swizzle atom (128 B or 64 B) is one K
+//   index holding 64 or 32 consecutive M/N elements; 8-row K groups `sbo`
+//   apart, M/N groups of one atom width `lbo` apart.
+// Shared addresses stay below 2^18, so a descriptor can be advanced by adding
+// (byte offset >> 4) to it.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t swizzle) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;   // descriptor version for sm_100
-  d |= (uint64_t)2 << 61;   // layout: 128-byte swizzle
+  d |= (uint64_t)swizzle << 61;
   return d;
+}
+constexpr uint32_t kSwizzle128B = 2;
+constexpr uint32_t kSwizzle64B = 4;
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return smem_desc(saddr, lbo, sbo, kSwizzle128B);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
@@ -276,6 +302,25 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | ((b_mn_major ? 1u : 0u) << 16)    // B major
          | ((uint32_t)(N >> 3) << 17)        // N / 8
          | ((uint32_t)(M >> 4) << 24);       // M / 16
+}
+
+// Launch with programmatic stream serialization allowed (PDL): the kernel may
+// start while the previous kernel on the stream is still running; it must
+// execute griddepcontrol.wait before touching that kernel's results.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Byte offset of bf16 element (row, col) inside a tile of 128-byte rows
