@@ -188,6 +188,43 @@ xmla_status xmla_decode_profiled(const xmla_yarn_cfg* cfg, const void* q, const 
                                  int32_t* status_dev, void* out, void* stream, void* attn_start,
                                  void* attn_stop);
 
+/* Size in bytes of the fixed device scratch used by xmla_decode_noalloc. */
+#define XMLA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* xmla_decode for callers that must not allocate device memory.  (The source
+ * pages describe the model, not a library; this entry point has no
+ * counterpart there.)
+ *
+ * Some callers cannot provide or allocate scratch: a plugin or backend inside
+ * an inference server whose host process owns every device allocation, code
+ * that runs on a latency-critical path where cudaMalloc's implicit device
+ * synchronisation and allocator locks are not acceptable, or a program whose
+ * memory is pre-carved into a fixed arena.  This entry point takes the same
+ * inputs and output as xmla_decode but no workspace: its scratch is a fixed
+ * XMLA_NOALLOC_SCRATCH_BYTES array compiled into the library, which every GPU
+ * that loads the library keeps until the process exits.  It calls no
+ * cudaMalloc, cudaFree or allocating routine.
+ *
+ * Limits and behaviour:
+ *   - Sizes whose workspace (xmla_decode_workspace_size) exceeds
+ *     XMLA_NOALLOC_SCRATCH_BYTES are rejected with XMLA_ERR_WORKSPACE before
+ *     anything is launched.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture on that device.
+ *   - All calls share the one array and it keeps the previous call's
+ *     contents.  Nothing in it has to start at zero: every value a call reads
+ *     was written earlier by the same call.  Calls whose work may overlap on
+ *     the GPU (concurrent streams, or several host threads) race on the array
+ *     and give wrong results; serialise them.
+ * Results equal xmla_decode's for the same arguments and split count. */
+xmla_status xmla_decode_noalloc(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
+                                const void* W_UV, const void* pool, int64_t num_blocks,
+                                const int32_t* block_table, int32_t max_blocks,
+                                const int32_t* seqlens, int32_t batch, int32_t q_len,
+                                int64_t max_seqlen, float softmax_scale, int32_t num_splits,
+                                int32_t* status_dev, void* out, void* stream);
+
 /* Self-test of the kernels' bounded wait: launches one CTA that waits on a
  * shared-memory barrier nothing ever arrives on, with the given limit in
  * nanoseconds, and records XMLA_ERR_TIMEOUT in *status_dev when the wait gives

@@ -30,6 +30,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "xmla_device.cuh"
 #include "yarn.cuh"
@@ -990,6 +991,59 @@ extern "C" xmla_status xmla_decode(const xmla_yarn_cfg* cfg, const void* q, cons
   return xmla_decode_profiled(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens,
                               batch, q_len, max_seqlen, softmax_scale, num_splits, workspace,
                               workspace_bytes, status_dev, out, stream, nullptr, nullptr);
+}
+
+// ---------------------------------------------------------------- decode without caller scratch
+
+namespace xmla {
+
+// Fixed device scratch for xmla_decode_noalloc.  It is part of the library's
+// module image, so every GPU that loads the library holds it until the
+// process exits; its size is the largest workspace that entry point accepts.
+constexpr size_t kNoAllocScratchBytes = (size_t)XMLA_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_noalloc_mutex;
+static void* g_noalloc_addr[64] = {};
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the real address is asked
+// from the runtime once per device (with that device current) and cached.
+static xmla_status noalloc_scratch(void** addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return XMLA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return XMLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return XMLA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return XMLA_OK;
+}
+
+}  // namespace xmla
+
+extern "C" xmla_status xmla_decode_noalloc(const xmla_yarn_cfg* cfg, const void* q,
+                                           const void* W_UK, const void* W_UV, const void* pool,
+                                           int64_t num_blocks, const int32_t* block_table,
+                                           int32_t max_blocks, const int32_t* seqlens,
+                                           int32_t batch, int32_t q_len, int64_t max_seqlen,
+                                           float softmax_scale, int32_t num_splits,
+                                           int32_t* status_dev, void* out, void* stream) {
+  int nsm = 0;
+  if (!xmla::device_ok(&nsm)) return XMLA_ERR_UNSUPPORTED;
+  const size_t need = xmla_decode_workspace_size(batch, q_len, max_seqlen, nsm, num_splits);
+  if (need == 0) return XMLA_ERR_SHAPE;
+  if (need > xmla::kNoAllocScratchBytes) return XMLA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const xmla_status st = xmla::noalloc_scratch(&scratch);
+  if (st != XMLA_OK) return st;
+  return xmla_decode(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens, batch,
+                     q_len, max_seqlen, softmax_scale, num_splits, scratch,
+                     xmla::kNoAllocScratchBytes, status_dev, out, stream);
 }
 
 extern "C" xmla_status xmla_selftest_wait_timeout(int32_t* status_dev, uint64_t timeout_ns,

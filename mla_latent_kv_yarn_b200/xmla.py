@@ -25,7 +25,8 @@ STATUS_NAMES = {
 EXPORTS = [
     "xmla_yarn_default", "xmla_yarn_inv_freq", "xmla_softmax_scale", "xmla_rope_yarn",
     "xmla_cache_append", "xmla_decode_workspace_size", "xmla_decode_num_splits", "xmla_decode",
-    "xmla_decode_profiled", "xmla_selftest_wait_timeout", "xmla_status_string",
+    "xmla_decode_profiled", "xmla_decode_noalloc", "xmla_selftest_wait_timeout",
+    "xmla_status_string",
 ]
 
 
@@ -80,6 +81,9 @@ def lib() -> ctypes.CDLL:
         L.xmla_decode.restype = ctypes.c_int
         L.xmla_decode_profiled.argtypes = L.xmla_decode.argtypes + [vp, vp]
         L.xmla_decode_profiled.restype = ctypes.c_int
+        L.xmla_decode_noalloc.argtypes = [cfgp, vp, vp, vp, vp, i64, vp, i32, vp, i32, i32, i64, f32,
+                                          i32, vp, vp, vp]
+        L.xmla_decode_noalloc.restype = ctypes.c_int
         L.xmla_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
         L.xmla_selftest_wait_timeout.restype = ctypes.c_int
         L.xmla_status_string.argtypes = [ctypes.c_int]
@@ -180,6 +184,19 @@ def xmla_decode_profiled(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_
                                       int(num_splits), _ptr(workspace), int(workspace_bytes),
                                       _ptr(status), _ptr(out), _stream(stream), ev[0], ev[1]),
            "xmla_decode_profiled")
+
+
+def xmla_decode_noalloc(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens,
+                        batch, q_len, max_seqlen, softmax_scale, num_splits, status, out,
+                        stream=None) -> None:
+    """xmla_decode with the library's fixed device scratch instead of a caller
+    workspace (for callers that may not allocate device memory)."""
+    _check(lib().xmla_decode_noalloc(ctypes.byref(cfg), _ptr(q), _ptr(W_UK), _ptr(W_UV), _ptr(pool),
+                                     int(num_blocks), _ptr(block_table), int(max_blocks),
+                                     _ptr(seqlens), int(batch), int(q_len), int(max_seqlen),
+                                     float(softmax_scale), int(num_splits), _ptr(status), _ptr(out),
+                                     _stream(stream)),
+           "xmla_decode_noalloc")
 
 
 def xmla_selftest_wait_timeout(status: torch.Tensor, timeout_ns: int, stream=None) -> None:
