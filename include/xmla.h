@@ -110,19 +110,24 @@ xmla_status xmla_rope_yarn(const xmla_yarn_cfg* cfg, void* x, int64_t rows, int3
 /* Append token rows to the paged latent cache ([P1] section 二 and [P5] MLA
  * section: per token and layer the cache holds the latent and the rope key).
  * For i < T:  pool[block_table[seq_ids[i]*max_blocks + positions[i]/64]]
- *                 [positions[i] % 64] = [c_kv[i] (512) | k_pe_rot[i] (64)]
- * as an exact bit copy.
+ *                 [positions[i] % 64] = [c_kv[i] (512) | k_rot[i] (64)]
+ * where k_rot[i] = k_pe[i] when rope_cfg is NULL (an exact bit copy of rows
+ * rotated beforehand, e.g. by xmla_rope_yarn), and otherwise the YaRN RoPE of
+ * k_pe[i] at positions[i] with rope_cfg, computed as xmla_rope_yarn does
+ * (float64 angle, one bf16 rounding).  c_kv is always copied bit-exactly.
  *   pool: device bf16 [num_blocks, 64, 576] (written);
  *   block_table: device int32 [batch, max_blocks];
  *   seq_ids: device int32 [T] in [0, batch); positions: device int64 [T];
- *   c_kv: device bf16 [T, 512]; k_pe_rot: device bf16 [T, 64] (already rotated).
+ *   c_kv: device bf16 [T, 512]; k_pe: device bf16 [T, 64];
+ *   rope_cfg: host pointer or NULL (see above).
  * A row whose seq id, position or block id falls outside its range is skipped
  * and XMLA_ERR_DEVICE_OOB is recorded in *status_dev (if not NULL).
  * T == 0 is a no-op.  Errors: XMLA_ERR_INVALID_ARG, XMLA_ERR_SHAPE, XMLA_ERR_CUDA. */
 xmla_status xmla_cache_append(void* pool, int64_t num_blocks, const int32_t* block_table,
                               int32_t max_blocks, int32_t batch, const int32_t* seq_ids,
-                              const int64_t* positions, const void* c_kv, const void* k_pe_rot,
-                              int64_t T, int32_t* status_dev, void* stream);
+                              const int64_t* positions, const void* c_kv, const void* k_pe,
+                              const xmla_yarn_cfg* rope_cfg, int64_t T, int32_t* status_dev,
+                              void* stream);
 
 /* Bytes of device workspace xmla_decode needs for these sizes on a device with
  * num_sms SMs (num_splits = 0 picks the split count automatically, > 0 forces

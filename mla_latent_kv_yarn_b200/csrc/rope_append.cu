@@ -39,12 +39,15 @@ __global__ void __launch_bounds__(256) rope_yarn_kernel(__nv_bfloat16* __restric
 
 // ---------------------------------------------------------------- device: append
 
-// One thread per 16-byte piece of a cache row (64 pieces of latent, 8 of rope key).
+// One thread per 16-byte piece of a cache row: 64 pieces of latent (bit copy)
+// and 8 pieces of rope key.  With rotation on, rope piece r instead rotates
+// the four pairs (4r .. 4r+3, 4r+32 .. 4r+35) at the row's position and
+// stores them.
 __global__ void __launch_bounds__(256) cache_append_kernel(
     uint4* __restrict__ pool, int64_t num_blocks, const int32_t* __restrict__ block_table,
     int32_t max_blocks, int32_t batch, const int32_t* __restrict__ seq_ids,
     const int64_t* __restrict__ positions, const uint4* __restrict__ c_kv,
-    const uint4* __restrict__ k_pe, int64_t T, int32_t* status) {
+    const uint4* __restrict__ k_pe, int64_t T, int32_t* status, int rotate, const RopeTable tab) {
   constexpr int kLatPieces = kDLatent * 2 / 16;  // 64
   constexpr int kRopePieces = kDRope * 2 / 16;   // 8
   constexpr int kRowPieces = kLatPieces + kRopePieces;
@@ -64,9 +67,32 @@ __global__ void __launch_bounds__(256) cache_append_kernel(
       record_status(status, XMLA_ERR_DEVICE_OOB);
       continue;
     }
-    const uint4 val = piece < kLatPieces ? c_kv[t * kLatPieces + piece]
-                                         : k_pe[t * kRopePieces + (piece - kLatPieces)];
-    pool[((int64_t)blk * kPage + pos % kPage) * kRowPieces + piece] = val;
+    uint4* row = pool + ((int64_t)blk * kPage + pos % kPage) * kRowPieces;
+    if (piece < kLatPieces) {
+      row[piece] = c_kv[t * kLatPieces + piece];
+    } else if (!rotate) {
+      row[piece] = k_pe[t * kRopePieces + (piece - kLatPieces)];
+    } else {
+      const int r = piece - kLatPieces;  // pairs 4r .. 4r+3
+      const uint2* src = reinterpret_cast<const uint2*>(k_pe + t * kRopePieces);
+      uint2* dst = reinterpret_cast<uint2*>(row + kLatPieces);
+      const uint2 lo = src[r], hi = src[r + 8];  // dims 4r.., 32+4r..
+      const __nv_bfloat16* xl = reinterpret_cast<const __nv_bfloat16*>(&lo);
+      const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&hi);
+      uint2 olo, ohi;
+      __nv_bfloat16* yl = reinterpret_cast<__nv_bfloat16*>(&olo);
+      __nv_bfloat16* yh = reinterpret_cast<__nv_bfloat16*>(&ohi);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        double y1, y2;
+        rope_pair((double)__bfloat162float(xl[e]), (double)__bfloat162float(xh[e]), pos, 4 * r + e,
+                  tab, &y1, &y2);
+        yl[e] = __double2bfloat16(y1);
+        yh[e] = __double2bfloat16(y2);
+      }
+      dst[r] = olo;
+      dst[r + 8] = ohi;
+    }
   }
 }
 
@@ -126,18 +152,24 @@ extern "C" xmla_status xmla_rope_yarn(const xmla_yarn_cfg* cfg, void* x, int64_t
 extern "C" xmla_status xmla_cache_append(void* pool, int64_t num_blocks, const int32_t* block_table,
                                          int32_t max_blocks, int32_t batch, const int32_t* seq_ids,
                                          const int64_t* positions, const void* c_kv,
-                                         const void* k_pe_rot, int64_t T, int32_t* status_dev,
-                                         void* stream) {
+                                         const void* k_pe, const xmla_yarn_cfg* rope_cfg, int64_t T,
+                                         int32_t* status_dev, void* stream) {
   if (T < 0 || num_blocks < 1 || max_blocks < 1 || batch < 1) return XMLA_ERR_SHAPE;
   if (T == 0) return XMLA_OK;
   if (pool == nullptr || block_table == nullptr || seq_ids == nullptr || positions == nullptr ||
-      c_kv == nullptr || k_pe_rot == nullptr)
+      c_kv == nullptr || k_pe == nullptr)
     return XMLA_ERR_INVALID_ARG;
-  if ((((uintptr_t)pool) | ((uintptr_t)c_kv) | ((uintptr_t)k_pe_rot)) & 15u)
+  if ((((uintptr_t)pool) | ((uintptr_t)c_kv) | ((uintptr_t)k_pe)) & 15u)
     return XMLA_ERR_INVALID_ARG;
+  RopeTable tab = {};
+  if (rope_cfg != nullptr) {
+    if (!yarn_cfg_ok(rope_cfg)) return XMLA_ERR_INVALID_ARG;
+    if (rope_cfg->rotary_dim != kDRope) return XMLA_ERR_SHAPE;
+    tab = make_rope_table(rope_cfg);
+  }
   const int64_t work = T * 72;
   cache_append_kernel<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(
       (uint4*)pool, num_blocks, block_table, max_blocks, batch, seq_ids, positions,
-      (const uint4*)c_kv, (const uint4*)k_pe_rot, T, status_dev);
+      (const uint4*)c_kv, (const uint4*)k_pe, T, status_dev, rope_cfg != nullptr ? 1 : 0, tab);
   return cudaGetLastError() == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
 }

@@ -5,9 +5,9 @@ table, sequence lengths, weights, workspace, output) and issues the library
 calls in decode order.  No arithmetic of the method happens here.
 
 One decode step over a layer ("the hot path"):
-  1. xmla_rope_yarn on k_pe of the step's q_len new tokens per sequence,
-  2. xmla_cache_append of those tokens' [c_kv | rotated k_pe] rows,
-  3. xmla_decode (q absorb with RoPE of q_pe -> split-K latent attention ->
+  1. xmla_cache_append of the step's q_len new tokens per sequence, rotating
+     their k_pe with YaRN RoPE as it stores [c_kv | rotated k_pe],
+  2. xmla_decode (q absorb with RoPE of q_pe -> split-K latent attention ->
      combine with W_UV).
 """
 from __future__ import annotations
@@ -89,12 +89,11 @@ def build_layer(cfg, wl: Workload, inp: LayerInputs, device, chunk: int = 1 << 2
     for t0 in range(0, T, chunk):
         t1 = min(T, t0 + chunk)
         c = inp.c_kv[t0:t1].to(device, non_blocking=True)
-        k = inp.k_pe[t0:t1].to(device, non_blocking=True).clone()  # rotated in place
+        k = inp.k_pe[t0:t1].to(device, non_blocking=True).contiguous()
         pos = inp.positions[t0:t1].to(device)
         sid = inp.seq_ids[t0:t1].to(device)
-        rope_rows(cfg, k, pos)
         xmla.xmla_cache_append(pool, inp.num_blocks, bt, bt.shape[1], wl.batch, sid, pos, c, k,
-                               t1 - t0, status)
+                               cfg, t1 - t0, status)
     return LayerState(pool=pool, block_table=bt, seqlens=inp.seqlens.to(device),
                       W_UK=inp.W_UK.to(device), W_UV=inp.W_UV.to(device),
                       num_blocks=inp.num_blocks, max_blocks=bt.shape[1])
@@ -134,11 +133,11 @@ class Decoder:
     def step(self, cfg, st: LayerState, q: torch.Tensor, c_new: torch.Tensor,
              k_new: torch.Tensor, new_pos: torch.Tensor, new_seq: torch.Tensor,
              softmax_scale: float, out=None, stream=None, events=None) -> torch.Tensor:
-        """One decode step.  q is raw; k_new (the q_len newest tokens' rope keys)
-        is rotated in place and appended with c_new before attending."""
-        rope_rows(cfg, k_new, new_pos, stream)
+        """One decode step on raw q: the q_len newest tokens (c_new, k_new raw)
+        are appended with their rope keys rotated, then the layer attends."""
         xmla.xmla_cache_append(st.pool, st.num_blocks, st.block_table, st.max_blocks, self.batch,
-                               new_seq, new_pos, c_new, k_new, c_new.shape[0], self.status, stream)
+                               new_seq, new_pos, c_new, k_new, cfg, c_new.shape[0], self.status,
+                               stream)
         return self.decode(cfg, st, q, softmax_scale, out, stream, events)
 
     def check_status(self) -> int:

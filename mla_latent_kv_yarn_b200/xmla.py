@@ -70,7 +70,7 @@ def lib() -> ctypes.CDLL:
         L.xmla_softmax_scale.restype = f64
         L.xmla_rope_yarn.argtypes = [cfgp, vp, i64, i32, i64, i64, i32, vp, vp]
         L.xmla_rope_yarn.restype = ctypes.c_int
-        L.xmla_cache_append.argtypes = [vp, i64, vp, i32, i32, vp, vp, vp, vp, i64, vp, vp]
+        L.xmla_cache_append.argtypes = [vp, i64, vp, i32, i32, vp, vp, vp, vp, cfgp, i64, vp, vp]
         L.xmla_cache_append.restype = ctypes.c_int
         L.xmla_decode_workspace_size.argtypes = [i32, i32, i64, i32, i32]
         L.xmla_decode_workspace_size.restype = sz
@@ -138,12 +138,13 @@ def xmla_rope_yarn(cfg: xmla_yarn_cfg, x: torch.Tensor, rows: int, n_heads: int,
 
 def xmla_cache_append(pool: torch.Tensor, num_blocks: int, block_table: torch.Tensor,
                       max_blocks: int, batch: int, seq_ids: torch.Tensor, positions: torch.Tensor,
-                      c_kv: torch.Tensor, k_pe_rot: torch.Tensor, T: int,
-                      status: torch.Tensor | None = None, stream=None) -> None:
+                      c_kv: torch.Tensor, k_pe: torch.Tensor, rope_cfg: xmla_yarn_cfg | None,
+                      T: int, status: torch.Tensor | None = None, stream=None) -> None:
     _check(lib().xmla_cache_append(_ptr(pool), int(num_blocks), _ptr(block_table),
                                    int(max_blocks), int(batch), _ptr(seq_ids), _ptr(positions),
-                                   _ptr(c_kv), _ptr(k_pe_rot), int(T), _ptr(status),
-                                   _stream(stream)),
+                                   _ptr(c_kv), _ptr(k_pe),
+                                   None if rope_cfg is None else ctypes.byref(rope_cfg), int(T),
+                                   _ptr(status), _stream(stream)),
            "xmla_cache_append")
 
 

@@ -85,8 +85,8 @@ def test_argument_validation_without_gpu(x):
     bad = x.xmla_yarn_default()
     bad.rotary_dim = 32
     assert L.xmla_rope_yarn(ctypes.byref(bad), None, 1, 1, 64, 64, 0, None, None) == 2
-    assert L.xmla_cache_append(None, 4, None, 1, 1, None, None, None, None, 0, None, None) == 0
-    assert L.xmla_cache_append(None, 4, None, 1, 1, None, None, None, None, 3, None, None) == 1
+    assert L.xmla_cache_append(None, 4, None, 1, 1, None, None, None, None, None, 0, None, None) == 0
+    assert L.xmla_cache_append(None, 4, None, 1, 1, None, None, None, None, None, 3, None, None) == 1
     assert L.xmla_selftest_wait_timeout(None, 1000, None) == 1
     for code in range(8):
         assert x.xmla_status_string(code)

@@ -64,7 +64,7 @@ def test_cache_append_is_a_bit_exact_scatter():
     pool = pool0.cuda()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     xmla.xmla_cache_append(pool, pool.shape[0], bt.cuda(), bt.shape[1], 3, sid.cuda(), pos.cuda(),
-                           c_bits.cuda(), k_bits.cuda(), T, status)
+                           c_bits.cuda(), k_bits.cuda(), None, T, status)
     torch.cuda.synchronize()
     want = pool0.numpy().view(np.uint16).copy()
     om.cache_append(want, bt.numpy(), sid.numpy(), pos.numpy(), c_bits.numpy().view(np.uint16),
@@ -81,13 +81,40 @@ def test_cache_append_skips_out_of_range_rows():
     k = torch.ones((5, 64), dtype=torch.bfloat16)
     pool = torch.zeros((3, 64, 576), dtype=torch.bfloat16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    xmla.xmla_cache_append(pool, 3, bt.cuda(), 2, 2, sid.cuda(), pos.cuda(), c.cuda(), k.cuda(), 5,
-                           status)
+    xmla.xmla_cache_append(pool, 3, bt.cuda(), 2, 2, sid.cuda(), pos.cuda(), c.cuda(), k.cuda(), None,
+                           5, status)
     torch.cuda.synchronize()
     assert int(status.item()) == 5
     p = pool.cpu().float()
     assert torch.all(p[1, 3] == 1) and torch.all(p[2, 10] == 1)    # the two valid rows landed
     assert float(p.sum()) == 2 * 576
+
+
+def test_cache_append_with_rope_rotates_the_key_and_copies_the_latent():
+    cfg, ocfg = gc.cfgs()
+    g = torch.Generator().manual_seed(12)
+    # distinct positions, some far past the original context (float64 angle matters there)
+    pos = torch.cat([torch.tensor([0, 1, 63, 4095, 262143, 262144, 524287]),
+                     torch.randperm(524287, generator=g)[:293] + 1]).unique()
+    T = pos.numel()
+    c = torch.randn((T, 512), generator=g).to(torch.bfloat16)
+    k = torch.randn((T, 64), generator=g).to(torch.bfloat16)
+    logical = torch.unique(pos // 64)
+    bt = torch.zeros((1, 524288 // 64), dtype=torch.int32)
+    bt[0, logical] = torch.arange(logical.numel(), dtype=torch.int32)
+    nblk = logical.numel()
+    pool = torch.zeros((nblk, 64, 576), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sid = torch.zeros(T, dtype=torch.int32)
+    xmla.xmla_cache_append(pool, nblk, bt.cuda(), bt.shape[1], 1, sid.cuda(), pos.cuda(), c.cuda(),
+                           k.cuda(), cfg, T, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = pool.cpu()
+    rows = got[bt[0, pos // 64].long(), (pos % 64).long()]
+    assert torch.equal(rows[:, :512].view(torch.int16), c.view(torch.int16))
+    want = om.rope(gc.f64(k), pos.numpy(), ocfg)
+    assert np.all(np.abs(gc.f64(rows[:, 512:]) - want) <= _half_ulp_bf16(want) * (1 + 1e-6))
 
 
 # ------------------------------------------------------------------ decode, small cases
