@@ -658,17 +658,28 @@ __global__ void __launch_bounds__(128) q_absorb_kernel(const __nv_bfloat16* __re
 constexpr int kSlices = 8;
 constexpr int kSliceDims = kDLatent / kSlices;  // 64
 constexpr int kCombineRows = 16;
+constexpr int kCombineThreads = 256;
+constexpr int kCombineGroups = kCombineThreads / 16;  // split rows read at once (16 threads x float4 each)
+constexpr int kCombineDepth = 10;                     // split rows each thread keeps in flight
 
-__global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(128)
+// Online (max, sum-of-exp2) pair merge.
+__device__ __forceinline__ void lse_merge(float& m, float& l, float m2, float l2) {
+  const float mx = fmaxf(m, m2);
+  if (mx == -INFINITY) return;
+  l = l * ex2(m - mx) + l2 * ex2(m2 - mx);
+  m = mx;
+}
+
+__global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThreads)
     combine_uv_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                       const __nv_bfloat16* __restrict__ W_UV, __nv_bfloat16* __restrict__ out,
                       int rows, int q_len, int groups, int nsplit, int rows_per_cta) {
   __shared__ __align__(16) __nv_bfloat16 w_s[kSliceDims][kDV];  // this slice's rows of W_UV[h]
   __shared__ float wt_s[kMaxSplits];                             // split weights of one row
-  __shared__ __align__(16) float4 acc_s[8][kSliceDims / 4];
+  __shared__ __align__(16) float4 acc_s[kCombineGroups][kSliceDims / 4];
   __shared__ float o_s[kCombineRows][kSliceDims];
-  __shared__ float out_s[kCombineRows][kDV];
-  __shared__ float red_s[8];
+  __shared__ float out_s[2][kCombineRows][kDV];
+  __shared__ float red_m[kCombineThreads / 32], red_l[kCombineThreads / 32];
   cg::cluster_group cluster = cg::this_cluster();
   const int slice = (int)cluster.block_rank();
   const int cid = blockIdx.x / kSlices;
@@ -677,60 +688,81 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(128)
   const int r0 = chunk * kCombineRows;
   const int nr = min(kCombineRows, rows - r0);
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
   pdl_launch_dependents();
   // W_UV does not depend on the decode kernel: stage it while that kernel finishes
   {
     const uint4* src = reinterpret_cast<const uint4*>(W_UV + ((int64_t)h * kDLatent + slice * kSliceDims) * kDV);
     uint4* dst = reinterpret_cast<uint4*>(&w_s[0][0]);
 #pragma unroll
-    for (int e = 0; e < kSliceDims * kDV / 8 / 128; ++e) dst[tid + 128 * e] = src[tid + 128 * e];
+    for (int e = 0; e < kSliceDims * kDV / 8 / kCombineThreads; ++e)
+      dst[tid + kCombineThreads * e] = src[tid + kCombineThreads * e];
   }
   pdl_wait();  // the split partials come from the decode kernel
 
+  const int q4 = tid & 15;  // float4 of the 64-dim slice
+  const int grp = tid >> 4;
   for (int rr = 0; rr < nr; ++rr) {
     const int r = r0 + rr;  // r = b*q_len + j
     const int b = r / q_len, j = r % q_len;
     const int ridx = j * kHeads + h;
     const int g = ridx / rows_per_cta;
     const int n = ridx % rows_per_cta;
-    const int64_t item0 = ((int64_t)b * groups + g) * nsplit;
-    const float2* ml = reinterpret_cast<const float2*>(part_ml) + item0 * rows_per_cta + n;
-    // max over the splits that saw any token
-    float mx = -INFINITY;
-    for (int s = tid; s < nsplit; s += 128) {
-      const float2 v = ml[(int64_t)s * rows_per_cta];
-      if (v.y > 0.f) mx = fmaxf(mx, v.x);
+    const int64_t row0 = ((int64_t)b * groups + g) * nsplit * rows_per_cta + n;  // split 0's row
+    const float2* ml = reinterpret_cast<const float2*>(part_ml) + row0;
+    const float* po = part_o + row0 * kDLatent + slice * kSliceDims + 4 * q4;
+    const int64_t o_stride = (int64_t)rows_per_cta * kDLatent;
+    // first batch of O rows: issued before the log-sum-exp so both latencies overlap
+    float4 v[kCombineDepth];
+#pragma unroll
+    for (int k = 0; k < kCombineDepth; ++k) {
+      const int sidx = grp + kCombineGroups * k;
+      v[k] = sidx < nsplit ? *reinterpret_cast<const float4*>(po + sidx * o_stride)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if ((tid & 31) == 0) red_s[tid >> 5] = mx;
-    __syncthreads();
-    mx = fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3]));
-    float lsum = 0.f;
-    for (int s = tid; s < nsplit; s += 128) {
-      const float2 v = ml[(int64_t)s * rows_per_cta];
-      const float wgt = v.y > 0.f ? ex2(v.x - mx) : 0.f;
-      wt_s[s] = wgt;
-      lsum = fmaf(wgt, v.y, lsum);
+    // global max M and sum L = sum_s l_s 2^(m_s - M) over the splits that saw tokens
+    float m = -INFINITY, l = 0.f;
+    for (int sidx = tid; sidx < nsplit; sidx += kCombineThreads) {
+      const float2 x = ml[(int64_t)sidx * rows_per_cta];
+      if (x.y > 0.f) lse_merge(m, l, x.x, x.y);
     }
-    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    if ((tid & 31) == 0) red_s[4 + (tid >> 5)] = lsum;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+      const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
+      lse_merge(m, l, m2, l2);
+    }
+    if (lane == 0) { red_m[tid >> 5] = m; red_l[tid >> 5] = l; }
     __syncthreads();
-    const float L = red_s[4] + red_s[5] + red_s[6] + red_s[7];
-    // this slice of the weighted sum: 16 threads x float4 cover the 64 dims of
-    // one split; the 8 thread groups take every 8th split
-    const int q4 = tid & 15;
-    const int grp = tid >> 4;
+    m = red_m[0];
+    l = red_l[0];
+#pragma unroll
+    for (int w = 1; w < kCombineThreads / 32; ++w) lse_merge(m, l, red_m[w], red_l[w]);
+    for (int sidx = tid; sidx < nsplit; sidx += kCombineThreads) {
+      const float2 x = ml[(int64_t)sidx * rows_per_cta];
+      wt_s[sidx] = x.y > 0.f ? ex2(x.x - m) : 0.f;
+    }
+    __syncthreads();
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float* po = part_o + (item0 * rows_per_cta + n) * kDLatent + slice * kSliceDims + 4 * q4;
-#pragma unroll 4
-    for (int s = grp; s < nsplit; s += 8) {
-      const float wgt = wt_s[s];
-      const float4 v = *reinterpret_cast<const float4*>(po + (int64_t)s * rows_per_cta * kDLatent);
-      if (wgt != 0.f) {
-        acc.x = fmaf(wgt, v.x, acc.x);
-        acc.y = fmaf(wgt, v.y, acc.y);
-        acc.z = fmaf(wgt, v.z, acc.z);
-        acc.w = fmaf(wgt, v.w, acc.w);
+    for (int s0 = 0;; s0 += kCombineGroups * kCombineDepth) {
+#pragma unroll
+      for (int k = 0; k < kCombineDepth; ++k) {
+        const int sidx = s0 + grp + kCombineGroups * k;
+        const float wgt = sidx < nsplit ? wt_s[sidx] : 0.f;
+        if (wgt != 0.f) {
+          acc.x = fmaf(wgt, v[k].x, acc.x);
+          acc.y = fmaf(wgt, v[k].y, acc.y);
+          acc.z = fmaf(wgt, v[k].z, acc.z);
+          acc.w = fmaf(wgt, v[k].w, acc.w);
+        }
+      }
+      const int s1 = s0 + kCombineGroups * kCombineDepth;
+      if (s1 >= nsplit) break;
+#pragma unroll
+      for (int k = 0; k < kCombineDepth; ++k) {
+        const int sidx = s1 + grp + kCombineGroups * k;
+        v[k] = sidx < nsplit ? *reinterpret_cast<const float4*>(po + sidx * o_stride)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     acc_s[grp][q4] = acc;
@@ -739,26 +771,28 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(128)
       const float* a = reinterpret_cast<const float*>(&acc_s[0][0]);
       float t = 0.f;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) t += a[k * kSliceDims + tid];
-      o_s[rr][tid] = L > 0.f ? t / L : 0.f;
+      for (int k = 0; k < kCombineGroups; ++k) t += a[k * kSliceDims + tid];
+      o_s[rr][tid] = l > 0.f ? t / l : 0.f;
     }
     __syncthreads();
   }
 
-  // partial out[r][v] = sum over this slice's 64 latent dims of o[r][c] W_UV[h][c][v]
+  // partial out[r][v] = sum over this slice's 64 latent dims of o[r][c] W_UV[h][c][v];
+  // the two halves of the CTA take 32 dims each
   {
-    const int v = tid;
+    const int v = tid & (kDV - 1);
+    const int hf = tid >> 7;
     float acc[kCombineRows];
 #pragma unroll
     for (int rr = 0; rr < kCombineRows; ++rr) acc[rr] = 0.f;
 #pragma unroll 8
-    for (int c = 0; c < kSliceDims; ++c) {
+    for (int c = 32 * hf; c < 32 * hf + 32; ++c) {
       const float wcv = __bfloat162float(w_s[c][v]);
 #pragma unroll
       for (int rr = 0; rr < kCombineRows; ++rr) acc[rr] = fmaf(o_s[rr][c], wcv, acc[rr]);
     }
 #pragma unroll
-    for (int rr = 0; rr < kCombineRows; ++rr) out_s[rr][v] = acc[rr];
+    for (int rr = 0; rr < kCombineRows; ++rr) out_s[hf][rr][v] = acc[rr];
   }
   cluster.sync();
   if (slice == 0) {
@@ -766,7 +800,10 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(128)
       const int rr = e / kDV, v = e % kDV;
       float t = 0.f;
 #pragma unroll
-      for (int k = 0; k < kSlices; ++k) t += cluster.map_shared_rank(&out_s[0][0], k)[rr * kDV + v];
+      for (int k = 0; k < kSlices; ++k) {
+        const float* peer = cluster.map_shared_rank(&out_s[0][0][0], k);
+        t += peer[rr * kDV + v] + peer[kCombineRows * kDV + rr * kDV + v];
+      }
       out[((int64_t)(r0 + rr) * kHeads + h) * kDV + v] = __float2bfloat16_rn(t);
     }
   }
@@ -975,7 +1012,7 @@ extern "C" xmla_status xmla_decode_profiled(const xmla_yarn_cfg* cfg, const void
   if (record_event(attn_stop, st) != cudaSuccess) return XMLA_ERR_CUDA;
 
   const int chunks = (rows + kCombineRows - 1) / kCombineRows;
-  e = launch_pdl(combine_uv_kernel, dim3(kSlices * kHeads * chunks), dim3(128), 0, st,
+  e = launch_pdl(combine_uv_kernel, dim3(kSlices * kHeads * chunks), dim3(kCombineThreads), 0, st,
                  (const float*)dp.part_o, (const float*)dp.part_ml, (const __nv_bfloat16*)W_UV,
                  (__nv_bfloat16*)out, rows, q_len, P.groups, P.nsplit, P.nr);
   return e == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
