@@ -58,6 +58,22 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest per-rank value (a time) across all ranks of the job."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank_step: int, steps: int, max_total_ms: float, world: int) -> float:
+    """Whole-job GB/s: what every rank streamed, over the slowest rank's time."""
+    return bytes_per_rank_step * world * steps / (max_total_ms * 1e-3) / 1e9
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -335,11 +351,7 @@ def run_xmla(args, wl):
     step_ms, _ = timed(graph, False)
     clk = clocks.stop()
     _, attn_ms = timed(graph_k, True)
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     status = dec.check_status()
 
     # ---- end to end through the API: pinned host inputs in, result out, every step
@@ -363,16 +375,12 @@ def run_xmla(args, wl):
         ee1[i].record(stream)
         ee1[i].synchronize()
         e2e_ms.append(ee0[i].elapsed_time(ee1[i]))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    e2e_total = max_over_ranks(sum(e2e_ms), dev)
 
     cache_bytes_layer = sum(wl.seqlens) * ROW_BYTES
     tokens_step = sum(wl.seqlens) * wl.layers * world
     bytes_step = cache_bytes_layer * wl.layers * world
-    gbs = bytes_step * args.steps / (total_ms * 1e-3) / 1e9
+    gbs = job_throughput(cache_bytes_layer * wl.layers, args.steps, total_ms, world)
     peak, peak_kind = measured_peaks()
     attn_mean_ms = statistics.mean(attn_ms)
     achieved = cache_bytes_layer / (attn_mean_ms * 1e-3) / 1e9
@@ -395,7 +403,8 @@ def run_xmla(args, wl):
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "algorithmic_bytes_per_launch": cache_bytes_layer,
                          "kernel_ms": round(attn_mean_ms, 5), "peak_source": peak_kind},
-            "e2e": {"value": round(bytes_step * args.steps / (e2e_total * 1e-3) / 1e9, 3),
+            "e2e": {"value": round(job_throughput(cache_bytes_layer * wl.layers, args.steps,
+                                                  e2e_total, world), 3),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "splits": dec.splits,
