@@ -227,7 +227,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       int32_t nb1 = n_pages > 1 ? bt[1] : 0;
       int32_t nb2 = n_pages > 2 ? bt[2] : 0;
       int32_t nb3 = n_pages > 3 ? bt[3] : 0;
+      const int64_t first_new = seqlen - p.q_len;  // first row appended by this step
+      bool waited = false;
       for (int i = 0; i < n_pages && ok; ++i) {
+        if (!waited && (p_begin + i + 1) * kPage > first_new) {
+          // this page holds rows written by the kernels launched just before:
+          // wait for them (through q_absorb's completion) before reading it
+          pdl_wait();
+          waited = true;
+        }
         int32_t blk = nb0;
         nb0 = nb1;
         nb1 = nb2;
@@ -266,7 +274,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         if (!q_issued) {
           // q_ext is the previous kernel's output: wait for it only after the
           // first page is on its way.
-          pdl_wait();
+          if (!waited) pdl_wait();
+          waited = true;
           mbar_arrive_expect_tx(bar(L::kBarQ), 9u * L::kQChunk);
           for (int c = 0; c < 9; ++c)
             tma_load_2d(base + L::kOffQ + c * L::kQChunk, &tmap_q, c * 64, qrow0, bar(L::kBarQ));
@@ -586,6 +595,9 @@ __global__ void __launch_bounds__(128) q_absorb_kernel(const __nv_bfloat16* __re
                                                        const RopeTable tab) {
   __shared__ float sq[kAbsorbRows][kDNope];
   __shared__ float part[16][kAbsorbRows][64];
+  // q and the cache rows of this step may come from the kernels launched just
+  // before; the decode kernel relies on this wait (see its producer)
+  pdl_wait();
   pdl_launch_dependents();
   const int h = blockIdx.x;
   const int cb = blockIdx.y;
@@ -983,13 +995,13 @@ extern "C" xmla_status xmla_decode_profiled(const xmla_yarn_cfg* cfg, const void
   if (!encode_rows576(&tmap_q, q_ext, (uint64_t)rows * kHeads, (uint32_t)P.nr)) return XMLA_ERR_CUDA;
 
   const float qscale = softmax_scale * kLog2e;
-  // q_absorb reads only the caller's inputs; it is an ordinary launch so that it
-  // (and hence the decode kernel chained to it) starts after every earlier
-  // write to the cache on this stream has landed.
-  q_absorb_kernel<<<dim3(kHeads, kDLatent / 64), 128, 0, st>>>(
-      (const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext, rows, q_len, qscale,
-      make_rope_table(cfg));
-  if (cudaGetLastError() != cudaSuccess) return XMLA_ERR_CUDA;
+  // Every kernel of the chain waits (griddepcontrol.wait) for its predecessor
+  // before reading anything a kernel of this step may have written, so once
+  // q_absorb completes all earlier work on the stream has landed.
+  if (launch_pdl(q_absorb_kernel, dim3(kHeads, kDLatent / 64), dim3(128), 0, st,
+                 (const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext, rows, q_len,
+                 qscale, make_rope_table(cfg)) != cudaSuccess)
+    return XMLA_ERR_CUDA;
 
   DecodeParams dp;
   dp.block_table = block_table;

@@ -21,6 +21,8 @@ __global__ void __launch_bounds__(256) rope_yarn_kernel(__nv_bfloat16* __restric
                                                         int64_t row_stride, int32_t offset,
                                                         const int64_t* __restrict__ positions,
                                                         const RopeTable tab) {
+  pdl_wait();  // inputs may come from the kernel launched just before
+  pdl_launch_dependents();
   const int64_t total = rows * (int64_t)n_heads * (kDRope / 2);
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x) {
@@ -48,6 +50,8 @@ __global__ void __launch_bounds__(256) cache_append_kernel(
     int32_t max_blocks, int32_t batch, const int32_t* __restrict__ seq_ids,
     const int64_t* __restrict__ positions, const uint4* __restrict__ c_kv,
     const uint4* __restrict__ k_pe, int64_t T, int32_t* status, int rotate, const RopeTable tab) {
+  pdl_wait();  // inputs may come from the kernel launched just before
+  pdl_launch_dependents();
   constexpr int kLatPieces = kDLatent * 2 / 16;  // 64
   constexpr int kRopePieces = kDRope * 2 / 16;   // 8
   constexpr int kRowPieces = kLatPieces + kRopePieces;
@@ -143,10 +147,11 @@ extern "C" xmla_status xmla_rope_yarn(const xmla_yarn_cfg* cfg, void* x, int64_t
     return XMLA_ERR_INVALID_ARG;
   const RopeTable tab = make_rope_table(cfg);
   const int64_t work = rows * n_heads * (kDRope / 2);
-  rope_yarn_kernel<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(
-      (__nv_bfloat16*)x, rows, n_heads, head_stride_elems, row_stride_elems, rope_offset_elems,
-      positions, tab);
-  return cudaGetLastError() == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+  const cudaError_t e = launch_pdl(rope_yarn_kernel, dim3(grid_for(work, 256)), dim3(256), 0,
+                                   (cudaStream_t)stream, (__nv_bfloat16*)x, rows, n_heads,
+                                   head_stride_elems, row_stride_elems, rope_offset_elems,
+                                   positions, tab);
+  return e == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
 }
 
 extern "C" xmla_status xmla_cache_append(void* pool, int64_t num_blocks, const int32_t* block_table,
@@ -168,8 +173,10 @@ extern "C" xmla_status xmla_cache_append(void* pool, int64_t num_blocks, const i
     tab = make_rope_table(rope_cfg);
   }
   const int64_t work = T * 72;
-  cache_append_kernel<<<grid_for(work, 256), 256, 0, (cudaStream_t)stream>>>(
-      (uint4*)pool, num_blocks, block_table, max_blocks, batch, seq_ids, positions,
-      (const uint4*)c_kv, (const uint4*)k_pe, T, status_dev, rope_cfg != nullptr ? 1 : 0, tab);
-  return cudaGetLastError() == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+  const cudaError_t e = launch_pdl(cache_append_kernel, dim3(grid_for(work, 256)), dim3(256), 0,
+                                   (cudaStream_t)stream, (uint4*)pool, num_blocks, block_table,
+                                   max_blocks, batch, seq_ids, positions, (const uint4*)c_kv,
+                                   (const uint4*)k_pe, T, status_dev, rope_cfg != nullptr ? 1 : 0,
+                                   tab);
+  return e == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
 }
