@@ -130,6 +130,25 @@ __device__ __forceinline__ void xpose_reduce32(float (&v)[32], int lane) {
   }
 }
 
+// The same over the 16 threads of one row parity (lane bits 0, 2, 3, 4; bit 1
+// kept): on return v[0] holds the reduction of value j = b0 + 2 b2 + 4 b3 + 8 b4.
+template <bool kMax>
+__device__ __forceinline__ void xpose_reduce16(float (&v)[16], int lane) {
+  constexpr int kMask[4] = {16, 8, 4, 1};
+#pragma unroll
+  for (int lv = 0; lv < 4; ++lv) {
+    const int w = 8 >> lv;  // values kept after this level
+    const bool upper = (lane & kMask[lv]) != 0;
+#pragma unroll
+    for (int k = 0; k < w; ++k) {
+      const float send = upper ? v[k] : v[k + w];
+      const float keep = upper ? v[k + w] : v[k];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, kMask[lv]);
+      v[k] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -382,22 +401,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
   } else {
     // ================================================================ softmax / epilogue
+    // S^T of a page is an M=64 accumulator: page token r sits in tensor-memory
+    // lane 32*(r/16) + r%16.  Each warp reads its quarter's 16 lanes with the
+    // 16x64b shape, which spreads them over all 32 threads: thread t holds token
+    // 8*(t&1) + (t>>2) of the quarter and the rows of one parity,
+    // n = pr + 2j (pr = (t>>1)&1, j < NR/2).
+    constexpr int kV = NR / 2;
+    constexpr int kH = kV / 2;
     const int tid = threadIdx.x - 32 * kSoftmaxWarp0;
     const int quarter = warp & 3;            // tensor-memory lane quarter this warp may access
-    const int tok = 16 * quarter + lane;     // token of the page held by this thread (lane < 16)
+    const int pr = (lane >> 1) & 1;
+    const int tok = 16 * quarter + 8 * (lane & 1) + (lane >> 2);  // token of the page
+    // after a transposed butterfly over the 16 threads of one parity, value 0
+    // of thread t belongs to row pr + 2*row_t
+    const int row_t = (lane & 1) + 2 * ((lane >> 2) & 1) + 4 * ((lane >> 3) & 1) + 8 * ((lane >> 4) & 1);
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quarter) << 16);
-    float l_part[NR];
+    float l_part[kV], mr[kV];  // per row of this thread: partial sum and running max
 #pragma unroll
-    for (int n = 0; n < NR; ++n) l_part[n] = 0.f;
-    // running maxima: a register copy for 32 rows, shared memory for 64
-    constexpr bool kRegM = NR == 32;
-    float mr[kRegM ? NR : 1];
-#pragma unroll
-    for (int n = 0; n < (kRegM ? NR : 1); ++n) mr[n] = -INFINITY;
-    auto mu = [&](int n) -> float {
-      if constexpr (kRegM) return mr[n];
-      else return m_used[n];
-    };
+    for (int j = 0; j < kV; ++j) {
+      l_part[j] = 0.f;
+      mr[j] = -INFINITY;
+    }
     const int64_t qpos0 = seqlen - p.q_len + j0;  // position of this CTA's first query
     bool ok = true;
     for (int i = 0; i < n_pages; ++i) {
@@ -406,13 +430,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                      p.wait_limit_ns);
       if (named_bar_or(1, kSoftmaxThreads, !ok)) { ok = false; break; }
       tc_fence_after();
-      float sv[NR];
+      float sv[kV];
 #pragma unroll
       for (int c = 0; c < NR / 32; ++c) {
-        float tmp[32];
-        tmem_ld32(t_lane + L::kColS + sb * NR + 32 * c, tmp);
+        float tmp[16];
+        tmem_ld16x64b_x16(t_lane + L::kColS + sb * NR + 32 * c, tmp);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) sv[32 * c + k] = tmp[k];
+        for (int k = 0; k < 16; ++k) sv[16 * c + k] = tmp[k];
       }
       tc_wait_ld();
       tc_fence_before();
@@ -421,19 +445,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const int64_t tpos = (p_begin + i) * kPage + tok;
       bool exceed = false;
 #pragma unroll
-      for (int n = 0; n < NR; ++n) {
-        const bool vis = lane < 16 && (n >> 5) < jn && tpos <= qpos0 + (n >> 5);
-        sv[n] = vis ? sv[n] : -INFINITY;
-        exceed |= sv[n] > mu(n) + kLazyMax;
+      for (int j = 0; j < kV; ++j) {
+        const int jr = j >> 4;  // query of row pr + 2j within this CTA
+        const bool vis = jr < jn && tpos <= qpos0 + jr;
+        sv[j] = vis ? sv[j] : -INFINITY;
+        exceed |= sv[j] > mr[j] + kLazyMax;
       }
       if (named_bar_or(1, kSoftmaxThreads, exceed)) {
 #pragma unroll
         for (int c = 0; c < NR / 32; ++c) {
-          float tmp[32];
+          float tmp[16];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) tmp[k] = sv[32 * c + k];
-          xpose_reduce32<true>(tmp, lane);
-          red[quarter * NR + 32 * c + lane] = tmp[0];
+          for (int k = 0; k < 16; ++k) tmp[k] = sv[16 * c + k];
+          xpose_reduce16<true>(tmp, lane);
+          red[quarter * NR + pr + 2 * (16 * c + row_t)] = tmp[0];
         }
         named_bar_sync(1, kSoftmaxThreads);
         if (tid < NR) {
@@ -468,13 +493,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           tc_wait_st();
         }
 #pragma unroll
-        for (int n = 0; n < NR; ++n) l_part[n] *= alpha_s[n];
+        for (int j = 0; j < kV; ++j) l_part[j] *= alpha_s[pr + 2 * j];
         if (tid < NR) m_used[tid] = m_next[tid];
         named_bar_sync(1, kSoftmaxThreads);
-        if constexpr (kRegM) {
 #pragma unroll
-          for (int n = 0; n < NR; ++n) mr[n] = m_used[n];
-        }
+        for (int j = 0; j < kV; ++j) mr[j] = m_used[pr + 2 * j];
       }
       if (i >= 2) {
         // P buffer (i & 1) is free once the PV of page i - 2 has completed
@@ -497,25 +520,32 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           dst[u] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      // P^T row of this token: NR bf16, written as 16-byte units in the swizzled
-      // MN-major layout the PV descriptor reads.
+      // probabilities (bf16-rounded, also summed in that precision)
+      float pb[kV];
+#pragma unroll
+      for (int j = 0; j < kV; ++j) {
+        const float pf = sv[j] == -INFINITY ? 0.f : ex2(sv[j] - mr[j]);
+        pb[j] = __bfloat162float(__float2bfloat16_rn(pf));
+        l_part[j] += pb[j];
+      }
+      // The thread pair (t, t^2) holds the two row parities of one token: swap
+      // halves so that each owns kV consecutive rows, then write its 16-byte
+      // units of the token's P^T row (MN-major, swizzled as the PV operand).
+      uint32_t w[kH];
+#pragma unroll
+      for (int k = 0; k < kH; ++k) {
+        const float own = pr == 0 ? pb[k] : pb[kH + k];
+        const float snd = pr == 0 ? pb[kH + k] : pb[k];
+        const float rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
+        w[k] = pr == 0 ? pack_bf16x2(own, rcv) : pack_bf16x2(rcv, own);
+      }
       uint8_t* prow = smem + L::kOffP + sb * L::kPBytes + tok * L::kPRow;
 #pragma unroll
-      for (int u = 0; u < NR / 8; ++u) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int n0 = 8 * u + 2 * e;
-          const float p0 = sv[n0] == -INFINITY ? 0.f : ex2(sv[n0] - mu(n0));
-          const float p1 = sv[n0 + 1] == -INFINITY ? 0.f : ex2(sv[n0 + 1] - mu(n0 + 1));
-          w[e] = pack_bf16x2(p0, p1);
-          const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
-          l_part[n0] += __low2float(hb);
-          l_part[n0 + 1] += __high2float(hb);
-        }
-        const int phys = NR == 32 ? (u ^ ((tok >> 1) & 3)) : (u ^ (tok & 7));
-        if (lane < 16)
-          *reinterpret_cast<uint4*>(prow + phys * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int u = 0; u < kH / 4; ++u) {
+        const int unit = pr * (kH / 4) + u;
+        const int phys = NR == 32 ? (unit ^ ((tok >> 1) & 3)) : (unit ^ (tok & 7));
+        *reinterpret_cast<uint4*>(prow + phys * 16) =
+            make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -550,11 +580,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
 #pragma unroll
       for (int c = 0; c < NR / 32; ++c) {
-        float tmp[32];
+        float tmp[16];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) tmp[k] = l_part[32 * c + k];
-        xpose_reduce32<false>(tmp, lane);
-        red[quarter * NR + 32 * c + lane] = tmp[0];
+        for (int k = 0; k < 16; ++k) tmp[k] = l_part[16 * c + k];
+        xpose_reduce16<false>(tmp, lane);
+        red[quarter * NR + pr + 2 * (16 * c + row_t)] = tmp[0];
       }
       named_bar_sync(1, kSoftmaxThreads);
       if (tid < nrows) {
