@@ -613,25 +613,43 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 // with pos_r = seqlens[b] - q_len + j (the q_len new tokens are the last cache
 // entries).  grid (32 heads, 8 blocks of 64 latent columns); 128 threads:
 // thread t owns 8 columns (t % 8) and 8 of the 128 nope dims (t / 8), holding
-// its 8 x 8 slice of W_UK in registers; partial sums meet in shared memory.
-// The column-block-0 CTAs also rotate the rope part.
+// its 8 x 8 slice of W_UK in registers (loaded before the wait on the kernel
+// launched just before, which it does not depend on); partial sums meet in
+// shared memory.  A ninth block per head rotates the rope part.
 constexpr int kAbsorbRows = 8;
 
-__global__ void __launch_bounds__(128) q_absorb_kernel(const __nv_bfloat16* __restrict__ q,
+// q and seqlens carry no __restrict__ so that their loads stay behind the
+// griddepcontrol.wait (a preceding kernel may have written them).
+__global__ void __launch_bounds__(128) q_absorb_kernel(const __nv_bfloat16* q,
                                                        const __nv_bfloat16* __restrict__ W_UK,
-                                                       const int32_t* __restrict__ seqlens,
+                                                       const int32_t* seqlens,
                                                        __nv_bfloat16* __restrict__ q_ext, int rows,
                                                        int q_len, float qscale,
                                                        const RopeTable tab) {
   __shared__ float sq[kAbsorbRows][kDNope];
   __shared__ float part[16][kAbsorbRows][64];
-  // q and the cache rows of this step may come from the kernels launched just
-  // before; the decode kernel relies on this wait (see its producer)
-  pdl_wait();
   pdl_launch_dependents();
   const int h = blockIdx.x;
   const int cb = blockIdx.y;
   const int t = threadIdx.x;
+  if (cb == kDLatent / 64) {
+    // q and the cache rows of this step may come from the kernels launched just
+    // before; every CTA waits (the decode kernel relies on it, see its producer)
+    pdl_wait();
+    constexpr int kPairs = kDRope / 2;
+    for (int e = t; e < rows * kPairs; e += blockDim.x) {
+      const int r = e / kPairs, i = e % kPairs;
+      const int64_t pos = (int64_t)seqlens[r / q_len] - q_len + (r % q_len);
+      const __nv_bfloat16* x = q + ((int64_t)r * kHeads + h) * kDQ + kDNope;
+      double y1, y2;
+      rope_pair((double)__bfloat162float(x[i]), (double)__bfloat162float(x[i + kPairs]), pos, i,
+                tab, &y1, &y2);
+      __nv_bfloat16* o = q_ext + ((int64_t)r * kHeads + h) * kDRow + kDLatent;
+      o[i] = __double2bfloat16(y1 * (double)qscale);
+      o[i + kPairs] = __double2bfloat16(y2 * (double)qscale);
+    }
+    return;
+  }
   const int c8 = t & 7;
   const int dg = t >> 3;
   float w[8][8];
@@ -646,6 +664,7 @@ __global__ void __launch_bounds__(128) q_absorb_kernel(const __nv_bfloat16* __re
       w[dd][2 * e + 1] = __high2float(pv[e]);
     }
   }
+  pdl_wait();
   for (int r0 = 0; r0 < rows; r0 += kAbsorbRows) {
     const int nr = min(kAbsorbRows, rows - r0);
     __syncthreads();
@@ -674,35 +693,29 @@ __global__ void __launch_bounds__(128) q_absorb_kernel(const __nv_bfloat16* __re
       q_ext[((int64_t)(r0 + r) * kHeads + h) * kDRow + cb * 64 + col] = __float2bfloat16_rn(s * qscale);
     }
   }
-  if (cb == 0) {
-    constexpr int kPairs = kDRope / 2;
-    for (int e = t; e < rows * kPairs; e += blockDim.x) {
-      const int r = e / kPairs, i = e % kPairs;
-      const int64_t pos = (int64_t)seqlens[r / q_len] - q_len + (r % q_len);
-      const __nv_bfloat16* x = q + ((int64_t)r * kHeads + h) * kDQ + kDNope;
-      double y1, y2;
-      rope_pair((double)__bfloat162float(x[i]), (double)__bfloat162float(x[i + kPairs]), pos, i,
-                tab, &y1, &y2);
-      __nv_bfloat16* o = q_ext + ((int64_t)r * kHeads + h) * kDRow + kDLatent;
-      o[i] = __double2bfloat16(y1 * (double)qscale);
-      o[i + kPairs] = __double2bfloat16(y2 * (double)qscale);
-    }
-  }
 }
 
 // ---------------------------------------------------------------- combine + W_UV
 
 // Cluster of 8 CTAs per (head h, chunk of up to kCombineRows output rows).
-// CTA `slice` owns latent dims [64 slice, 64 slice + 64): for every row it
-// merges the splits' partial O by their log-sum-exp weights, normalises, and
-// multiplies by the matching 64 rows of W_UV[h]; the 8 partial outputs of a
-// row are summed through distributed shared memory by the cluster's CTA 0.
+// CTA `slice` owns latent dims [64 slice, 64 slice + 64).  All rows of the
+// chunk are merged together: 16 groups of 16 threads (one float4 of the slice
+// each) are shared out over the rows, and a row's splits are dealt round-robin
+// over its groups, so one pass of loads covers the chunk.  Every split is
+// weighted by 2^(m_s - M) against the row's overall maximum M and the sum is
+// divided by L = sum_s l_s 2^(m_s - M).  The CTA then multiplies its merged
+// 64 dims by the matching 64 rows of W_UV[h] and sends each 16-column block of
+// that product to the CTA that owns the block (distributed shared memory); the
+// owner adds the 8 contributions and writes its 16 output columns.
 constexpr int kSlices = 8;
-constexpr int kSliceDims = kDLatent / kSlices;  // 64
+constexpr int kSliceDims = kDLatent / kSlices;        // 64
 constexpr int kCombineRows = 16;
 constexpr int kCombineThreads = 256;
-constexpr int kCombineGroups = kCombineThreads / 16;  // split rows read at once (16 threads x float4 each)
+constexpr int kCombineWarps = kCombineThreads / 32;
+constexpr int kCombineGroups = kCombineThreads / 16;  // 16 threads x float4 cover a split row's slice
 constexpr int kCombineDepth = 10;                     // split rows each thread keeps in flight
+constexpr int kStatDepth = 4;                         // (m, l) pairs each lane keeps in flight
+constexpr int kColsPerSlice = kDV / kSlices;          // 16
 
 // Online (max, sum-of-exp2) pair merge.
 __device__ __forceinline__ void lse_merge(float& m, float& l, float m2, float l2) {
@@ -712,16 +725,28 @@ __device__ __forceinline__ void lse_merge(float& m, float& l, float m2, float l2
   m = mx;
 }
 
-__global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThreads)
-    combine_uv_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThreads, 3)
+    combine_uv_kernel(const float* part_o, const float* part_ml,
                       const __nv_bfloat16* __restrict__ W_UV, __nv_bfloat16* __restrict__ out,
                       int rows, int q_len, int groups, int nsplit, int rows_per_cta) {
+  // part_o and part_ml are written by the kernel launched just before this one,
+  // which lets this grid start early: they carry no __restrict__, so their loads
+  // are not taken as invariant and stay behind the griddepcontrol.wait below.
   __shared__ __align__(16) __nv_bfloat16 w_s[kSliceDims][kDV];  // this slice's rows of W_UV[h]
-  __shared__ float wt_s[kMaxSplits];                             // split weights of one row
   __shared__ __align__(16) float4 acc_s[kCombineGroups][kSliceDims / 4];
-  __shared__ float o_s[kCombineRows][kSliceDims];
-  __shared__ float out_s[2][kCombineRows][kDV];
-  __shared__ float red_m[kCombineThreads / 32], red_l[kCombineThreads / 32];
+  __shared__ __align__(16) float o_s[kCombineRows][kSliceDims];
+  __shared__ __align__(16) float inbox[kSlices][kCombineRows][kColsPerSlice];  // by sender slice
+  __shared__ float stat_m[kCombineRows][kCombineWarps], stat_l[kCombineRows][kCombineWarps];
   cg::cluster_group cluster = cg::this_cluster();
   const int slice = (int)cluster.block_rank();
   const int cid = blockIdx.x / kSlices;
@@ -731,7 +756,11 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThread
   const int nr = min(kCombineRows, rows - r0);
   const int tid = threadIdx.x;
   const int lane = tid & 31;
+  const int warp = tid >> 5;
   pdl_launch_dependents();
+  // first half of the barrier that guarantees every CTA of the cluster runs
+  // before any of them writes into another's shared memory
+  cluster_arrive_relaxed();
   // W_UV does not depend on the decode kernel: stage it while that kernel finishes
   {
     const uint4* src = reinterpret_cast<const uint4*>(W_UV + ((int64_t)h * kDLatent + slice * kSliceDims) * kDV);
@@ -740,116 +769,146 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThread
     for (int e = 0; e < kSliceDims * kDV / 8 / kCombineThreads; ++e)
       dst[tid + kCombineThreads * e] = src[tid + kCombineThreads * e];
   }
-  pdl_wait();  // the split partials come from the decode kernel
 
-  const int q4 = tid & 15;  // float4 of the 64-dim slice
-  const int grp = tid >> 4;
-  for (int rr = 0; rr < nr; ++rr) {
+  // partial row of split 0 for chunk row rr; split s is s * rows_per_cta rows further
+  auto split0_row = [&](int rr) -> int64_t {
     const int r = r0 + rr;  // r = b*q_len + j
     const int b = r / q_len, j = r % q_len;
     const int ridx = j * kHeads + h;
-    const int g = ridx / rows_per_cta;
-    const int n = ridx % rows_per_cta;
-    const int64_t row0 = ((int64_t)b * groups + g) * nsplit * rows_per_cta + n;  // split 0's row
-    const float2* ml = reinterpret_cast<const float2*>(part_ml) + row0;
-    const float* po = part_o + row0 * kDLatent + slice * kSliceDims + 4 * q4;
-    const int64_t o_stride = (int64_t)rows_per_cta * kDLatent;
-    // first batch of O rows: issued before the log-sum-exp so both latencies overlap
-    float4 v[kCombineDepth];
+    return ((int64_t)b * groups + ridx / rows_per_cta) * nsplit * rows_per_cta + ridx % rows_per_cta;
+  };
+  const int q4 = tid & 15;  // float4 of the 64-dim slice
+  const int grp = tid >> 4;
+  const int gpr = max(1, kCombineGroups / nr);  // groups per row
+  const int my_rr = grp / gpr;
+  const int sub = grp % gpr;
+  const bool active = my_rr < nr;
+  const int64_t base = active ? split0_row(my_rr) : 0;
+  const float* po = part_o + base * kDLatent + slice * kSliceDims + 4 * q4;
+  const float* pm = part_ml + 2 * base;          // m of split s at pm[s * m_stride]
+  const int o_stride = rows_per_cta * kDLatent;  // floats between splits (nsplit * o_stride < 2^31)
+  const int m_stride = 2 * rows_per_cta;
+  const int wpr = max(1, kCombineWarps / nr);    // warps per row for the statistics
+
+  pdl_wait();  // the split partials come from the decode kernel
+
+  // first batch of this thread's split rows, issued before the row statistics
+  // so that both sets of loads are in flight together.  A split that saw no
+  // token has m = -inf (and l = 0); only m is needed to recognise it.
+  float4 v[kCombineDepth];
+  float ms[kCombineDepth];
 #pragma unroll
-    for (int k = 0; k < kCombineDepth; ++k) {
-      const int sidx = grp + kCombineGroups * k;
-      v[k] = sidx < nsplit ? *reinterpret_cast<const float4*>(po + sidx * o_stride)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    // global max M and sum L = sum_s l_s 2^(m_s - M) over the splits that saw tokens
-    float m = -INFINITY, l = 0.f;
-    for (int sidx = tid; sidx < nsplit; sidx += kCombineThreads) {
-      const float2 x = ml[(int64_t)sidx * rows_per_cta];
-      if (x.y > 0.f) lse_merge(m, l, x.x, x.y);
-    }
+  for (int k = 0; k < kCombineDepth; ++k) {
+    const int s = sub + gpr * k;
+    const bool in = active && s < nsplit;
+    v[k] = in ? *reinterpret_cast<const float4*>(po + s * o_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+    ms[k] = in ? pm[s * m_stride] : -INFINITY;
+  }
+
+  // row statistics: `wpr` warps share a row's splits (part p takes splits
+  // 32 p + lane, then every 32 wpr further); each warp reduces its share
+  {
+    const int part = warp % wpr;
+    for (int rr = warp / wpr; rr < nr; rr += kCombineWarps / wpr) {
+      const float2* rml = reinterpret_cast<const float2*>(part_ml) + split0_row(rr);
+      float m = -INFINITY, l = 0.f;
+      for (int s0 = 32 * part; s0 < nsplit; s0 += 32 * wpr * kStatDepth) {
+        float2 x[kStatDepth];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-      const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-      lse_merge(m, l, m2, l2);
-    }
-    if (lane == 0) { red_m[tid >> 5] = m; red_l[tid >> 5] = l; }
-    __syncthreads();
-    m = red_m[0];
-    l = red_l[0];
+        for (int k = 0; k < kStatDepth; ++k) {
+          const int s = s0 + lane + 32 * wpr * k;
+          x[k] = s < nsplit ? rml[(int64_t)s * rows_per_cta] : make_float2(-INFINITY, 0.f);
+        }
 #pragma unroll
-    for (int w = 1; w < kCombineThreads / 32; ++w) lse_merge(m, l, red_m[w], red_l[w]);
-    for (int sidx = tid; sidx < nsplit; sidx += kCombineThreads) {
-      const float2 x = ml[(int64_t)sidx * rows_per_cta];
-      wt_s[sidx] = x.y > 0.f ? ex2(x.x - m) : 0.f;
+        for (int k = 0; k < kStatDepth; ++k)
+          if (x[k].y > 0.f) lse_merge(m, l, x[k].x, x[k].y);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
+        lse_merge(m, l, m2, l2);
+      }
+      if (lane == 0) {
+        stat_m[rr][part] = m;
+        stat_l[rr][part] = l;
+      }
     }
-    __syncthreads();
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0;; s0 += kCombineGroups * kCombineDepth) {
+  }
+  __syncthreads();
+
+  // weighted sum of this thread's split rows (the partial O of a split that saw
+  // no token was never written: it is skipped, not multiplied by zero)
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (active) {
+    float M = stat_m[my_rr][0];
+    for (int p = 1; p < wpr; ++p) M = fmaxf(M, stat_m[my_rr][p]);
+    for (int k0 = 0;; k0 += kCombineDepth) {
 #pragma unroll
       for (int k = 0; k < kCombineDepth; ++k) {
-        const int sidx = s0 + grp + kCombineGroups * k;
-        const float wgt = sidx < nsplit ? wt_s[sidx] : 0.f;
-        if (wgt != 0.f) {
+        if (ms[k] != -INFINITY) {
+          const float wgt = ex2(ms[k] - M);
           acc.x = fmaf(wgt, v[k].x, acc.x);
           acc.y = fmaf(wgt, v[k].y, acc.y);
           acc.z = fmaf(wgt, v[k].z, acc.z);
           acc.w = fmaf(wgt, v[k].w, acc.w);
         }
       }
-      const int s1 = s0 + kCombineGroups * kCombineDepth;
-      if (s1 >= nsplit) break;
+      const int k1 = k0 + kCombineDepth;
+      if (sub + gpr * k1 >= nsplit) break;
 #pragma unroll
       for (int k = 0; k < kCombineDepth; ++k) {
-        const int sidx = s1 + grp + kCombineGroups * k;
-        v[k] = sidx < nsplit ? *reinterpret_cast<const float4*>(po + sidx * o_stride)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int s = sub + gpr * (k1 + k);
+        const bool in = s < nsplit;
+        v[k] = in ? *reinterpret_cast<const float4*>(po + s * o_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+        ms[k] = in ? pm[s * m_stride] : -INFINITY;
       }
     }
-    acc_s[grp][q4] = acc;
-    __syncthreads();
-    if (tid < kSliceDims) {
-      const float* a = reinterpret_cast<const float*>(&acc_s[0][0]);
-      float t = 0.f;
-#pragma unroll
-      for (int k = 0; k < kCombineGroups; ++k) t += a[k * kSliceDims + tid];
-      o_s[rr][tid] = l > 0.f ? t / l : 0.f;
-    }
-    __syncthreads();
   }
+  acc_s[grp][q4] = acc;
+  __syncthreads();
+  for (int e = tid; e < nr * kSliceDims; e += kCombineThreads) {
+    const int rr = e / kSliceDims, d = e % kSliceDims;
+    float M = stat_m[rr][0];
+    for (int p = 1; p < wpr; ++p) M = fmaxf(M, stat_m[rr][p]);
+    float L = 0.f;
+    for (int p = 0; p < wpr; ++p)
+      if (stat_l[rr][p] > 0.f) L += stat_l[rr][p] * ex2(stat_m[rr][p] - M);
+    const float* a = reinterpret_cast<const float*>(&acc_s[rr * gpr][0]) + d;
+    float t = 0.f;
+    for (int g = 0; g < gpr; ++g) t += a[g * kSliceDims];
+    o_s[rr][d] = L > 0.f ? t / L : 0.f;
+  }
+  __syncthreads();
 
-  // partial out[r][v] = sum over this slice's 64 latent dims of o[r][c] W_UV[h][c][v];
-  // the two halves of the CTA take 32 dims each
+  // slice product: sum over the slice's 64 latent dims c of o[r][c] W_UV[h][c][v]
+  // for the column pair (2 vp, 2 vp + 1), sent to the CTA owning that column block
+  cluster_wait_acquire();  // every CTA of the cluster is running
   {
-    const int v = tid & (kDV - 1);
-    const int hf = tid >> 7;
-    float acc[kCombineRows];
-#pragma unroll
-    for (int rr = 0; rr < kCombineRows; ++rr) acc[rr] = 0.f;
-#pragma unroll 8
-    for (int c = 32 * hf; c < 32 * hf + 32; ++c) {
-      const float wcv = __bfloat162float(w_s[c][v]);
-#pragma unroll
-      for (int rr = 0; rr < kCombineRows; ++rr) acc[rr] = fmaf(o_s[rr][c], wcv, acc[rr]);
-    }
-#pragma unroll
-    for (int rr = 0; rr < kCombineRows; ++rr) out_s[hf][rr][v] = acc[rr];
-  }
-  cluster.sync();
-  if (slice == 0) {
-    for (int e = tid; e < nr * kDV; e += blockDim.x) {
-      const int rr = e / kDV, v = e % kDV;
-      float t = 0.f;
-#pragma unroll
-      for (int k = 0; k < kSlices; ++k) {
-        const float* peer = cluster.map_shared_rank(&out_s[0][0][0], k);
-        t += peer[rr * kDV + v] + peer[kCombineRows * kDV + rr * kDV + v];
+    const int vp = tid & (kDV / 2 - 1);
+    const int owner = (2 * vp) / kColsPerSlice;
+    float* dst = cluster.map_shared_rank(&inbox[slice][0][0], owner);
+    for (int rr = tid / (kDV / 2); rr < nr; rr += kCombineThreads / (kDV / 2)) {
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll 16
+      for (int c = 0; c < kSliceDims; ++c) {
+        const float2 w = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&w_s[c][0])[vp]);
+        const float x = o_s[rr][c];
+        a0 = fmaf(x, w.x, a0);
+        a1 = fmaf(x, w.y, a1);
       }
-      out[((int64_t)(r0 + rr) * kHeads + h) * kDV + v] = __float2bfloat16_rn(t);
+      *reinterpret_cast<float2*>(dst + rr * kColsPerSlice + (2 * vp) % kColsPerSlice) = make_float2(a0, a1);
     }
   }
-  cluster.sync();  // keep every CTA's shared memory alive until CTA 0 has read it
+  cluster_arrive_release();
+  cluster_wait_acquire();  // all 8 contributions have landed in this CTA's inbox
+  if (tid < nr * kColsPerSlice) {
+    const int rr = tid / kColsPerSlice, c = tid % kColsPerSlice;
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < kSlices; ++k) t += inbox[k][rr][c];
+    out[((int64_t)(r0 + rr) * kHeads + h) * kDV + slice * kColsPerSlice + c] = __float2bfloat16_rn(t);
+  }
 }
 
 // ---------------------------------------------------------------- self-test kernel
@@ -1028,7 +1087,7 @@ extern "C" xmla_status xmla_decode_profiled(const xmla_yarn_cfg* cfg, const void
   // Every kernel of the chain waits (griddepcontrol.wait) for its predecessor
   // before reading anything a kernel of this step may have written, so once
   // q_absorb completes all earlier work on the stream has landed.
-  if (launch_pdl(q_absorb_kernel, dim3(kHeads, kDLatent / 64), dim3(128), 0, st,
+  if (launch_pdl(q_absorb_kernel, dim3(kHeads, kDLatent / 64 + 1), dim3(128), 0, st,
                  (const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext, rows, q_len,
                  qscale, make_rope_table(cfg)) != cudaSuccess)
     return XMLA_ERR_CUDA;

@@ -16,10 +16,14 @@ namespace xmla {
 
 // One thread per (vector, pair).  Angle formed in float64 from the exact
 // integer position; the rotated pair is rounded once to bf16.
-__global__ void __launch_bounds__(256) rope_yarn_kernel(__nv_bfloat16* __restrict__ x, int64_t rows,
+//
+// Inputs that the kernel launched just before may write carry no __restrict__
+// (here and in the kernels below): such loads are then not taken as invariant
+// and cannot be hoisted above the griddepcontrol.wait that orders them.
+__global__ void __launch_bounds__(256) rope_yarn_kernel(__nv_bfloat16* x, int64_t rows,
                                                         int32_t n_heads, int64_t head_stride,
                                                         int64_t row_stride, int32_t offset,
-                                                        const int64_t* __restrict__ positions,
+                                                        const int64_t* positions,
                                                         const RopeTable tab) {
   pdl_wait();  // inputs may come from the kernel launched just before
   pdl_launch_dependents();
@@ -46,10 +50,9 @@ __global__ void __launch_bounds__(256) rope_yarn_kernel(__nv_bfloat16* __restric
 // the four pairs (4r .. 4r+3, 4r+32 .. 4r+35) at the row's position and
 // stores them.
 __global__ void __launch_bounds__(256) cache_append_kernel(
-    uint4* __restrict__ pool, int64_t num_blocks, const int32_t* __restrict__ block_table,
-    int32_t max_blocks, int32_t batch, const int32_t* __restrict__ seq_ids,
-    const int64_t* __restrict__ positions, const uint4* __restrict__ c_kv,
-    const uint4* __restrict__ k_pe, int64_t T, int32_t* status, int rotate, const RopeTable tab) {
+    uint4* pool, int64_t num_blocks, const int32_t* block_table, int32_t max_blocks,
+    int32_t batch, const int32_t* seq_ids, const int64_t* positions, const uint4* c_kv,
+    const uint4* k_pe, int64_t T, int32_t* status, int rotate, const RopeTable tab) {
   pdl_wait();  // inputs may come from the kernel launched just before
   pdl_launch_dependents();
   constexpr int kLatPieces = kDLatent * 2 / 16;  // 64
