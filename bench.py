@@ -387,7 +387,8 @@ def run_xmla(args, wl):
     ksha = hashlib.sha256(open(os.path.join(ROOT, "mla_latent_kv_yarn_b200", "csrc",
                                             "mla_decode.cu"), "rb").read()).hexdigest()
     traffic = traffic_record(ksha, wl.name)
-    launches = 4 * wl.layers * args.steps
+    # per layer and step: prologue (append + q absorb), split-K attention, combine
+    launches = 3 * wl.layers * args.steps
 
     if rank == 0:
         line = {

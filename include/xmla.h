@@ -193,6 +193,27 @@ xmla_status xmla_decode_profiled(const xmla_yarn_cfg* cfg, const void* q, const 
                                  int32_t* status_dev, void* out, void* stream, void* attn_start,
                                  void* attn_stop);
 
+/* One decode step ([P5] MLA section; [P1] sections 一 and 二): append the
+ * step's T new token rows to the cache, then attend.  The result is that of
+ *   xmla_cache_append(pool, num_blocks, block_table, max_blocks, batch, seq_ids,
+ *                     positions, c_kv, k_pe, cfg, T, status_dev, stream);
+ *   xmla_decode_profiled(cfg, q, ..., attn_start, attn_stop);
+ * (k_pe is raw and is rotated with cfg at positions[i]), but the append runs
+ * inside the first kernel of the decode chain, beside the query absorb, which
+ * saves one kernel boundary.  Arguments as in those two calls; T >= 0 (T == 0
+ * appends nothing); c_kv and k_pe 16-byte aligned.  A new row must not share
+ * its cache slot with another row of the same call.  Errors: the union of
+ * theirs. */
+xmla_status xmla_decode_step(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
+                             const void* W_UV, void* pool, int64_t num_blocks,
+                             const int32_t* block_table, int32_t max_blocks,
+                             const int32_t* seqlens, int32_t batch, int32_t q_len,
+                             int64_t max_seqlen, const int32_t* seq_ids, const int64_t* positions,
+                             const void* c_kv, const void* k_pe, int64_t T, float softmax_scale,
+                             int32_t num_splits, void* workspace, size_t workspace_bytes,
+                             int32_t* status_dev, void* out, void* stream, void* attn_start,
+                             void* attn_stop);
+
 /* Size in bytes of the fixed device scratch used by xmla_decode_noalloc. */
 #define XMLA_NOALLOC_SCRATCH_BYTES (32u << 20)
 

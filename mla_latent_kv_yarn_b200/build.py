@@ -15,8 +15,9 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libxmla.so")
-SOURCES = ["rope_append.cu", "mla_decode.cu"]
-HEADERS = ["xmla_device.cuh", os.path.join("..", "..", "include", "xmla.h")]
+SOURCES = ["rope_append.cu", "mla_decode.cu", "absorb_combine.cu", "xmla_api.cu"]
+HEADERS = ["xmla_device.cuh", "yarn.cuh", "append.cuh", "decode_chain.h",
+           os.path.join("..", "..", "include", "xmla.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -1,0 +1,383 @@
+// The two small kernels around the split-K attention of a decode call:
+// q absorb (optionally fused with the step's cache append) before it, and the
+// split merge with the W_UV product after it.
+//
+// [P5] "mHC+MLA+MTP 是什么？拆开给 Agent 用的百亿 MoE", section "MLA：256K 上下文的
+//      '内存革命'": kv_b_proj maps the 512-dim latent to 32 heads x (128 K_nope +
+//      128 V); the absorbed form applies its K half (W_UK) to the query and its V
+//      half (W_UV) to the probability-weighted latent sum.
+// [P1] "256K 长上下文真能本地用：Xing4.0 原生长上下文的工程代价拆解", section 一: q_pe
+//      is rotated by YaRN RoPE at the query's position.
+#include <cooperative_groups.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "append.cuh"
+#include "decode_chain.h"
+
+namespace cg = cooperative_groups;
+
+namespace xmla {
+
+// ---------------------------------------------------------------- q absorb
+
+// q_ext[r, h] = qscale * [W_UK[h]^T q_nope[r, h] | rope(q_pe[r, h], pos_r)], r = b*q_len + j,
+// with pos_r = seqlens[b] - q_len + j (the q_len new tokens are the last cache
+// entries).  Blocks (32 heads x 8 blocks of 64 latent columns) of 128 threads:
+// thread t owns 8 columns (t % 8) and 8 of the 128 nope dims (t / 8), holding
+// its 8 x 8 slice of W_UK in registers (loaded before the wait on the kernel
+// launched just before, which it does not depend on); partial sums meet in
+// shared memory.  A ninth block per head rotates the rope part.
+constexpr int kAbsorbRows = 8;
+constexpr int kAbsorbThreads = 128;
+constexpr int kAbsorbBlocks = kHeads * (kDLatent / 64 + 1);
+
+// Block (h, cb) of the absorb; cb == 8 is the rope block.  Every block waits
+// (griddepcontrol.wait) before reading q or seqlens: a preceding kernel may
+// have written them, and the split-K kernel relies on that wait (its producer
+// reads cache rows appended by the kernel before this one).
+__device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat16* q,
+                                               const __nv_bfloat16* __restrict__ W_UK,
+                                               const int32_t* seqlens,
+                                               __nv_bfloat16* __restrict__ q_ext, int rows,
+                                               int q_len, float qscale, const RopeTable& tab) {
+  __shared__ float sq[kAbsorbRows][kDNope];
+  __shared__ float part[16][kAbsorbRows][64];
+  const int t = threadIdx.x;
+  if (cb == kDLatent / 64) {
+    pdl_wait();
+    constexpr int kPairs = kDRope / 2;
+    for (int e = t; e < rows * kPairs; e += kAbsorbThreads) {
+      const int r = e / kPairs, i = e % kPairs;
+      const int64_t pos = (int64_t)seqlens[r / q_len] - q_len + (r % q_len);
+      const __nv_bfloat16* x = q + ((int64_t)r * kHeads + h) * kDQ + kDNope;
+      double y1, y2;
+      rope_pair((double)__bfloat162float(x[i]), (double)__bfloat162float(x[i + kPairs]), pos, i,
+                tab, &y1, &y2);
+      __nv_bfloat16* o = q_ext + ((int64_t)r * kHeads + h) * kDRow + kDLatent;
+      o[i] = __double2bfloat16(y1 * (double)qscale);
+      o[i + kPairs] = __double2bfloat16(y2 * (double)qscale);
+    }
+    return;
+  }
+  const int c8 = t & 7;
+  const int dg = t >> 3;
+  float w[8][8];
+#pragma unroll
+  for (int dd = 0; dd < 8; ++dd) {
+    const uint4 v = *reinterpret_cast<const uint4*>(
+        W_UK + ((int64_t)h * kDNope + dg * 8 + dd) * kDLatent + cb * 64 + c8 * 8);
+    const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      w[dd][2 * e] = __low2float(pv[e]);
+      w[dd][2 * e + 1] = __high2float(pv[e]);
+    }
+  }
+  pdl_wait();
+  for (int r0 = 0; r0 < rows; r0 += kAbsorbRows) {
+    const int nr = min(kAbsorbRows, rows - r0);
+    __syncthreads();
+    for (int e = t; e < nr * kDNope; e += kAbsorbThreads) {
+      const int r = e / kDNope, d = e % kDNope;
+      sq[r][d] = __bfloat162float(q[((int64_t)(r0 + r) * kHeads + h) * kDQ + d]);
+    }
+    __syncthreads();
+    for (int r = 0; r < nr; ++r) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int dd = 0; dd < 8; ++dd) {
+        const float x = sq[r][dg * 8 + dd];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = fmaf(x, w[dd][k], acc[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) part[dg][r][c8 * 8 + k] = acc[k];
+    }
+    __syncthreads();
+    for (int o = t; o < nr * 64; o += kAbsorbThreads) {
+      const int r = o / 64, col = o % 64;
+      float s = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) s += part[k][r][col];
+      q_ext[((int64_t)(r0 + r) * kHeads + h) * kDRow + cb * 64 + col] = __float2bfloat16_rn(s * qscale);
+    }
+  }
+}
+
+// q and seqlens carry no __restrict__ so that their loads stay behind the
+// griddepcontrol.wait (a preceding kernel may have written them).
+__global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
+    const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
+    __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, float qscale, const RopeTable tab) {
+  pdl_launch_dependents();
+  q_absorb_block(blockIdx.x % kHeads, blockIdx.x / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
+                 qscale, tab);
+}
+
+// The first kernel of a decode step: the absorb blocks above, followed by
+// blocks that append the step's new cache rows (one thread per 16-byte piece).
+// Both halves only wait for the kernel launched before this one, so the
+// append and the absorb run side by side.
+__global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
+    const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
+    __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, float qscale, const RopeTable q_tab,
+    const AppendArgs ap, const RopeTable k_tab) {
+  pdl_launch_dependents();
+  if (blockIdx.x < kAbsorbBlocks) {
+    q_absorb_block(blockIdx.x % kHeads, blockIdx.x / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
+                   qscale, q_tab);
+    return;
+  }
+  pdl_wait();
+  const int64_t total = ap.T * kRowPieces;
+  const int64_t idx = (int64_t)(blockIdx.x - kAbsorbBlocks) * kAbsorbThreads + threadIdx.x;
+  if (idx < total)
+    append_piece(idx, ap.pool, ap.num_blocks, ap.block_table, ap.max_blocks, ap.batch, ap.seq_ids,
+                 ap.positions, ap.c_kv, ap.k_pe, ap.status, ap.rotate, k_tab);
+}
+
+cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
+                            const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
+                            float qscale, const RopeTable& tab, cudaStream_t st) {
+  return launch_pdl(q_absorb_kernel, dim3(kAbsorbBlocks), dim3(kAbsorbThreads), 0, st, q, W_UK,
+                    seqlens, q_ext, rows, q_len, qscale, tab);
+}
+
+cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
+                                 const int32_t* seqlens, __nv_bfloat16* q_ext, int rows,
+                                 int q_len, float qscale, const RopeTable& q_tab,
+                                 const AppendArgs& ap, const RopeTable& k_tab, cudaStream_t st) {
+  const int64_t append_blocks = (ap.T * kRowPieces + kAbsorbThreads - 1) / kAbsorbThreads;
+  if (append_blocks > (1 << 20)) return cudaErrorInvalidValue;
+  return launch_pdl(step_prologue_kernel, dim3((unsigned)(kAbsorbBlocks + append_blocks)),
+                    dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, qscale,
+                    q_tab, ap, k_tab);
+}
+
+// ---------------------------------------------------------------- combine + W_UV
+
+// Cluster of 8 CTAs per (head h, chunk of up to kCombineRows output rows).
+// CTA `slice` owns latent dims [64 slice, 64 slice + 64).  All rows of the
+// chunk are merged together: 16 groups of 16 threads (one float4 of the slice
+// each) are shared out over the rows, and a row's splits are dealt round-robin
+// over its groups, so one pass of loads covers the chunk.  Every split is
+// weighted by 2^(m_s - M) against the row's overall maximum M and the sum is
+// divided by L = sum_s l_s 2^(m_s - M).  The CTA then multiplies its merged
+// 64 dims by the matching 64 rows of W_UV[h] and sends each 16-column block of
+// that product to the CTA that owns the block (distributed shared memory); the
+// owner adds the 8 contributions and writes its 16 output columns.
+constexpr int kSlices = 8;
+constexpr int kSliceDims = kDLatent / kSlices;        // 64
+constexpr int kCombineRows = 16;
+constexpr int kCombineThreads = 256;
+constexpr int kCombineWarps = kCombineThreads / 32;
+constexpr int kCombineGroups = kCombineThreads / 16;  // 16 threads x float4 cover a split row's slice
+constexpr int kCombineDepth = 10;                     // split rows each thread keeps in flight
+constexpr int kStatDepth = 4;                         // (m, l) pairs each lane keeps in flight
+constexpr int kColsPerSlice = kDV / kSlices;          // 16
+
+// Online (max, sum-of-exp2) pair merge.
+__device__ __forceinline__ void lse_merge(float& m, float& l, float m2, float l2) {
+  const float mx = fmaxf(m, m2);
+  if (mx == -INFINITY) return;
+  l = l * ex2(m - mx) + l2 * ex2(m2 - mx);
+  m = mx;
+}
+
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThreads, 3)
+    combine_uv_kernel(const float* part_o, const float* part_ml,
+                      const __nv_bfloat16* __restrict__ W_UV, __nv_bfloat16* __restrict__ out,
+                      int rows, int q_len, int groups, int nsplit, int rows_per_cta) {
+  // part_o and part_ml are written by the kernel launched just before this one,
+  // which lets this grid start early: they carry no __restrict__, so their loads
+  // are not taken as invariant and stay behind the griddepcontrol.wait below.
+  __shared__ __align__(16) __nv_bfloat16 w_s[kSliceDims][kDV];  // this slice's rows of W_UV[h]
+  __shared__ __align__(16) float4 acc_s[kCombineGroups][kSliceDims / 4];
+  __shared__ __align__(16) float o_s[kCombineRows][kSliceDims];
+  __shared__ __align__(16) float inbox[kSlices][kCombineRows][kColsPerSlice];  // by sender slice
+  __shared__ float stat_m[kCombineRows][kCombineWarps], stat_l[kCombineRows][kCombineWarps];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int slice = (int)cluster.block_rank();
+  const int cid = blockIdx.x / kSlices;
+  const int h = cid % kHeads;
+  const int chunk = cid / kHeads;
+  const int r0 = chunk * kCombineRows;
+  const int nr = min(kCombineRows, rows - r0);
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  pdl_launch_dependents();
+  // first half of the barrier that guarantees every CTA of the cluster runs
+  // before any of them writes into another's shared memory
+  cluster_arrive_relaxed();
+  // W_UV does not depend on the decode kernel: stage it while that kernel finishes
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(W_UV + ((int64_t)h * kDLatent + slice * kSliceDims) * kDV);
+    uint4* dst = reinterpret_cast<uint4*>(&w_s[0][0]);
+#pragma unroll
+    for (int e = 0; e < kSliceDims * kDV / 8 / kCombineThreads; ++e)
+      dst[tid + kCombineThreads * e] = src[tid + kCombineThreads * e];
+  }
+
+  // partial row of split 0 for chunk row rr; split s is s * rows_per_cta rows further
+  auto split0_row = [&](int rr) -> int64_t {
+    const int r = r0 + rr;  // r = b*q_len + j
+    const int b = r / q_len, j = r % q_len;
+    const int ridx = j * kHeads + h;
+    return ((int64_t)b * groups + ridx / rows_per_cta) * nsplit * rows_per_cta + ridx % rows_per_cta;
+  };
+  const int q4 = tid & 15;  // float4 of the 64-dim slice
+  const int grp = tid >> 4;
+  const int gpr = max(1, kCombineGroups / nr);  // groups per row
+  const int my_rr = grp / gpr;
+  const int sub = grp % gpr;
+  const bool active = my_rr < nr;
+  const int64_t base = active ? split0_row(my_rr) : 0;
+  const float* po = part_o + base * kDLatent + slice * kSliceDims + 4 * q4;
+  const float* pm = part_ml + 2 * base;          // m of split s at pm[s * m_stride]
+  const int o_stride = rows_per_cta * kDLatent;  // floats between splits (nsplit * o_stride < 2^31)
+  const int m_stride = 2 * rows_per_cta;
+  const int wpr = max(1, kCombineWarps / nr);    // warps per row for the statistics
+
+  pdl_wait();  // the split partials come from the decode kernel
+
+  // first batch of this thread's split rows, issued before the row statistics
+  // so that both sets of loads are in flight together.  A split that saw no
+  // token has m = -inf (and l = 0); only m is needed to recognise it.
+  float4 v[kCombineDepth];
+  float ms[kCombineDepth];
+#pragma unroll
+  for (int k = 0; k < kCombineDepth; ++k) {
+    const int s = sub + gpr * k;
+    const bool in = active && s < nsplit;
+    v[k] = in ? *reinterpret_cast<const float4*>(po + s * o_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+    ms[k] = in ? pm[s * m_stride] : -INFINITY;
+  }
+
+  // row statistics: `wpr` warps share a row's splits (part p takes splits
+  // 32 p + lane, then every 32 wpr further); each warp reduces its share
+  {
+    const int part = warp % wpr;
+    for (int rr = warp / wpr; rr < nr; rr += kCombineWarps / wpr) {
+      const float2* rml = reinterpret_cast<const float2*>(part_ml) + split0_row(rr);
+      float m = -INFINITY, l = 0.f;
+      for (int s0 = 32 * part; s0 < nsplit; s0 += 32 * wpr * kStatDepth) {
+        float2 x[kStatDepth];
+#pragma unroll
+        for (int k = 0; k < kStatDepth; ++k) {
+          const int s = s0 + lane + 32 * wpr * k;
+          x[k] = s < nsplit ? rml[(int64_t)s * rows_per_cta] : make_float2(-INFINITY, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < kStatDepth; ++k)
+          if (x[k].y > 0.f) lse_merge(m, l, x[k].x, x[k].y);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
+        lse_merge(m, l, m2, l2);
+      }
+      if (lane == 0) {
+        stat_m[rr][part] = m;
+        stat_l[rr][part] = l;
+      }
+    }
+  }
+  __syncthreads();
+
+  // weighted sum of this thread's split rows (the partial O of a split that saw
+  // no token was never written: it is skipped, not multiplied by zero)
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (active) {
+    float M = stat_m[my_rr][0];
+    for (int p = 1; p < wpr; ++p) M = fmaxf(M, stat_m[my_rr][p]);
+    for (int k0 = 0;; k0 += kCombineDepth) {
+#pragma unroll
+      for (int k = 0; k < kCombineDepth; ++k) {
+        if (ms[k] != -INFINITY) {
+          const float wgt = ex2(ms[k] - M);
+          acc.x = fmaf(wgt, v[k].x, acc.x);
+          acc.y = fmaf(wgt, v[k].y, acc.y);
+          acc.z = fmaf(wgt, v[k].z, acc.z);
+          acc.w = fmaf(wgt, v[k].w, acc.w);
+        }
+      }
+      const int k1 = k0 + kCombineDepth;
+      if (sub + gpr * k1 >= nsplit) break;
+#pragma unroll
+      for (int k = 0; k < kCombineDepth; ++k) {
+        const int s = sub + gpr * (k1 + k);
+        const bool in = s < nsplit;
+        v[k] = in ? *reinterpret_cast<const float4*>(po + s * o_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+        ms[k] = in ? pm[s * m_stride] : -INFINITY;
+      }
+    }
+  }
+  acc_s[grp][q4] = acc;
+  __syncthreads();
+  for (int e = tid; e < nr * kSliceDims; e += kCombineThreads) {
+    const int rr = e / kSliceDims, d = e % kSliceDims;
+    float M = stat_m[rr][0];
+    for (int p = 1; p < wpr; ++p) M = fmaxf(M, stat_m[rr][p]);
+    float L = 0.f;
+    for (int p = 0; p < wpr; ++p)
+      if (stat_l[rr][p] > 0.f) L += stat_l[rr][p] * ex2(stat_m[rr][p] - M);
+    const float* a = reinterpret_cast<const float*>(&acc_s[rr * gpr][0]) + d;
+    float t = 0.f;
+    for (int g = 0; g < gpr; ++g) t += a[g * kSliceDims];
+    o_s[rr][d] = L > 0.f ? t / L : 0.f;
+  }
+  __syncthreads();
+
+  // slice product: sum over the slice's 64 latent dims c of o[r][c] W_UV[h][c][v]
+  // for the column pair (2 vp, 2 vp + 1), sent to the CTA owning that column block
+  cluster_wait_acquire();  // every CTA of the cluster is running
+  {
+    const int vp = tid & (kDV / 2 - 1);
+    const int owner = (2 * vp) / kColsPerSlice;
+    float* dst = cluster.map_shared_rank(&inbox[slice][0][0], owner);
+    for (int rr = tid / (kDV / 2); rr < nr; rr += kCombineThreads / (kDV / 2)) {
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll 16
+      for (int c = 0; c < kSliceDims; ++c) {
+        const float2 w = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&w_s[c][0])[vp]);
+        const float x = o_s[rr][c];
+        a0 = fmaf(x, w.x, a0);
+        a1 = fmaf(x, w.y, a1);
+      }
+      *reinterpret_cast<float2*>(dst + rr * kColsPerSlice + (2 * vp) % kColsPerSlice) = make_float2(a0, a1);
+    }
+  }
+  cluster_arrive_release();
+  cluster_wait_acquire();  // all 8 contributions have landed in this CTA's inbox
+  if (tid < nr * kColsPerSlice) {
+    const int rr = tid / kColsPerSlice, c = tid % kColsPerSlice;
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < kSlices; ++k) t += inbox[k][rr][c];
+    out[((int64_t)(r0 + rr) * kHeads + h) * kDV + slice * kColsPerSlice + c] = __float2bfloat16_rn(t);
+  }
+}
+
+cudaError_t launch_combine(const float* part_o, const float* part_ml, const __nv_bfloat16* W_UV,
+                           __nv_bfloat16* out, int rows, int q_len, int groups, int nsplit,
+                           int rows_per_cta, cudaStream_t st) {
+  const int chunks = (rows + kCombineRows - 1) / kCombineRows;
+  return launch_pdl(combine_uv_kernel, dim3(kSlices * kHeads * chunks), dim3(kCombineThreads), 0,
+                    st, part_o, part_ml, W_UV, out, rows, q_len, groups, nsplit, rows_per_cta);
+}
+
+}  // namespace xmla

@@ -1,0 +1,82 @@
+// Host-side interface between the kernels of one decode call and the C ABI.
+//
+// A decode call runs three kernels on one stream, chained with programmatic
+// dependent launch (each waits with griddepcontrol.wait for its predecessor
+// before reading anything that predecessor may write):
+//   q_absorb   (absorb_combine.cu)  q_ext = c * [W_UK^T q_nope | rope(q_pe)]
+//   split-K    (mla_decode.cu)      per-split (m, l, O) over the paged cache
+//   combine    (absorb_combine.cu)  log-sum-exp merge of the splits, then W_UV
+// The decode-step entry fuses the cache append into the first kernel
+// (step_prologue_kernel in absorb_combine.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "xmla_device.cuh"
+#include "yarn.cuh"
+
+namespace xmla {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxSplits = 1024;
+
+// Arguments of the split-K attention kernel.  Partial results are laid out
+// per work item (sequence b, row group g, split s) in that order.
+struct DecodeParams {
+  const int32_t* block_table;
+  const int32_t* seqlens;
+  float* part_o;   // [items, NR, 512] unnormalised O of each split
+  float* part_ml;  // [items, NR, 2] running max m (log2 units) and sum l
+  int32_t* status;
+  int64_t num_blocks;
+  int64_t max_seqlen;
+  uint64_t wait_limit_ns;
+  int32_t max_blocks;
+  int32_t batch;
+  int32_t q_len;
+  int32_t groups;
+  int32_t nsplit;
+};
+
+// Split-K attention over `items` work items; nr = rows per CTA (32 or 64).
+// pool_map: 576-column rows of the cache pool, box 64 x 64; q_map: rows of
+// q_ext, box 64 x nr (both 128-byte swizzled).
+cudaError_t launch_split_kv(int nr, const CUtensorMap& pool_map, const CUtensorMap& q_map,
+                            const DecodeParams& dp, int64_t items, cudaStream_t st);
+
+// q_ext[r, h] for rows r = b*q_len + j; qscale = softmax scale * log2 e.
+cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
+                            const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
+                            float qscale, const RopeTable& tab, cudaStream_t st);
+
+// The new tokens of a decode step, appended by step_prologue_kernel.
+struct AppendArgs {
+  uint4* pool;
+  int64_t num_blocks;
+  const int32_t* block_table;
+  int32_t max_blocks;
+  int32_t batch;
+  const int32_t* seq_ids;
+  const int64_t* positions;
+  const uint4* c_kv;
+  const uint4* k_pe;
+  int64_t T;
+  int32_t* status;
+  int rotate;
+};
+
+// q_absorb and the cache append of the same step in one launch.
+cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
+                                 const int32_t* seqlens, __nv_bfloat16* q_ext, int rows,
+                                 int q_len, float qscale, const RopeTable& q_tab,
+                                 const AppendArgs& ap, const RopeTable& k_tab, cudaStream_t st);
+
+// Merge of the splits and the W_UV product, written to out[rows, 32, 128].
+cudaError_t launch_combine(const float* part_o, const float* part_ml, const __nv_bfloat16* W_UV,
+                           __nv_bfloat16* out, int rows, int q_len, int groups, int nsplit,
+                           int rows_per_cta, cudaStream_t st);
+
+}  // namespace xmla

@@ -1,4 +1,4 @@
-// MLA decode over the paged latent cache, weight-absorbed form.
+// Split-K MLA decode attention over the paged latent cache (weight-absorbed form).
 //
 // [P5] "mHC+MLA+MTP 是什么？拆开给 Agent 用的百亿 MoE", section "MLA：256K 上下文的
 //      '内存革命'": per token and layer the cache keeps the 512-dim latent c_kv
@@ -10,40 +10,26 @@
 //      cache, not the weights, is what long contexts pay for; reading it is the
 //      whole cost of a decode step.
 //
-// Three kernels per call, chained with programmatic dependent launch:
-//   q_absorb   q_ext[b,j,h] = c * [W_UK[h]^T q_nope | rope(q_pe)]   (c = scale * log2 e)
-//   decode     one CTA per (sequence, row group, KV split): 64-token pages are
-//              streamed by TMA into a shared-memory ring; S^T = page . q_ext^T
-//              (M = 64 tokens, N = rows, K = 576) and O^T += c_kv^T . P^T (M = 128
-//              latent dims x 4, N = rows, K = 64 tokens) run on tcgen05 with fp32
-//              accumulators in tensor memory; S is double-buffered so the QK of
-//              page i+1 runs while the softmax of page i does; the online softmax
-//              (base 2, lazy max update) runs in registers.  Writes per-split
-//              (m, l, O).
-//   combine    a cluster of 8 CTAs per (head, row chunk) merges the splits by their
-//              log-sum-exp over 64-dim slices of the latent and applies W_UV; the
-//              slices' partial outputs are summed through distributed shared memory.
-#include <cooperative_groups.h>
+// One CTA per (sequence, row group, KV split): 64-token pages are streamed by
+// TMA into a shared-memory ring; S^T = page . q_ext^T (M = 64 tokens, N = rows,
+// K = 576) and O^T += c_kv^T . P^T (M = 128 latent dims x 4, N = rows, K = 64
+// tokens) run on tcgen05 with fp32 accumulators in tensor memory; S is
+// double-buffered so the QK of page i+1 runs while the softmax of page i does;
+// the online softmax (base 2, lazy max update) runs in registers.  Writes the
+// split's (m, l, O); the combine kernel merges the splits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <cmath>
 #include <cstdint>
-#include <cstring>
-#include <mutex>
 
-#include "xmla_device.cuh"
-#include "yarn.cuh"
-
-namespace cg = cooperative_groups;
+#include "decode_chain.h"
 
 namespace xmla {
 
-constexpr float kLog2e = 1.4426950408889634f;
 // A row's running maximum is only raised when a score exceeds it by more than
 // this (log2 units), so probabilities stay <= 2^kLazyMax before normalisation.
 constexpr float kLazyMax = 8.0f;
-constexpr int kMaxSplits = 1024;
 constexpr int kSoftmaxThreads = 128;
 constexpr int kSoftmaxWarp0 = 3;  // warps: 0 TMA producer, 1 QK issuer, 2 PV issuer, 3-6 softmax
 constexpr int kDecodeThreads = 32 * kSoftmaxWarp0 + kSoftmaxThreads;
@@ -97,21 +83,6 @@ struct DecodeLayout {
   static constexpr uint32_t kTmemCols = 6 * NR <= 256 ? 256 : 512;
 };
 
-struct DecodeParams {
-  const int32_t* block_table;
-  const int32_t* seqlens;
-  float* part_o;   // [items, NR, 512]
-  float* part_ml;  // [items, NR, 2]
-  int32_t* status;
-  int64_t num_blocks;
-  int64_t max_seqlen;
-  uint64_t wait_limit_ns;
-  int32_t max_blocks;
-  int32_t batch;
-  int32_t q_len;
-  int32_t groups;
-  int32_t nsplit;
-};
 
 // Warp transpose-reduction: on return v[0] of lane L holds the reduction over
 // the 32 lanes of input row L (31 shuffles for 32 rows).
@@ -607,392 +578,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------- q absorb
-
-// q_ext[r, h] = qscale * [W_UK[h]^T q_nope[r, h] | rope(q_pe[r, h], pos_r)], r = b*q_len + j,
-// with pos_r = seqlens[b] - q_len + j (the q_len new tokens are the last cache
-// entries).  grid (32 heads, 8 blocks of 64 latent columns); 128 threads:
-// thread t owns 8 columns (t % 8) and 8 of the 128 nope dims (t / 8), holding
-// its 8 x 8 slice of W_UK in registers (loaded before the wait on the kernel
-// launched just before, which it does not depend on); partial sums meet in
-// shared memory.  A ninth block per head rotates the rope part.
-constexpr int kAbsorbRows = 8;
-
-// q and seqlens carry no __restrict__ so that their loads stay behind the
-// griddepcontrol.wait (a preceding kernel may have written them).
-__global__ void __launch_bounds__(128) q_absorb_kernel(const __nv_bfloat16* q,
-                                                       const __nv_bfloat16* __restrict__ W_UK,
-                                                       const int32_t* seqlens,
-                                                       __nv_bfloat16* __restrict__ q_ext, int rows,
-                                                       int q_len, float qscale,
-                                                       const RopeTable tab) {
-  __shared__ float sq[kAbsorbRows][kDNope];
-  __shared__ float part[16][kAbsorbRows][64];
-  pdl_launch_dependents();
-  const int h = blockIdx.x;
-  const int cb = blockIdx.y;
-  const int t = threadIdx.x;
-  if (cb == kDLatent / 64) {
-    // q and the cache rows of this step may come from the kernels launched just
-    // before; every CTA waits (the decode kernel relies on it, see its producer)
-    pdl_wait();
-    constexpr int kPairs = kDRope / 2;
-    for (int e = t; e < rows * kPairs; e += blockDim.x) {
-      const int r = e / kPairs, i = e % kPairs;
-      const int64_t pos = (int64_t)seqlens[r / q_len] - q_len + (r % q_len);
-      const __nv_bfloat16* x = q + ((int64_t)r * kHeads + h) * kDQ + kDNope;
-      double y1, y2;
-      rope_pair((double)__bfloat162float(x[i]), (double)__bfloat162float(x[i + kPairs]), pos, i,
-                tab, &y1, &y2);
-      __nv_bfloat16* o = q_ext + ((int64_t)r * kHeads + h) * kDRow + kDLatent;
-      o[i] = __double2bfloat16(y1 * (double)qscale);
-      o[i + kPairs] = __double2bfloat16(y2 * (double)qscale);
-    }
-    return;
-  }
-  const int c8 = t & 7;
-  const int dg = t >> 3;
-  float w[8][8];
-#pragma unroll
-  for (int dd = 0; dd < 8; ++dd) {
-    const uint4 v = *reinterpret_cast<const uint4*>(
-        W_UK + ((int64_t)h * kDNope + dg * 8 + dd) * kDLatent + cb * 64 + c8 * 8);
-    const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      w[dd][2 * e] = __low2float(pv[e]);
-      w[dd][2 * e + 1] = __high2float(pv[e]);
-    }
-  }
-  pdl_wait();
-  for (int r0 = 0; r0 < rows; r0 += kAbsorbRows) {
-    const int nr = min(kAbsorbRows, rows - r0);
-    __syncthreads();
-    for (int e = t; e < nr * kDNope; e += blockDim.x) {
-      const int r = e / kDNope, d = e % kDNope;
-      sq[r][d] = __bfloat162float(q[((int64_t)(r0 + r) * kHeads + h) * kDQ + d]);
-    }
-    __syncthreads();
-    for (int r = 0; r < nr; ++r) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int dd = 0; dd < 8; ++dd) {
-        const float x = sq[r][dg * 8 + dd];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = fmaf(x, w[dd][k], acc[k]);
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) part[dg][r][c8 * 8 + k] = acc[k];
-    }
-    __syncthreads();
-    for (int o = t; o < nr * 64; o += blockDim.x) {
-      const int r = o / 64, col = o % 64;
-      float s = 0.f;
-#pragma unroll
-      for (int k = 0; k < 16; ++k) s += part[k][r][col];
-      q_ext[((int64_t)(r0 + r) * kHeads + h) * kDRow + cb * 64 + col] = __float2bfloat16_rn(s * qscale);
-    }
-  }
-}
-
-// ---------------------------------------------------------------- combine + W_UV
-
-// Cluster of 8 CTAs per (head h, chunk of up to kCombineRows output rows).
-// CTA `slice` owns latent dims [64 slice, 64 slice + 64).  All rows of the
-// chunk are merged together: 16 groups of 16 threads (one float4 of the slice
-// each) are shared out over the rows, and a row's splits are dealt round-robin
-// over its groups, so one pass of loads covers the chunk.  Every split is
-// weighted by 2^(m_s - M) against the row's overall maximum M and the sum is
-// divided by L = sum_s l_s 2^(m_s - M).  The CTA then multiplies its merged
-// 64 dims by the matching 64 rows of W_UV[h] and sends each 16-column block of
-// that product to the CTA that owns the block (distributed shared memory); the
-// owner adds the 8 contributions and writes its 16 output columns.
-constexpr int kSlices = 8;
-constexpr int kSliceDims = kDLatent / kSlices;        // 64
-constexpr int kCombineRows = 16;
-constexpr int kCombineThreads = 256;
-constexpr int kCombineWarps = kCombineThreads / 32;
-constexpr int kCombineGroups = kCombineThreads / 16;  // 16 threads x float4 cover a split row's slice
-constexpr int kCombineDepth = 10;                     // split rows each thread keeps in flight
-constexpr int kStatDepth = 4;                         // (m, l) pairs each lane keeps in flight
-constexpr int kColsPerSlice = kDV / kSlices;          // 16
-
-// Online (max, sum-of-exp2) pair merge.
-__device__ __forceinline__ void lse_merge(float& m, float& l, float m2, float l2) {
-  const float mx = fmaxf(m, m2);
-  if (mx == -INFINITY) return;
-  l = l * ex2(m - mx) + l2 * ex2(m2 - mx);
-  m = mx;
-}
-
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThreads, 3)
-    combine_uv_kernel(const float* part_o, const float* part_ml,
-                      const __nv_bfloat16* __restrict__ W_UV, __nv_bfloat16* __restrict__ out,
-                      int rows, int q_len, int groups, int nsplit, int rows_per_cta) {
-  // part_o and part_ml are written by the kernel launched just before this one,
-  // which lets this grid start early: they carry no __restrict__, so their loads
-  // are not taken as invariant and stay behind the griddepcontrol.wait below.
-  __shared__ __align__(16) __nv_bfloat16 w_s[kSliceDims][kDV];  // this slice's rows of W_UV[h]
-  __shared__ __align__(16) float4 acc_s[kCombineGroups][kSliceDims / 4];
-  __shared__ __align__(16) float o_s[kCombineRows][kSliceDims];
-  __shared__ __align__(16) float inbox[kSlices][kCombineRows][kColsPerSlice];  // by sender slice
-  __shared__ float stat_m[kCombineRows][kCombineWarps], stat_l[kCombineRows][kCombineWarps];
-  cg::cluster_group cluster = cg::this_cluster();
-  const int slice = (int)cluster.block_rank();
-  const int cid = blockIdx.x / kSlices;
-  const int h = cid % kHeads;
-  const int chunk = cid / kHeads;
-  const int r0 = chunk * kCombineRows;
-  const int nr = min(kCombineRows, rows - r0);
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  pdl_launch_dependents();
-  // first half of the barrier that guarantees every CTA of the cluster runs
-  // before any of them writes into another's shared memory
-  cluster_arrive_relaxed();
-  // W_UV does not depend on the decode kernel: stage it while that kernel finishes
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(W_UV + ((int64_t)h * kDLatent + slice * kSliceDims) * kDV);
-    uint4* dst = reinterpret_cast<uint4*>(&w_s[0][0]);
-#pragma unroll
-    for (int e = 0; e < kSliceDims * kDV / 8 / kCombineThreads; ++e)
-      dst[tid + kCombineThreads * e] = src[tid + kCombineThreads * e];
-  }
-
-  // partial row of split 0 for chunk row rr; split s is s * rows_per_cta rows further
-  auto split0_row = [&](int rr) -> int64_t {
-    const int r = r0 + rr;  // r = b*q_len + j
-    const int b = r / q_len, j = r % q_len;
-    const int ridx = j * kHeads + h;
-    return ((int64_t)b * groups + ridx / rows_per_cta) * nsplit * rows_per_cta + ridx % rows_per_cta;
-  };
-  const int q4 = tid & 15;  // float4 of the 64-dim slice
-  const int grp = tid >> 4;
-  const int gpr = max(1, kCombineGroups / nr);  // groups per row
-  const int my_rr = grp / gpr;
-  const int sub = grp % gpr;
-  const bool active = my_rr < nr;
-  const int64_t base = active ? split0_row(my_rr) : 0;
-  const float* po = part_o + base * kDLatent + slice * kSliceDims + 4 * q4;
-  const float* pm = part_ml + 2 * base;          // m of split s at pm[s * m_stride]
-  const int o_stride = rows_per_cta * kDLatent;  // floats between splits (nsplit * o_stride < 2^31)
-  const int m_stride = 2 * rows_per_cta;
-  const int wpr = max(1, kCombineWarps / nr);    // warps per row for the statistics
-
-  pdl_wait();  // the split partials come from the decode kernel
-
-  // first batch of this thread's split rows, issued before the row statistics
-  // so that both sets of loads are in flight together.  A split that saw no
-  // token has m = -inf (and l = 0); only m is needed to recognise it.
-  float4 v[kCombineDepth];
-  float ms[kCombineDepth];
-#pragma unroll
-  for (int k = 0; k < kCombineDepth; ++k) {
-    const int s = sub + gpr * k;
-    const bool in = active && s < nsplit;
-    v[k] = in ? *reinterpret_cast<const float4*>(po + s * o_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
-    ms[k] = in ? pm[s * m_stride] : -INFINITY;
-  }
-
-  // row statistics: `wpr` warps share a row's splits (part p takes splits
-  // 32 p + lane, then every 32 wpr further); each warp reduces its share
-  {
-    const int part = warp % wpr;
-    for (int rr = warp / wpr; rr < nr; rr += kCombineWarps / wpr) {
-      const float2* rml = reinterpret_cast<const float2*>(part_ml) + split0_row(rr);
-      float m = -INFINITY, l = 0.f;
-      for (int s0 = 32 * part; s0 < nsplit; s0 += 32 * wpr * kStatDepth) {
-        float2 x[kStatDepth];
-#pragma unroll
-        for (int k = 0; k < kStatDepth; ++k) {
-          const int s = s0 + lane + 32 * wpr * k;
-          x[k] = s < nsplit ? rml[(int64_t)s * rows_per_cta] : make_float2(-INFINITY, 0.f);
-        }
-#pragma unroll
-        for (int k = 0; k < kStatDepth; ++k)
-          if (x[k].y > 0.f) lse_merge(m, l, x[k].x, x[k].y);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-        const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-        lse_merge(m, l, m2, l2);
-      }
-      if (lane == 0) {
-        stat_m[rr][part] = m;
-        stat_l[rr][part] = l;
-      }
-    }
-  }
-  __syncthreads();
-
-  // weighted sum of this thread's split rows (the partial O of a split that saw
-  // no token was never written: it is skipped, not multiplied by zero)
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (active) {
-    float M = stat_m[my_rr][0];
-    for (int p = 1; p < wpr; ++p) M = fmaxf(M, stat_m[my_rr][p]);
-    for (int k0 = 0;; k0 += kCombineDepth) {
-#pragma unroll
-      for (int k = 0; k < kCombineDepth; ++k) {
-        if (ms[k] != -INFINITY) {
-          const float wgt = ex2(ms[k] - M);
-          acc.x = fmaf(wgt, v[k].x, acc.x);
-          acc.y = fmaf(wgt, v[k].y, acc.y);
-          acc.z = fmaf(wgt, v[k].z, acc.z);
-          acc.w = fmaf(wgt, v[k].w, acc.w);
-        }
-      }
-      const int k1 = k0 + kCombineDepth;
-      if (sub + gpr * k1 >= nsplit) break;
-#pragma unroll
-      for (int k = 0; k < kCombineDepth; ++k) {
-        const int s = sub + gpr * (k1 + k);
-        const bool in = s < nsplit;
-        v[k] = in ? *reinterpret_cast<const float4*>(po + s * o_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
-        ms[k] = in ? pm[s * m_stride] : -INFINITY;
-      }
-    }
-  }
-  acc_s[grp][q4] = acc;
-  __syncthreads();
-  for (int e = tid; e < nr * kSliceDims; e += kCombineThreads) {
-    const int rr = e / kSliceDims, d = e % kSliceDims;
-    float M = stat_m[rr][0];
-    for (int p = 1; p < wpr; ++p) M = fmaxf(M, stat_m[rr][p]);
-    float L = 0.f;
-    for (int p = 0; p < wpr; ++p)
-      if (stat_l[rr][p] > 0.f) L += stat_l[rr][p] * ex2(stat_m[rr][p] - M);
-    const float* a = reinterpret_cast<const float*>(&acc_s[rr * gpr][0]) + d;
-    float t = 0.f;
-    for (int g = 0; g < gpr; ++g) t += a[g * kSliceDims];
-    o_s[rr][d] = L > 0.f ? t / L : 0.f;
-  }
-  __syncthreads();
-
-  // slice product: sum over the slice's 64 latent dims c of o[r][c] W_UV[h][c][v]
-  // for the column pair (2 vp, 2 vp + 1), sent to the CTA owning that column block
-  cluster_wait_acquire();  // every CTA of the cluster is running
-  {
-    const int vp = tid & (kDV / 2 - 1);
-    const int owner = (2 * vp) / kColsPerSlice;
-    float* dst = cluster.map_shared_rank(&inbox[slice][0][0], owner);
-    for (int rr = tid / (kDV / 2); rr < nr; rr += kCombineThreads / (kDV / 2)) {
-      float a0 = 0.f, a1 = 0.f;
-#pragma unroll 16
-      for (int c = 0; c < kSliceDims; ++c) {
-        const float2 w = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&w_s[c][0])[vp]);
-        const float x = o_s[rr][c];
-        a0 = fmaf(x, w.x, a0);
-        a1 = fmaf(x, w.y, a1);
-      }
-      *reinterpret_cast<float2*>(dst + rr * kColsPerSlice + (2 * vp) % kColsPerSlice) = make_float2(a0, a1);
-    }
-  }
-  cluster_arrive_release();
-  cluster_wait_acquire();  // all 8 contributions have landed in this CTA's inbox
-  if (tid < nr * kColsPerSlice) {
-    const int rr = tid / kColsPerSlice, c = tid % kColsPerSlice;
-    float t = 0.f;
-#pragma unroll
-    for (int k = 0; k < kSlices; ++k) t += inbox[k][rr][c];
-    out[((int64_t)(r0 + rr) * kHeads + h) * kDV + slice * kColsPerSlice + c] = __float2bfloat16_rn(t);
-  }
-}
-
-// ---------------------------------------------------------------- self-test kernel
-
-__global__ void wait_timeout_selftest_kernel(int32_t* status, uint64_t limit_ns) {
-  __shared__ uint64_t bar_word;
-  const uint32_t b = smem_u32(&bar_word);
-  mbar_init(b, 1);
-  fence_barrier_init();
-  // nothing ever arrives on this barrier: the bounded wait must give up
-  mbar_wait(b, 0, nullptr, status, limit_ns);
-}
-
-// ---------------------------------------------------------------- host plan
-
-struct Plan {
-  int nr;       // rows per CTA (32 or 64)
-  int groups;   // row groups per sequence
-  int nsplit;   // KV splits per (sequence, group)
-  int64_t items;
-  size_t off_qext, off_o, off_ml, bytes;
-};
-
-static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
-static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_sms,
-                      int32_t num_splits, Plan* pl) {
-  if (B < 1 || q_len < 1 || q_len > kMaxQLen || max_seqlen < q_len ||
-      max_seqlen > (int64_t)0x7fffffff - kPage || num_sms < 1 || num_splits < 0)
-    return false;
-  Plan P;
-  P.nr = q_len == 1 ? 32 : 64;
-  P.groups = (q_len * 32 + P.nr - 1) / P.nr;
-  const int64_t max_pages = (max_seqlen + kPage - 1) / kPage;
-  int64_t ns;
-  if (num_splits > 0) {
-    ns = num_splits;
-  } else {
-    const int64_t units = (int64_t)B * P.groups;
-    ns = units >= num_sms ? 1 : num_sms / units;
-    const int64_t cap = max_pages >= 2 ? max_pages / 2 : 1;  // at least two pages per split
-    if (ns > cap) ns = cap;
-  }
-  if (ns < 1) ns = 1;
-  if (ns > kMaxSplits) return false;
-  P.nsplit = (int)ns;
-  P.items = (int64_t)B * P.groups * P.nsplit;
-  if (P.items > 0x7fffffff) return false;
-  const size_t qext = (size_t)B * q_len * kHeads * kDRow * 2;
-  P.off_qext = 0;
-  P.off_o = align_up(qext, 1024);
-  P.off_ml = align_up(P.off_o + (size_t)P.items * P.nr * kDLatent * 4, 1024);
-  P.bytes = align_up(P.off_ml + (size_t)P.items * P.nr * 2 * 4, 1024);
-  *pl = P;
-  return true;
-}
-
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// 2-D map over rows of 576 bf16 (1152 B), box = 64 columns x box_rows rows,
-// 128-byte swizzle (the layout the tensor-core descriptors above expect).
-static bool encode_rows576(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kDRow, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kDRow * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int NR>
 static cudaError_t launch_decode(const CUtensorMap& tp, const CUtensorMap& tq, const DecodeParams& dp,
                                  int64_t items, cudaStream_t st) {
@@ -1011,196 +596,12 @@ static cudaError_t launch_decode(const CUtensorMap& tp, const CUtensorMap& tq, c
                     st, tp, tq, dp);
 }
 
-static bool device_ok(int* num_sms) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  int major = 0, minor = 0;
-  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-  cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev);
-  return major == 10 && minor == 0;
+
+cudaError_t launch_split_kv(int nr, const CUtensorMap& pool_map, const CUtensorMap& q_map,
+                            const DecodeParams& dp, int64_t items, cudaStream_t st) {
+  if (nr == 32) return launch_decode<32>(pool_map, q_map, dp, items, st);
+  if (nr == 64) return launch_decode<64>(pool_map, q_map, dp, items, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace xmla
-
-using namespace xmla;
-
-extern "C" size_t xmla_decode_workspace_size(int32_t batch, int32_t q_len, int64_t max_seqlen,
-                                             int32_t num_sms, int32_t num_splits) {
-  Plan P;
-  return make_plan(batch, q_len, max_seqlen, num_sms, num_splits, &P) ? P.bytes : 0;
-}
-
-extern "C" int32_t xmla_decode_num_splits(int32_t batch, int32_t q_len, int64_t max_seqlen,
-                                          int32_t num_sms, int32_t num_splits) {
-  Plan P;
-  return make_plan(batch, q_len, max_seqlen, num_sms, num_splits, &P) ? P.nsplit : 0;
-}
-
-static cudaError_t record_event(void* ev, cudaStream_t st) {
-  if (ev == nullptr) return cudaSuccess;
-  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  cudaError_t e = cudaStreamIsCapturing(st, &cs);
-  if (e != cudaSuccess) return e;
-  // inside a graph capture the record must become an event-record node
-  return cs == cudaStreamCaptureStatusActive
-             ? cudaEventRecordWithFlags((cudaEvent_t)ev, st, cudaEventRecordExternal)
-             : cudaEventRecord((cudaEvent_t)ev, st);
-}
-
-extern "C" xmla_status xmla_decode_profiled(const xmla_yarn_cfg* cfg, const void* q,
-                                            const void* W_UK, const void* W_UV,
-                                            const void* pool, int64_t num_blocks,
-                                            const int32_t* block_table, int32_t max_blocks,
-                                            const int32_t* seqlens, int32_t batch, int32_t q_len,
-                                            int64_t max_seqlen, float softmax_scale,
-                                            int32_t num_splits, void* workspace,
-                                            size_t workspace_bytes, int32_t* status_dev, void* out,
-                                            void* stream, void* attn_start, void* attn_stop) {
-  if (q == nullptr || W_UK == nullptr || W_UV == nullptr || pool == nullptr ||
-      block_table == nullptr || seqlens == nullptr || workspace == nullptr || out == nullptr)
-    return XMLA_ERR_INVALID_ARG;
-  if (!yarn_cfg_ok(cfg)) return XMLA_ERR_INVALID_ARG;
-  if (cfg->rotary_dim != kDRope) return XMLA_ERR_SHAPE;
-  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return XMLA_ERR_INVALID_ARG;
-  if ((((uintptr_t)pool) & 15u) || (((uintptr_t)workspace) & 255u) || (((uintptr_t)q) & 15u) ||
-      (((uintptr_t)W_UK) & 15u) || (((uintptr_t)W_UV) & 15u) || (((uintptr_t)out) & 15u))
-    return XMLA_ERR_INVALID_ARG;
-  if (num_blocks < 1 || num_blocks * kPage >= 0x7fffffffLL || max_blocks < 1 ||
-      (int64_t)max_blocks * kPage < max_seqlen)
-    return XMLA_ERR_SHAPE;
-  int nsm = 0;
-  if (!device_ok(&nsm)) return XMLA_ERR_UNSUPPORTED;
-  Plan P;
-  if (!make_plan(batch, q_len, max_seqlen, nsm, num_splits, &P)) return XMLA_ERR_SHAPE;
-  if (workspace_bytes < P.bytes) return XMLA_ERR_WORKSPACE;
-  cudaStream_t st = (cudaStream_t)stream;
-  uint8_t* ws = (uint8_t*)workspace;
-  __nv_bfloat16* q_ext = (__nv_bfloat16*)(ws + P.off_qext);
-  const int rows = batch * q_len;
-
-  CUtensorMap tmap_pool, tmap_q;
-  if (!encode_rows576(&tmap_pool, pool, (uint64_t)num_blocks * kPage, kPage)) return XMLA_ERR_CUDA;
-  if (!encode_rows576(&tmap_q, q_ext, (uint64_t)rows * kHeads, (uint32_t)P.nr)) return XMLA_ERR_CUDA;
-
-  const float qscale = softmax_scale * kLog2e;
-  // Every kernel of the chain waits (griddepcontrol.wait) for its predecessor
-  // before reading anything a kernel of this step may have written, so once
-  // q_absorb completes all earlier work on the stream has landed.
-  if (launch_pdl(q_absorb_kernel, dim3(kHeads, kDLatent / 64 + 1), dim3(128), 0, st,
-                 (const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext, rows, q_len,
-                 qscale, make_rope_table(cfg)) != cudaSuccess)
-    return XMLA_ERR_CUDA;
-
-  DecodeParams dp;
-  dp.block_table = block_table;
-  dp.seqlens = seqlens;
-  dp.part_o = (float*)(ws + P.off_o);
-  dp.part_ml = (float*)(ws + P.off_ml);
-  dp.status = status_dev;
-  dp.num_blocks = num_blocks;
-  dp.max_seqlen = max_seqlen;
-  dp.wait_limit_ns = kWaitLimitNs;
-  dp.max_blocks = max_blocks;
-  dp.batch = batch;
-  dp.q_len = q_len;
-  dp.groups = P.groups;
-  dp.nsplit = P.nsplit;
-  if (record_event(attn_start, st) != cudaSuccess) return XMLA_ERR_CUDA;
-  cudaError_t e = P.nr == 32 ? launch_decode<32>(tmap_pool, tmap_q, dp, P.items, st)
-                             : launch_decode<64>(tmap_pool, tmap_q, dp, P.items, st);
-  if (e != cudaSuccess) return XMLA_ERR_CUDA;
-  if (record_event(attn_stop, st) != cudaSuccess) return XMLA_ERR_CUDA;
-
-  const int chunks = (rows + kCombineRows - 1) / kCombineRows;
-  e = launch_pdl(combine_uv_kernel, dim3(kSlices * kHeads * chunks), dim3(kCombineThreads), 0, st,
-                 (const float*)dp.part_o, (const float*)dp.part_ml, (const __nv_bfloat16*)W_UV,
-                 (__nv_bfloat16*)out, rows, q_len, P.groups, P.nsplit, P.nr);
-  return e == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
-}
-
-extern "C" xmla_status xmla_decode(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
-                                   const void* W_UV, const void* pool, int64_t num_blocks,
-                                   const int32_t* block_table, int32_t max_blocks,
-                                   const int32_t* seqlens, int32_t batch, int32_t q_len,
-                                   int64_t max_seqlen, float softmax_scale, int32_t num_splits,
-                                   void* workspace, size_t workspace_bytes, int32_t* status_dev,
-                                   void* out, void* stream) {
-  return xmla_decode_profiled(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens,
-                              batch, q_len, max_seqlen, softmax_scale, num_splits, workspace,
-                              workspace_bytes, status_dev, out, stream, nullptr, nullptr);
-}
-
-// ---------------------------------------------------------------- decode without caller scratch
-
-namespace xmla {
-
-// Fixed device scratch for xmla_decode_noalloc.  It is part of the library's
-// module image, so every GPU that loads the library holds it until the
-// process exits; its size is the largest workspace that entry point accepts.
-constexpr size_t kNoAllocScratchBytes = (size_t)XMLA_NOALLOC_SCRATCH_BYTES;
-static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-
-static std::mutex g_noalloc_mutex;
-static void* g_noalloc_addr[64] = {};
-
-// Device address of the scratch array on the current device.  In host code
-// the array's name is only a host-side stand-in, so the real address is asked
-// from the runtime once per device (with that device current) and cached.
-static xmla_status noalloc_scratch(void** addr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return XMLA_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return XMLA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return XMLA_ERR_CUDA;
-    g_noalloc_addr[dev] = p;
-  }
-  *addr = g_noalloc_addr[dev];
-  return XMLA_OK;
-}
-
-}  // namespace xmla
-
-extern "C" xmla_status xmla_decode_noalloc(const xmla_yarn_cfg* cfg, const void* q,
-                                           const void* W_UK, const void* W_UV, const void* pool,
-                                           int64_t num_blocks, const int32_t* block_table,
-                                           int32_t max_blocks, const int32_t* seqlens,
-                                           int32_t batch, int32_t q_len, int64_t max_seqlen,
-                                           float softmax_scale, int32_t num_splits,
-                                           int32_t* status_dev, void* out, void* stream) {
-  int nsm = 0;
-  if (!xmla::device_ok(&nsm)) return XMLA_ERR_UNSUPPORTED;
-  const size_t need = xmla_decode_workspace_size(batch, q_len, max_seqlen, nsm, num_splits);
-  if (need == 0) return XMLA_ERR_SHAPE;
-  if (need > xmla::kNoAllocScratchBytes) return XMLA_ERR_WORKSPACE;
-  void* scratch = nullptr;
-  const xmla_status st = xmla::noalloc_scratch(&scratch);
-  if (st != XMLA_OK) return st;
-  return xmla_decode(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens, batch,
-                     q_len, max_seqlen, softmax_scale, num_splits, scratch,
-                     xmla::kNoAllocScratchBytes, status_dev, out, stream);
-}
-
-extern "C" xmla_status xmla_selftest_wait_timeout(int32_t* status_dev, uint64_t timeout_ns,
-                                                  void* stream) {
-  if (status_dev == nullptr) return XMLA_ERR_INVALID_ARG;
-  wait_timeout_selftest_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(status_dev, timeout_ns);
-  return cudaGetLastError() == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
-}
-
-extern "C" const char* xmla_status_string(xmla_status s) {
-  switch (s) {
-    case XMLA_OK: return "ok";
-    case XMLA_ERR_INVALID_ARG: return "invalid argument";
-    case XMLA_ERR_SHAPE: return "unsupported shape";
-    case XMLA_ERR_WORKSPACE: return "workspace too small";
-    case XMLA_ERR_CUDA: return "CUDA error";
-    case XMLA_ERR_DEVICE_OOB: return "device: index out of range";
-    case XMLA_ERR_TIMEOUT: return "device: bounded wait timed out";
-    case XMLA_ERR_UNSUPPORTED: return "device not supported (needs sm_100a)";
-  }
-  return "unknown status";
-}

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 
+#include "append.cuh"
 #include "xmla_device.cuh"
 #include "yarn.cuh"
 
@@ -45,62 +46,18 @@ __global__ void __launch_bounds__(256) rope_yarn_kernel(__nv_bfloat16* x, int64_
 
 // ---------------------------------------------------------------- device: append
 
-// One thread per 16-byte piece of a cache row: 64 pieces of latent (bit copy)
-// and 8 pieces of rope key.  With rotation on, rope piece r instead rotates
-// the four pairs (4r .. 4r+3, 4r+32 .. 4r+35) at the row's position and
-// stores them.
+// One thread per 16-byte piece of a cache row (append_piece in append.cuh).
 __global__ void __launch_bounds__(256) cache_append_kernel(
     uint4* pool, int64_t num_blocks, const int32_t* block_table, int32_t max_blocks,
     int32_t batch, const int32_t* seq_ids, const int64_t* positions, const uint4* c_kv,
     const uint4* k_pe, int64_t T, int32_t* status, int rotate, const RopeTable tab) {
   pdl_wait();  // inputs may come from the kernel launched just before
   pdl_launch_dependents();
-  constexpr int kLatPieces = kDLatent * 2 / 16;  // 64
-  constexpr int kRopePieces = kDRope * 2 / 16;   // 8
-  constexpr int kRowPieces = kLatPieces + kRopePieces;
   const int64_t total = T * kRowPieces;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = idx / kRowPieces;
-    const int piece = (int)(idx % kRowPieces);
-    const int32_t s = seq_ids[t];
-    const int64_t pos = positions[t];
-    if (s < 0 || s >= batch || pos < 0 || pos >= (int64_t)max_blocks * kPage) {
-      record_status(status, XMLA_ERR_DEVICE_OOB);
-      continue;
-    }
-    const int32_t blk = block_table[(int64_t)s * max_blocks + pos / kPage];
-    if (blk < 0 || (int64_t)blk >= num_blocks) {
-      record_status(status, XMLA_ERR_DEVICE_OOB);
-      continue;
-    }
-    uint4* row = pool + ((int64_t)blk * kPage + pos % kPage) * kRowPieces;
-    if (piece < kLatPieces) {
-      row[piece] = c_kv[t * kLatPieces + piece];
-    } else if (!rotate) {
-      row[piece] = k_pe[t * kRopePieces + (piece - kLatPieces)];
-    } else {
-      const int r = piece - kLatPieces;  // pairs 4r .. 4r+3
-      const uint2* src = reinterpret_cast<const uint2*>(k_pe + t * kRopePieces);
-      uint2* dst = reinterpret_cast<uint2*>(row + kLatPieces);
-      const uint2 lo = src[r], hi = src[r + 8];  // dims 4r.., 32+4r..
-      const __nv_bfloat16* xl = reinterpret_cast<const __nv_bfloat16*>(&lo);
-      const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&hi);
-      uint2 olo, ohi;
-      __nv_bfloat16* yl = reinterpret_cast<__nv_bfloat16*>(&olo);
-      __nv_bfloat16* yh = reinterpret_cast<__nv_bfloat16*>(&ohi);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        double y1, y2;
-        rope_pair((double)__bfloat162float(xl[e]), (double)__bfloat162float(xh[e]), pos, 4 * r + e,
-                  tab, &y1, &y2);
-        yl[e] = __double2bfloat16(y1);
-        yh[e] = __double2bfloat16(y2);
-      }
-      dst[r] = olo;
-      dst[r + 8] = ohi;
-    }
-  }
+       idx += (int64_t)gridDim.x * blockDim.x)
+    append_piece(idx, pool, num_blocks, block_table, max_blocks, batch, seq_ids, positions, c_kv,
+                 k_pe, status, rotate, tab);
 }
 
 static int grid_for(int64_t work, int threads) {
@@ -175,7 +132,7 @@ extern "C" xmla_status xmla_cache_append(void* pool, int64_t num_blocks, const i
     if (rope_cfg->rotary_dim != kDRope) return XMLA_ERR_SHAPE;
     tab = make_rope_table(rope_cfg);
   }
-  const int64_t work = T * 72;
+  const int64_t work = T * kRowPieces;
   const cudaError_t e = launch_pdl(cache_append_kernel, dim3(grid_for(work, 256)), dim3(256), 0,
                                    (cudaStream_t)stream, (uint4*)pool, num_blocks, block_table,
                                    max_blocks, batch, seq_ids, positions, (const uint4*)c_kv,

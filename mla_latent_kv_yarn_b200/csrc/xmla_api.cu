@@ -1,0 +1,341 @@
+// C ABI of the decode path: argument checks, the workspace plan, TMA tensor
+// maps, and the launch of the kernel chain (decode_chain.h).
+//
+// [P5] "mHC+MLA+MTP 是什么？拆开给 Agent 用的百亿 MoE", section "MLA：256K 上下文的
+//      '内存革命'": attention over the cached latent, absorbed form.
+// [P1] "256K 长上下文真能本地用：Xing4.0 原生长上下文的工程代价拆解", sections 一 and 二:
+//      YaRN RoPE on q_pe; the cache read dominates a long-context decode step.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "decode_chain.h"
+
+namespace xmla {
+
+// ---------------------------------------------------------------- self-test kernel
+
+__global__ void wait_timeout_selftest_kernel(int32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar_word;
+  const uint32_t b = smem_u32(&bar_word);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  // nothing ever arrives on this barrier: the bounded wait must give up
+  mbar_wait(b, 0, nullptr, status, limit_ns);
+}
+
+// ---------------------------------------------------------------- host plan
+
+struct Plan {
+  int nr;       // rows per CTA (32 or 64)
+  int groups;   // row groups per sequence
+  int nsplit;   // KV splits per (sequence, group)
+  int64_t items;
+  size_t off_qext, off_o, off_ml, bytes;
+};
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_sms,
+                      int32_t num_splits, Plan* pl) {
+  if (B < 1 || q_len < 1 || q_len > kMaxQLen || max_seqlen < q_len ||
+      max_seqlen > (int64_t)0x7fffffff - kPage || num_sms < 1 || num_splits < 0)
+    return false;
+  Plan P;
+  P.nr = q_len == 1 ? 32 : 64;
+  P.groups = (q_len * 32 + P.nr - 1) / P.nr;
+  const int64_t max_pages = (max_seqlen + kPage - 1) / kPage;
+  int64_t ns;
+  if (num_splits > 0) {
+    ns = num_splits;
+  } else {
+    const int64_t units = (int64_t)B * P.groups;
+    ns = units >= num_sms ? 1 : num_sms / units;
+    const int64_t cap = max_pages >= 2 ? max_pages / 2 : 1;  // at least two pages per split
+    if (ns > cap) ns = cap;
+  }
+  if (ns < 1) ns = 1;
+  if (ns > kMaxSplits) return false;
+  P.nsplit = (int)ns;
+  P.items = (int64_t)B * P.groups * P.nsplit;
+  if (P.items > 0x7fffffff) return false;
+  const size_t qext = (size_t)B * q_len * kHeads * kDRow * 2;
+  P.off_qext = 0;
+  P.off_o = align_up(qext, 1024);
+  P.off_ml = align_up(P.off_o + (size_t)P.items * P.nr * kDLatent * 4, 1024);
+  P.bytes = align_up(P.off_ml + (size_t)P.items * P.nr * 2 * 4, 1024);
+  *pl = P;
+  return true;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over rows of 576 bf16 (1152 B), box = 64 columns x box_rows rows,
+// 128-byte swizzle (the layout the tensor-core descriptors above expect).
+static bool encode_rows576(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kDRow, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kDRow * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool device_ok(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev);
+  return major == 10 && minor == 0;
+}
+
+}  // namespace xmla
+
+using namespace xmla;
+
+extern "C" size_t xmla_decode_workspace_size(int32_t batch, int32_t q_len, int64_t max_seqlen,
+                                             int32_t num_sms, int32_t num_splits) {
+  Plan P;
+  return make_plan(batch, q_len, max_seqlen, num_sms, num_splits, &P) ? P.bytes : 0;
+}
+
+extern "C" int32_t xmla_decode_num_splits(int32_t batch, int32_t q_len, int64_t max_seqlen,
+                                          int32_t num_sms, int32_t num_splits) {
+  Plan P;
+  return make_plan(batch, q_len, max_seqlen, num_sms, num_splits, &P) ? P.nsplit : 0;
+}
+
+static cudaError_t record_event(void* ev, cudaStream_t st) {
+  if (ev == nullptr) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  // inside a graph capture the record must become an event-record node
+  return cs == cudaStreamCaptureStatusActive
+             ? cudaEventRecordWithFlags((cudaEvent_t)ev, st, cudaEventRecordExternal)
+             : cudaEventRecord((cudaEvent_t)ev, st);
+}
+
+// The decode chain shared by the entries below; `ap` (nullable) adds the
+// step's cache append to the first kernel.
+static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
+                              const void* W_UV, const void* pool, int64_t num_blocks,
+                              const int32_t* block_table, int32_t max_blocks,
+                              const int32_t* seqlens, int32_t batch, int32_t q_len,
+                              int64_t max_seqlen, float softmax_scale, int32_t num_splits,
+                              void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                              void* out, void* stream, void* attn_start, void* attn_stop,
+                              const AppendArgs* ap) {
+  if (q == nullptr || W_UK == nullptr || W_UV == nullptr || pool == nullptr ||
+      block_table == nullptr || seqlens == nullptr || workspace == nullptr || out == nullptr)
+    return XMLA_ERR_INVALID_ARG;
+  if (!yarn_cfg_ok(cfg)) return XMLA_ERR_INVALID_ARG;
+  if (cfg->rotary_dim != kDRope) return XMLA_ERR_SHAPE;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return XMLA_ERR_INVALID_ARG;
+  if ((((uintptr_t)pool) & 15u) || (((uintptr_t)workspace) & 255u) || (((uintptr_t)q) & 15u) ||
+      (((uintptr_t)W_UK) & 15u) || (((uintptr_t)W_UV) & 15u) || (((uintptr_t)out) & 15u))
+    return XMLA_ERR_INVALID_ARG;
+  if (num_blocks < 1 || num_blocks * kPage >= 0x7fffffffLL || max_blocks < 1 ||
+      (int64_t)max_blocks * kPage < max_seqlen)
+    return XMLA_ERR_SHAPE;
+  int nsm = 0;
+  if (!device_ok(&nsm)) return XMLA_ERR_UNSUPPORTED;
+  Plan P;
+  if (!make_plan(batch, q_len, max_seqlen, nsm, num_splits, &P)) return XMLA_ERR_SHAPE;
+  if (workspace_bytes < P.bytes) return XMLA_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* ws = (uint8_t*)workspace;
+  __nv_bfloat16* q_ext = (__nv_bfloat16*)(ws + P.off_qext);
+  const int rows = batch * q_len;
+
+  CUtensorMap tmap_pool, tmap_q;
+  if (!encode_rows576(&tmap_pool, pool, (uint64_t)num_blocks * kPage, kPage)) return XMLA_ERR_CUDA;
+  if (!encode_rows576(&tmap_q, q_ext, (uint64_t)rows * kHeads, (uint32_t)P.nr)) return XMLA_ERR_CUDA;
+
+  const float qscale = softmax_scale * kLog2e;
+  const RopeTable tab = make_rope_table(cfg);
+  // Every kernel of the chain waits (griddepcontrol.wait) for its predecessor
+  // before reading anything a kernel of this step may have written, so once
+  // the first kernel completes all earlier work on the stream has landed.
+  const cudaError_t e0 =
+      ap != nullptr
+          ? launch_step_prologue((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
+                                 rows, q_len, qscale, tab, *ap, tab, st)
+          : launch_q_absorb((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
+                            rows, q_len, qscale, tab, st);
+  if (e0 != cudaSuccess) return XMLA_ERR_CUDA;
+
+  DecodeParams dp;
+  dp.block_table = block_table;
+  dp.seqlens = seqlens;
+  dp.part_o = (float*)(ws + P.off_o);
+  dp.part_ml = (float*)(ws + P.off_ml);
+  dp.status = status_dev;
+  dp.num_blocks = num_blocks;
+  dp.max_seqlen = max_seqlen;
+  dp.wait_limit_ns = kWaitLimitNs;
+  dp.max_blocks = max_blocks;
+  dp.batch = batch;
+  dp.q_len = q_len;
+  dp.groups = P.groups;
+  dp.nsplit = P.nsplit;
+  if (record_event(attn_start, st) != cudaSuccess) return XMLA_ERR_CUDA;
+  if (launch_split_kv(P.nr, tmap_pool, tmap_q, dp, P.items, st) != cudaSuccess) return XMLA_ERR_CUDA;
+  if (record_event(attn_stop, st) != cudaSuccess) return XMLA_ERR_CUDA;
+  const cudaError_t e = launch_combine(dp.part_o, dp.part_ml, (const __nv_bfloat16*)W_UV,
+                                       (__nv_bfloat16*)out, rows, q_len, P.groups, P.nsplit, P.nr,
+                                       st);
+  return e == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+}
+
+extern "C" xmla_status xmla_decode_profiled(const xmla_yarn_cfg* cfg, const void* q,
+                                            const void* W_UK, const void* W_UV,
+                                            const void* pool, int64_t num_blocks,
+                                            const int32_t* block_table, int32_t max_blocks,
+                                            const int32_t* seqlens, int32_t batch, int32_t q_len,
+                                            int64_t max_seqlen, float softmax_scale,
+                                            int32_t num_splits, void* workspace,
+                                            size_t workspace_bytes, int32_t* status_dev, void* out,
+                                            void* stream, void* attn_start, void* attn_stop) {
+  return run_decode(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens, batch,
+                    q_len, max_seqlen, softmax_scale, num_splits, workspace, workspace_bytes,
+                    status_dev, out, stream, attn_start, attn_stop, nullptr);
+}
+
+extern "C" xmla_status xmla_decode_step(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
+                                        const void* W_UV, void* pool, int64_t num_blocks,
+                                        const int32_t* block_table, int32_t max_blocks,
+                                        const int32_t* seqlens, int32_t batch, int32_t q_len,
+                                        int64_t max_seqlen, const int32_t* seq_ids,
+                                        const int64_t* positions, const void* c_kv,
+                                        const void* k_pe, int64_t T, float softmax_scale,
+                                        int32_t num_splits, void* workspace,
+                                        size_t workspace_bytes, int32_t* status_dev, void* out,
+                                        void* stream, void* attn_start, void* attn_stop) {
+  if (T < 0) return XMLA_ERR_SHAPE;
+  if (T > 0 && (seq_ids == nullptr || positions == nullptr || c_kv == nullptr || k_pe == nullptr))
+    return XMLA_ERR_INVALID_ARG;
+  if ((((uintptr_t)c_kv) | ((uintptr_t)k_pe)) & 15u) return XMLA_ERR_INVALID_ARG;
+  AppendArgs ap;
+  ap.pool = (uint4*)pool;
+  ap.num_blocks = num_blocks;
+  ap.block_table = block_table;
+  ap.max_blocks = max_blocks;
+  ap.batch = batch;
+  ap.seq_ids = seq_ids;
+  ap.positions = positions;
+  ap.c_kv = (const uint4*)c_kv;
+  ap.k_pe = (const uint4*)k_pe;
+  ap.T = T;
+  ap.status = status_dev;
+  ap.rotate = 1;
+  return run_decode(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens, batch,
+                    q_len, max_seqlen, softmax_scale, num_splits, workspace, workspace_bytes,
+                    status_dev, out, stream, attn_start, attn_stop, &ap);
+}
+
+extern "C" xmla_status xmla_decode(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
+                                   const void* W_UV, const void* pool, int64_t num_blocks,
+                                   const int32_t* block_table, int32_t max_blocks,
+                                   const int32_t* seqlens, int32_t batch, int32_t q_len,
+                                   int64_t max_seqlen, float softmax_scale, int32_t num_splits,
+                                   void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                                   void* out, void* stream) {
+  return xmla_decode_profiled(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens,
+                              batch, q_len, max_seqlen, softmax_scale, num_splits, workspace,
+                              workspace_bytes, status_dev, out, stream, nullptr, nullptr);
+}
+
+// ---------------------------------------------------------------- decode without caller scratch
+
+namespace xmla {
+
+// Fixed device scratch for xmla_decode_noalloc.  It is part of the library's
+// module image, so every GPU that loads the library holds it until the
+// process exits; its size is the largest workspace that entry point accepts.
+constexpr size_t kNoAllocScratchBytes = (size_t)XMLA_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_noalloc_mutex;
+static void* g_noalloc_addr[64] = {};
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the real address is asked
+// from the runtime once per device (with that device current) and cached.
+static xmla_status noalloc_scratch(void** addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return XMLA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return XMLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return XMLA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return XMLA_OK;
+}
+
+}  // namespace xmla
+
+extern "C" xmla_status xmla_decode_noalloc(const xmla_yarn_cfg* cfg, const void* q,
+                                           const void* W_UK, const void* W_UV, const void* pool,
+                                           int64_t num_blocks, const int32_t* block_table,
+                                           int32_t max_blocks, const int32_t* seqlens,
+                                           int32_t batch, int32_t q_len, int64_t max_seqlen,
+                                           float softmax_scale, int32_t num_splits,
+                                           int32_t* status_dev, void* out, void* stream) {
+  int nsm = 0;
+  if (!xmla::device_ok(&nsm)) return XMLA_ERR_UNSUPPORTED;
+  const size_t need = xmla_decode_workspace_size(batch, q_len, max_seqlen, nsm, num_splits);
+  if (need == 0) return XMLA_ERR_SHAPE;
+  if (need > xmla::kNoAllocScratchBytes) return XMLA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const xmla_status st = xmla::noalloc_scratch(&scratch);
+  if (st != XMLA_OK) return st;
+  return xmla_decode(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens, batch,
+                     q_len, max_seqlen, softmax_scale, num_splits, scratch,
+                     xmla::kNoAllocScratchBytes, status_dev, out, stream);
+}
+
+extern "C" xmla_status xmla_selftest_wait_timeout(int32_t* status_dev, uint64_t timeout_ns,
+                                                  void* stream) {
+  if (status_dev == nullptr) return XMLA_ERR_INVALID_ARG;
+  wait_timeout_selftest_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(status_dev, timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+}
+
+extern "C" const char* xmla_status_string(xmla_status s) {
+  switch (s) {
+    case XMLA_OK: return "ok";
+    case XMLA_ERR_INVALID_ARG: return "invalid argument";
+    case XMLA_ERR_SHAPE: return "unsupported shape";
+    case XMLA_ERR_WORKSPACE: return "workspace too small";
+    case XMLA_ERR_CUDA: return "CUDA error";
+    case XMLA_ERR_DEVICE_OOB: return "device: index out of range";
+    case XMLA_ERR_TIMEOUT: return "device: bounded wait timed out";
+    case XMLA_ERR_UNSUPPORTED: return "device not supported (needs sm_100a)";
+  }
+  return "unknown status";
+}

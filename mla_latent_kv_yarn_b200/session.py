@@ -132,13 +132,25 @@ class Decoder:
 
     def step(self, cfg, st: LayerState, q: torch.Tensor, c_new: torch.Tensor,
              k_new: torch.Tensor, new_pos: torch.Tensor, new_seq: torch.Tensor,
-             softmax_scale: float, out=None, stream=None, events=None) -> torch.Tensor:
+             softmax_scale: float, out=None, stream=None, events=None,
+             fused: bool = True) -> torch.Tensor:
         """One decode step on raw q: the q_len newest tokens (c_new, k_new raw)
-        are appended with their rope keys rotated, then the layer attends."""
-        xmla.xmla_cache_append(st.pool, st.num_blocks, st.block_table, st.max_blocks, self.batch,
-                               new_seq, new_pos, c_new, k_new, cfg, c_new.shape[0], self.status,
-                               stream)
-        return self.decode(cfg, st, q, softmax_scale, out, stream, events)
+        are appended with their rope keys rotated, then the layer attends.
+        fused=True uses xmla_decode_step (append inside the first kernel);
+        fused=False issues xmla_cache_append and then xmla_decode_profiled."""
+        out = self.out if out is None else out
+        if not fused:
+            xmla.xmla_cache_append(st.pool, st.num_blocks, st.block_table, st.max_blocks,
+                                   self.batch, new_seq, new_pos, c_new, k_new, cfg, c_new.shape[0],
+                                   self.status, stream)
+            return self.decode(cfg, st, q, softmax_scale, out, stream, events)
+        ev = events or (None, None)
+        xmla.xmla_decode_step(cfg, q, st.W_UK, st.W_UV, st.pool, st.num_blocks, st.block_table,
+                              st.max_blocks, st.seqlens, self.batch, self.q_len, self.max_seqlen,
+                              new_seq, new_pos, c_new, k_new, c_new.shape[0], softmax_scale,
+                              self.num_splits, self.workspace, self.ws_bytes, self.status, out,
+                              stream, ev[0], ev[1])
+        return out
 
     def check_status(self) -> int:
         return int(self.status.item())

@@ -25,7 +25,8 @@ STATUS_NAMES = {
 EXPORTS = [
     "xmla_yarn_default", "xmla_yarn_inv_freq", "xmla_softmax_scale", "xmla_rope_yarn",
     "xmla_cache_append", "xmla_decode_workspace_size", "xmla_decode_num_splits", "xmla_decode",
-    "xmla_decode_profiled", "xmla_decode_noalloc", "xmla_selftest_wait_timeout",
+    "xmla_decode_profiled", "xmla_decode_step", "xmla_decode_noalloc",
+    "xmla_selftest_wait_timeout",
     "xmla_status_string",
 ]
 
@@ -81,6 +82,9 @@ def lib() -> ctypes.CDLL:
         L.xmla_decode.restype = ctypes.c_int
         L.xmla_decode_profiled.argtypes = L.xmla_decode.argtypes + [vp, vp]
         L.xmla_decode_profiled.restype = ctypes.c_int
+        L.xmla_decode_step.argtypes = [cfgp, vp, vp, vp, vp, i64, vp, i32, vp, i32, i32, i64, vp, vp,
+                                       vp, vp, i64, f32, i32, vp, sz, vp, vp, vp, vp, vp]
+        L.xmla_decode_step.restype = ctypes.c_int
         L.xmla_decode_noalloc.argtypes = [cfgp, vp, vp, vp, vp, i64, vp, i32, vp, i32, i32, i64, f32,
                                           i32, vp, vp, vp]
         L.xmla_decode_noalloc.restype = ctypes.c_int
@@ -185,6 +189,23 @@ def xmla_decode_profiled(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_
                                       int(num_splits), _ptr(workspace), int(workspace_bytes),
                                       _ptr(status), _ptr(out), _stream(stream), ev[0], ev[1]),
            "xmla_decode_profiled")
+
+
+def xmla_decode_step(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens, batch,
+                     q_len, max_seqlen, seq_ids, positions, c_kv, k_pe, T, softmax_scale,
+                     num_splits, workspace, workspace_bytes, status, out, stream=None,
+                     attn_start=None, attn_stop=None) -> None:
+    """Append the step's T new rows (k_pe raw, rotated with cfg) and decode."""
+    ev = [None if e is None else (e.cuda_event if hasattr(e, "cuda_event") else int(e))
+          for e in (attn_start, attn_stop)]
+    _check(lib().xmla_decode_step(ctypes.byref(cfg), _ptr(q), _ptr(W_UK), _ptr(W_UV), _ptr(pool),
+                                  int(num_blocks), _ptr(block_table), int(max_blocks), _ptr(seqlens),
+                                  int(batch), int(q_len), int(max_seqlen), _ptr(seq_ids),
+                                  _ptr(positions), _ptr(c_kv), _ptr(k_pe), int(T),
+                                  float(softmax_scale), int(num_splits), _ptr(workspace),
+                                  int(workspace_bytes), _ptr(status), _ptr(out), _stream(stream),
+                                  ev[0], ev[1]),
+           "xmla_decode_step")
 
 
 def xmla_decode_noalloc(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens,

@@ -31,7 +31,7 @@ def f64(t: torch.Tensor) -> np.ndarray:
 
 
 def gpu_step(wl: workloads.Workload, inp: workloads.LayerInputs, cfg, *, num_splits: int = 0,
-             pool_fill=0.0, decoder: session.Decoder | None = None):
+             pool_fill=0.0, decoder: session.Decoder | None = None, fused: bool = True):
     """Fill the cache with every token but each sequence's q_len newest, then run
     one decode step (RoPE q, RoPE + append the new tokens, decode)."""
     dev = torch.device("cuda")
@@ -40,7 +40,7 @@ def gpu_step(wl: workloads.Workload, inp: workloads.LayerInputs, cfg, *, num_spl
     dec = decoder or session.Decoder(wl.batch, wl.q_len, wl.max_seqlen, dev, num_splits)
     q = inp.q.to(dev).clone()
     out = dec.step(cfg, st, q, new.c_kv.to(dev), new.k_pe.to(dev).clone(), new.positions.to(dev),
-                   new.seq_ids.to(dev), xmla.xmla_softmax_scale(cfg, 192))
+                   new.seq_ids.to(dev), xmla.xmla_softmax_scale(cfg, 192), fused=fused)
     torch.cuda.synchronize()
     return out.clone(), dec, st
 

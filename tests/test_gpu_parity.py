@@ -147,6 +147,45 @@ def test_decode_matches_expanded_oracle(batch, q_len, seqlens, splits):
     gc.assert_close(out, gc.oracle_out(wl, inp, ocfg), f"{batch}x{q_len} {seqlens} s={splits}")
 
 
+@pytest.mark.parametrize("batch,q_len,seqlens", [(1, 1, [300]), (2, 4, [1000, 257]),
+                                                 (4, 1, [8, 16, 24, 40])])
+def test_fused_step_equals_append_then_decode(batch, q_len, seqlens):
+    """xmla_decode_step runs the append inside the first kernel of the chain;
+    its output and the cache it leaves must be bit-identical to
+    xmla_cache_append followed by xmla_decode."""
+    wl = workloads.custom(batch, q_len, seqlens, seed=7 + sum(seqlens))
+    cfg, _ = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    out_f, dec_f, st_f = gc.gpu_step(wl, inp, cfg, fused=True)
+    out_u, dec_u, st_u = gc.gpu_step(wl, inp, cfg, fused=False)
+    assert dec_f.check_status() == 0 and dec_u.check_status() == 0
+    assert torch.equal(out_f.view(torch.int16), out_u.view(torch.int16))
+    assert torch.equal(st_f.pool.view(torch.int16), st_u.pool.view(torch.int16))
+
+
+def test_fused_step_with_no_new_rows_is_a_plain_decode():
+    wl = workloads.custom(2, 2, [129, 70], seed=11)
+    cfg, _ = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    dev = torch.device("cuda")
+    st = session.build_layer(cfg, wl, inp, dev)  # every token, new ones included
+    dec = session.Decoder(wl.batch, wl.q_len, wl.max_seqlen, dev)
+    q = inp.q.to(dev)
+    scale = xmla.xmla_softmax_scale(cfg, 192)
+    ref = dec.decode(cfg, st, q, scale).clone()
+    empty_i32 = torch.empty(0, dtype=torch.int32, device=dev)
+    empty_i64 = torch.empty(0, dtype=torch.int64, device=dev)
+    empty_bf = torch.empty((0, 576), dtype=torch.bfloat16, device=dev)
+    out = torch.empty_like(ref)
+    xmla.xmla_decode_step(cfg, q, st.W_UK, st.W_UV, st.pool, st.num_blocks, st.block_table,
+                          st.max_blocks, st.seqlens, wl.batch, wl.q_len, wl.max_seqlen, empty_i32,
+                          empty_i64, empty_bf, empty_bf, 0, scale, 0, dec.workspace, dec.ws_bytes,
+                          dec.status, out)
+    torch.cuda.synchronize()
+    assert dec.check_status() == 0
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+
+
 def test_decode_ignores_garbage_past_sequence_end():
     """Cache rows past a sequence's end (inside its last block) hold NaN here."""
     wl = workloads.custom(2, 1, [100, 130], seed=21)
