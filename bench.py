@@ -231,6 +231,18 @@ def run_reference(args, wl):
 
 # ------------------------------------------------------------------ GPU arm
 
+# the translation unit of the split-K kernel: its source and the headers it includes
+KERNEL_SOURCES = ["mla_decode.cu", "decode_chain.h", "xmla_device.cuh", "yarn.cuh"]
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "mla_latent_kv_yarn_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def traffic_record(kernel_src_sha: str, name: str):
     """DRAM bytes per launch of the split-K kernel from a committed ncu summary,
     valid only while the kernel source is unchanged."""
@@ -238,7 +250,7 @@ def traffic_record(kernel_src_sha: str, name: str):
     try:
         with open(p) as f:
             d = json.load(f)
-        if d.get("kernel_source_sha256") == kernel_src_sha:
+        if d.get("kernel_sources_sha256") == kernel_src_sha:
             return float(d["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -384,8 +396,7 @@ def run_xmla(args, wl):
     peak, peak_kind = measured_peaks()
     attn_mean_ms = statistics.mean(attn_ms)
     achieved = cache_bytes_layer / (attn_mean_ms * 1e-3) / 1e9
-    ksha = hashlib.sha256(open(os.path.join(ROOT, "mla_latent_kv_yarn_b200", "csrc",
-                                            "mla_decode.cu"), "rb").read()).hexdigest()
+    ksha = kernel_sources_sha()
     traffic = traffic_record(ksha, wl.name)
     # per layer and step: prologue (append + q absorb), split-K attention, combine
     launches = 3 * wl.layers * args.steps
