@@ -232,7 +232,7 @@ def run_reference(args, wl):
 # ------------------------------------------------------------------ GPU arm
 
 # the translation unit of the split-K kernel: its source and the headers it includes
-KERNEL_SOURCES = ["mla_decode.cu", "decode_chain.h", "xmla_device.cuh", "yarn.cuh"]
+KERNEL_SOURCES = ["mla_decode.cu", "split_kv.h", "xmla_device.cuh"]
 
 
 def kernel_sources_sha() -> str:

@@ -159,32 +159,29 @@ cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_
 // ---------------------------------------------------------------- combine + W_UV
 
 // Cluster of 8 CTAs per (head h, chunk of up to kCombineRows output rows).
-// CTA `slice` owns latent dims [64 slice, 64 slice + 64).  All rows of the
-// chunk are merged together: 16 groups of 16 threads (one float4 of the slice
-// each) are shared out over the rows, and a row's splits are dealt round-robin
-// over its groups, so one pass of loads covers the chunk.  Every split is
-// weighted by 2^(m_s - M) against the row's overall maximum M and the sum is
-// divided by L = sum_s l_s 2^(m_s - M).  The CTA then multiplies its merged
-// 64 dims by the matching 64 rows of W_UV[h] and sends each 16-column block of
-// that product to the CTA that owns the block (distributed shared memory); the
-// owner adds the 8 contributions and writes its 16 output columns.
+// CTA `slice` owns latent dims [64 slice, 64 slice + 64).
+//  * Merge.  16 groups of 16 threads (one float4 of the slice each) are shared
+//    out over the chunk's rows, and a row's splits are dealt round-robin over
+//    its groups, so one pass of loads covers the chunk.  Lane k of a group also
+//    loads (m, l) of the group's k-th split; a group merges its splits against
+//    its own maximum m_g (weights 2^(m_s - m_g), shared by shuffles), so no
+//    pass over the row's statistics precedes the loads.  The groups of a row
+//    are then combined with weights 2^(m_g - M) against the row maximum M and
+//    divided by L = sum_g l_g 2^(m_g - M).  A split that saw no token (l = 0,
+//    partial O never written) is skipped, not multiplied by zero.
+//  * W_UV.  The merged, normalised 64 dims are multiplied by the slice's 64
+//    rows of W_UV[h]; with fewer than 4 rows the 64 dims are also split over
+//    the threads.  Each 16-column block of the product is written into the
+//    shared memory of the CTA that owns the block (distributed shared memory);
+//    the owner adds the 8 contributions in a fixed order and writes out.
 constexpr int kSlices = 8;
 constexpr int kSliceDims = kDLatent / kSlices;        // 64
 constexpr int kCombineRows = 16;
 constexpr int kCombineThreads = 256;
-constexpr int kCombineWarps = kCombineThreads / 32;
 constexpr int kCombineGroups = kCombineThreads / 16;  // 16 threads x float4 cover a split row's slice
-constexpr int kCombineDepth = 10;                     // split rows each thread keeps in flight
-constexpr int kStatDepth = 4;                         // (m, l) pairs each lane keeps in flight
+constexpr int kCombineDepth = 10;                     // split rows each thread keeps in flight (<= 16)
 constexpr int kColsPerSlice = kDV / kSlices;          // 16
-
-// Online (max, sum-of-exp2) pair merge.
-__device__ __forceinline__ void lse_merge(float& m, float& l, float m2, float l2) {
-  const float mx = fmaxf(m, m2);
-  if (mx == -INFINITY) return;
-  l = l * ex2(m - mx) + l2 * ex2(m2 - mx);
-  m = mx;
-}
+static_assert(kCombineDepth <= 16, "a group's lanes carry (m, l) of at most 16 splits");
 
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -196,6 +193,13 @@ __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void fma4(float4& acc, float w, const float4& x) {
+  acc.x = fmaf(w, x.x, acc.x);
+  acc.y = fmaf(w, x.y, acc.y);
+  acc.z = fmaf(w, x.z, acc.z);
+  acc.w = fmaf(w, x.w, acc.w);
+}
+
 __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThreads, 3)
     combine_uv_kernel(const float* part_o, const float* part_ml,
                       const __nv_bfloat16* __restrict__ W_UV, __nv_bfloat16* __restrict__ out,
@@ -205,9 +209,10 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThread
   // are not taken as invariant and stay behind the griddepcontrol.wait below.
   __shared__ __align__(16) __nv_bfloat16 w_s[kSliceDims][kDV];  // this slice's rows of W_UV[h]
   __shared__ __align__(16) float4 acc_s[kCombineGroups][kSliceDims / 4];
+  __shared__ float grp_m[kCombineGroups], grp_l[kCombineGroups];
   __shared__ __align__(16) float o_s[kCombineRows][kSliceDims];
+  __shared__ __align__(16) float prod_s[kCombineRows][kDV];  // [c part * nr + row][v]
   __shared__ __align__(16) float inbox[kSlices][kCombineRows][kColsPerSlice];  // by sender slice
-  __shared__ float stat_m[kCombineRows][kCombineWarps], stat_l[kCombineRows][kCombineWarps];
   cg::cluster_group cluster = cg::this_cluster();
   const int slice = (int)cluster.block_rank();
   const int cid = blockIdx.x / kSlices;
@@ -216,8 +221,6 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThread
   const int r0 = chunk * kCombineRows;
   const int nr = min(kCombineRows, rows - r0);
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
   pdl_launch_dependents();
   // first half of the barrier that guarantees every CTA of the cluster runs
   // before any of them writes into another's shared memory
@@ -231,134 +234,125 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThread
       dst[tid + kCombineThreads * e] = src[tid + kCombineThreads * e];
   }
 
-  // partial row of split 0 for chunk row rr; split s is s * rows_per_cta rows further
-  auto split0_row = [&](int rr) -> int64_t {
-    const int r = r0 + rr;  // r = b*q_len + j
-    const int b = r / q_len, j = r % q_len;
-    const int ridx = j * kHeads + h;
-    return ((int64_t)b * groups + ridx / rows_per_cta) * nsplit * rows_per_cta + ridx % rows_per_cta;
-  };
-  const int q4 = tid & 15;  // float4 of the 64-dim slice
+  // thread -> (row, group of the row, float4 of the slice)
+  const int q4 = tid & 15;
   const int grp = tid >> 4;
   const int gpr = max(1, kCombineGroups / nr);  // groups per row
   const int my_rr = grp / gpr;
   const int sub = grp % gpr;
   const bool active = my_rr < nr;
-  const int64_t base = active ? split0_row(my_rr) : 0;
+  int64_t base = 0;  // partial row of split 0; split s is s * rows_per_cta rows further
+  if (active) {
+    const int r = r0 + my_rr;  // r = b*q_len + j
+    const int b = r / q_len, j = r % q_len;
+    const int ridx = j * kHeads + h;
+    base = ((int64_t)b * groups + ridx / rows_per_cta) * nsplit * rows_per_cta + ridx % rows_per_cta;
+  }
   const float* po = part_o + base * kDLatent + slice * kSliceDims + 4 * q4;
-  const float* pm = part_ml + 2 * base;          // m of split s at pm[s * m_stride]
+  const float2* pml = reinterpret_cast<const float2*>(part_ml) + base;
   const int o_stride = rows_per_cta * kDLatent;  // floats between splits (nsplit * o_stride < 2^31)
-  const int m_stride = 2 * rows_per_cta;
-  const int wpr = max(1, kCombineWarps / nr);    // warps per row for the statistics
 
   pdl_wait();  // the split partials come from the decode kernel
 
-  // first batch of this thread's split rows, issued before the row statistics
-  // so that both sets of loads are in flight together.  A split that saw no
-  // token has m = -inf (and l = 0); only m is needed to recognise it.
   float4 v[kCombineDepth];
-  float ms[kCombineDepth];
 #pragma unroll
   for (int k = 0; k < kCombineDepth; ++k) {
     const int s = sub + gpr * k;
-    const bool in = active && s < nsplit;
-    v[k] = in ? *reinterpret_cast<const float4*>(po + s * o_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
-    ms[k] = in ? pm[s * m_stride] : -INFINITY;
+    v[k] = active && s < nsplit ? *reinterpret_cast<const float4*>(po + s * o_stride)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  const int s_lane = sub + gpr * q4;  // the split whose (m, l) this lane loads
+  const float2 ml = active && s_lane < nsplit ? pml[(int64_t)s_lane * rows_per_cta]
+                                              : make_float2(-INFINITY, 0.f);
 
-  // row statistics: `wpr` warps share a row's splits (part p takes splits
-  // 32 p + lane, then every 32 wpr further); each warp reduces its share
-  {
-    const int part = warp % wpr;
-    for (int rr = warp / wpr; rr < nr; rr += kCombineWarps / wpr) {
-      const float2* rml = reinterpret_cast<const float2*>(part_ml) + split0_row(rr);
-      float m = -INFINITY, l = 0.f;
-      for (int s0 = 32 * part; s0 < nsplit; s0 += 32 * wpr * kStatDepth) {
-        float2 x[kStatDepth];
+  // group maximum over its first 16 splits (lanes of one group: 16 consecutive)
+  float m_g = ml.y > 0.f ? ml.x : -INFINITY;
 #pragma unroll
-        for (int k = 0; k < kStatDepth; ++k) {
-          const int s = s0 + lane + 32 * wpr * k;
-          x[k] = s < nsplit ? rml[(int64_t)s * rows_per_cta] : make_float2(-INFINITY, 0.f);
-        }
+  for (int o = 8; o > 0; o >>= 1) m_g = fmaxf(m_g, __shfl_xor_sync(0xffffffffu, m_g, o));
+  float l_g = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int k = 0; k < kStatDepth; ++k)
-          if (x[k].y > 0.f) lse_merge(m, l, x[k].x, x[k].y);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-        const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-        lse_merge(m, l, m2, l2);
-      }
-      if (lane == 0) {
-        stat_m[rr][part] = m;
-        stat_l[rr][part] = l;
-      }
+  for (int k = 0; k < kCombineDepth; ++k) {
+    const float mk = __shfl_sync(0xffffffffu, ml.x, k, 16);
+    const float lk = __shfl_sync(0xffffffffu, ml.y, k, 16);
+    if (lk > 0.f) {  // also false past the group's last split
+      const float w = ex2(mk - m_g);
+      l_g = fmaf(w, lk, l_g);
+      fma4(acc, w, v[k]);
     }
   }
-  __syncthreads();
-
-  // weighted sum of this thread's split rows (the partial O of a split that saw
-  // no token was never written: it is skipped, not multiplied by zero)
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  // splits past the first kCombineDepth of the group (many splits per group only):
+  // loaded one by one, merged online
   if (active) {
-    float M = stat_m[my_rr][0];
-    for (int p = 1; p < wpr; ++p) M = fmaxf(M, stat_m[my_rr][p]);
-    for (int k0 = 0;; k0 += kCombineDepth) {
-#pragma unroll
-      for (int k = 0; k < kCombineDepth; ++k) {
-        if (ms[k] != -INFINITY) {
-          const float wgt = ex2(ms[k] - M);
-          acc.x = fmaf(wgt, v[k].x, acc.x);
-          acc.y = fmaf(wgt, v[k].y, acc.y);
-          acc.z = fmaf(wgt, v[k].z, acc.z);
-          acc.w = fmaf(wgt, v[k].w, acc.w);
+    for (int s = sub + gpr * kCombineDepth; s < nsplit; s += gpr) {
+      const float2 x = pml[(int64_t)s * rows_per_cta];
+      if (x.y > 0.f) {
+        if (x.x > m_g) {
+          const float c = m_g == -INFINITY ? 0.f : ex2(m_g - x.x);
+          l_g *= c;
+          acc.x *= c;
+          acc.y *= c;
+          acc.z *= c;
+          acc.w *= c;
+          m_g = x.x;
         }
-      }
-      const int k1 = k0 + kCombineDepth;
-      if (sub + gpr * k1 >= nsplit) break;
-#pragma unroll
-      for (int k = 0; k < kCombineDepth; ++k) {
-        const int s = sub + gpr * (k1 + k);
-        const bool in = s < nsplit;
-        v[k] = in ? *reinterpret_cast<const float4*>(po + s * o_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
-        ms[k] = in ? pm[s * m_stride] : -INFINITY;
+        const float w = ex2(x.x - m_g);
+        l_g = fmaf(w, x.y, l_g);
+        fma4(acc, w, *reinterpret_cast<const float4*>(po + s * o_stride));
       }
     }
   }
   acc_s[grp][q4] = acc;
+  if (q4 == 0) {
+    grp_m[grp] = m_g;
+    grp_l[grp] = l_g;
+  }
   __syncthreads();
   for (int e = tid; e < nr * kSliceDims; e += kCombineThreads) {
     const int rr = e / kSliceDims, d = e % kSliceDims;
-    float M = stat_m[rr][0];
-    for (int p = 1; p < wpr; ++p) M = fmaxf(M, stat_m[rr][p]);
-    float L = 0.f;
-    for (int p = 0; p < wpr; ++p)
-      if (stat_l[rr][p] > 0.f) L += stat_l[rr][p] * ex2(stat_m[rr][p] - M);
-    const float* a = reinterpret_cast<const float*>(&acc_s[rr * gpr][0]) + d;
-    float t = 0.f;
-    for (int g = 0; g < gpr; ++g) t += a[g * kSliceDims];
+    const int g0 = rr * gpr;
+    float M = -INFINITY;
+    for (int g = 0; g < gpr; ++g) M = fmaxf(M, grp_m[g0 + g]);
+    float L = 0.f, t = 0.f;
+    for (int g = 0; g < gpr; ++g) {
+      if (grp_l[g0 + g] > 0.f) {
+        const float w = ex2(grp_m[g0 + g] - M);
+        L = fmaf(w, grp_l[g0 + g], L);
+        t = fmaf(w, reinterpret_cast<const float*>(&acc_s[g0 + g][0])[d], t);
+      }
+    }
     o_s[rr][d] = L > 0.f ? t / L : 0.f;
   }
   __syncthreads();
 
-  // slice product: sum over the slice's 64 latent dims c of o[r][c] W_UV[h][c][v]
-  // for the column pair (2 vp, 2 vp + 1), sent to the CTA owning that column block
-  cluster_wait_acquire();  // every CTA of the cluster is running
+  // slice product prod[r][v] = sum over the slice's 64 dims c of o[r][c] W_UV[h][c][v]:
+  // thread = (column pair vp, unit u of 4); with cs = 4 / nr parts of the 64 dims
+  // (cs = 1 from 4 rows up), unit u takes dims part u % cs of rows u / cs, u / cs + 4 / cs, ...
   {
     const int vp = tid & (kDV / 2 - 1);
-    const int owner = (2 * vp) / kColsPerSlice;
-    float* dst = cluster.map_shared_rank(&inbox[slice][0][0], owner);
-    for (int rr = tid / (kDV / 2); rr < nr; rr += kCombineThreads / (kDV / 2)) {
+    const int u = tid / (kDV / 2);
+    const int cs = nr >= 4 ? 1 : (nr == 1 ? 4 : 2);
+    const int cq = u % cs;
+    const int c0 = cq * (kSliceDims / cs), c1 = c0 + kSliceDims / cs;
+    for (int rr = u / cs; rr < nr; rr += 4 / cs) {
       float a0 = 0.f, a1 = 0.f;
 #pragma unroll 16
-      for (int c = 0; c < kSliceDims; ++c) {
+      for (int c = c0; c < c1; ++c) {
         const float2 w = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&w_s[c][0])[vp]);
         const float x = o_s[rr][c];
         a0 = fmaf(x, w.x, a0);
         a1 = fmaf(x, w.y, a1);
       }
-      *reinterpret_cast<float2*>(dst + rr * kColsPerSlice + (2 * vp) % kColsPerSlice) = make_float2(a0, a1);
+      *reinterpret_cast<float2*>(&prod_s[cq * nr + rr][2 * vp]) = make_float2(a0, a1);
+    }
+    __syncthreads();
+    cluster_wait_acquire();  // every CTA of the cluster is running
+    for (int e = tid; e < nr * kDV; e += kCombineThreads) {
+      const int rr = e / kDV, v = e % kDV;
+      float t = prod_s[rr][v];
+      for (int k = 1; k < cs; ++k) t += prod_s[k * nr + rr][v];
+      float* dst = cluster.map_shared_rank(&inbox[slice][0][0], v / kColsPerSlice);
+      dst[rr * kColsPerSlice + v % kColsPerSlice] = t;
     }
   }
   cluster_arrive_release();

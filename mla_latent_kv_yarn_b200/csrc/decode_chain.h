@@ -15,37 +15,13 @@
 
 #include <cstdint>
 
+#include "split_kv.h"
 #include "xmla_device.cuh"
 #include "yarn.cuh"
 
 namespace xmla {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kMaxSplits = 1024;
-
-// Arguments of the split-K attention kernel.  Partial results are laid out
-// per work item (sequence b, row group g, split s) in that order.
-struct DecodeParams {
-  const int32_t* block_table;
-  const int32_t* seqlens;
-  float* part_o;   // [items, NR, 512] unnormalised O of each split
-  float* part_ml;  // [items, NR, 2] running max m (log2 units) and sum l
-  int32_t* status;
-  int64_t num_blocks;
-  int64_t max_seqlen;
-  uint64_t wait_limit_ns;
-  int32_t max_blocks;
-  int32_t batch;
-  int32_t q_len;
-  int32_t groups;
-  int32_t nsplit;
-};
-
-// Split-K attention over `items` work items; nr = rows per CTA (32 or 64).
-// pool_map: 576-column rows of the cache pool, box 64 x 64; q_map: rows of
-// q_ext, box 64 x nr (both 128-byte swizzled).
-cudaError_t launch_split_kv(int nr, const CUtensorMap& pool_map, const CUtensorMap& q_map,
-                            const DecodeParams& dp, int64_t items, cudaStream_t st);
 
 // q_ext[r, h] for rows r = b*q_len + j; qscale = softmax scale * log2 e.
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,

@@ -23,7 +23,8 @@
 #include <cmath>
 #include <cstdint>
 
-#include "decode_chain.h"
+#include "split_kv.h"
+#include "xmla_device.cuh"
 
 namespace xmla {
 

@@ -134,6 +134,9 @@ SMALL = [
     (2, 4, [1000, 257], 0),
     (1, 8, [2000], 0),
     (1, 4, [4], 0),
+    # more splits per combine group than it keeps in flight (merged online)
+    (2, 8, [1500, 900], 0),
+    (1, 1, [20000], 200),
 ]
 
 
