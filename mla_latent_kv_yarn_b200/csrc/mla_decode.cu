@@ -211,22 +211,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       int li = 0, ri = 0;
       uint32_t lph = 0, rph = 0;
       int64_t lat_issued = 0, rope_issued = 0;
-      bool ok = true, q_issued = false;
+      bool ok = true;
       // block ids are fetched four pages ahead so their load latency is hidden
       const int32_t* bt = p.block_table + (int64_t)b * p.max_blocks + p_begin;
       int32_t nb0 = bt[0];
       int32_t nb1 = n_pages > 1 ? bt[1] : 0;
       int32_t nb2 = n_pages > 2 ? bt[2] : 0;
       int32_t nb3 = n_pages > 3 ? bt[3] : 0;
-      const int64_t first_new = seqlen - p.q_len;  // first row appended by this step
-      bool waited = false;
+      // q_ext, the rows this step appends, and any cache rows an earlier kernel
+      // on the stream may still be writing: all of them are read only after
+      // the kernels launched before have completed.  (This CTA could only start
+      // once the previous kernel's CTAs had left its SM, so the wait is short.)
+      // q_ext is loaded first, so the first QK product waits only for its page.
+      pdl_wait();
+      mbar_arrive_expect_tx(bar(L::kBarQ), 9u * L::kQChunk);
+      for (int c = 0; c < 9; ++c)
+        tma_load_2d(base + L::kOffQ + c * L::kQChunk, &tmap_q, c * 64, qrow0, bar(L::kBarQ));
       for (int i = 0; i < n_pages && ok; ++i) {
-        if (!waited && (p_begin + i + 1) * kPage > first_new) {
-          // this page holds rows written by the kernels launched just before:
-          // wait for them (through q_absorb's completion) before reading it
-          pdl_wait();
-          waited = true;
-        }
         int32_t blk = nb0;
         nb0 = nb1;
         nb1 = nb2;
@@ -262,20 +263,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                          bar(L::kBarRopeFull + ri), stream_policy);
         ++rope_issued;
         if (++ri == L::kRopeSlots) { ri = 0; rph ^= 1u; }
-        if (!q_issued) {
-          // q_ext is the previous kernel's output: wait for it only after the
-          // first page is on its way.
-          if (!waited) pdl_wait();
-          waited = true;
-          mbar_arrive_expect_tx(bar(L::kBarQ), 9u * L::kQChunk);
-          for (int c = 0; c < 9; ++c)
-            tma_load_2d(base + L::kOffQ + c * L::kQChunk, &tmap_q, c * 64, qrow0, bar(L::kBarQ));
-          q_issued = true;
-        }
       }
       // Every copy issued must land before the CTA may exit: wait for the last
       // phase armed on each slot (immediate when the consumer already saw it).
-      if (q_issued) mbar_wait(bar(L::kBarQ), 0, nullptr, p.status, p.wait_limit_ns);
+      mbar_wait(bar(L::kBarQ), 0, nullptr, p.status, p.wait_limit_ns);
       for (int s = 0; s < L::kLatSlots; ++s) {
         if (lat_issued > s) {
           const int64_t last = s + ((lat_issued - 1 - s) / L::kLatSlots) * L::kLatSlots;
