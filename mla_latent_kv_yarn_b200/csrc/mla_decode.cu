@@ -207,7 +207,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if (lane == 0 && n_pages > 0) {
       tma_prefetch_desc(&tmap_pool);
       tma_prefetch_desc(&tmap_q);
-      const uint64_t stream_policy = policy_evict_first();
+      // Pages are read once at q_len 1: evict them first.  With two row groups
+      // (q_len > 1) both groups' CTAs stream the same pages at about the same
+      // time, and the second read should find them in L2.
+      const uint64_t stream_policy = NR == 32 ? policy_evict_first() : policy_evict_normal();
       int li = 0, ri = 0;
       uint32_t lph = 0, rph = 0;
       int64_t lat_issued = 0, rope_issued = 0;
