@@ -35,6 +35,12 @@ with its reason in the design notes of the repository):
   * kv_b_proj output rows [256h, 256h+128) are head h's K_nope rows (W_UK[h],
     shape [128, 512]) and rows [256h+128, 256h+256) its V rows; W_UV[h] is
     their transpose, shape [512, 128].  No bias (attention_bias false).
+  * kv_a_proj_with_mqa ([P5] MLA section: Linear(hidden_size, 512 + 64);
+    hidden_size 3584 from the model summary page "Xing4.0" (alphasignal.ai),
+    architecture paragraph) has no bias (attention_bias false) and no norm
+    is printed between it and the cache: output columns [0, 512) are c_kv,
+    [512, 576) the raw rope key, each rounded to bf16 as a bf16 Linear does
+    before RoPE and caching.
   * A context of N tokens holds positions 0..N-1 and includes the q_len new
     tokens, which are its last q_len entries; query j sits at position
     N - q_len + j and sees tokens t <= N - q_len + j.
@@ -254,6 +260,25 @@ def mla_attention_absorbed(q: np.ndarray, c_kv: np.ndarray, k_pe_rot: np.ndarray
     P = P / P.sum(axis=1, keepdims=True)
     o_lat = (P @ c_kv).reshape(q_len, H, -1)                                # [q_len, H, 512]
     return np.einsum("jhc,hcv->jhv", o_lat, W_UV)
+
+
+HIDDEN = 3584  # model hidden size (the summary page's architecture paragraph)
+
+
+def kv_a_projection(hidden: np.ndarray, W_kva: np.ndarray,
+                    bias: np.ndarray | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """kv_a_proj_with_mqa of token hidden states, before any rounding.
+
+    [P5] MLA section: kv_a_proj_with_mqa = Linear(hidden_size,
+    kv_lora_rank + qk_rope_head_dim) compresses each token into the 512-dim
+    latent and the 64-dim (not yet rotated) rope key.  hidden: [T, HIDDEN];
+    W_kva: [576, HIDDEN] (Linear weight layout: output x input); bias: [576]
+    or None.  Returns (c_kv [T, 512], k_pe [T, 64]) in float64.
+    """
+    out = np.asarray(hidden, dtype=np.float64) @ np.asarray(W_kva, dtype=np.float64).T
+    if bias is not None:
+        out = out + np.asarray(bias, dtype=np.float64)
+    return out[:, :D_LATENT], out[:, D_LATENT:]
 
 
 def cache_append(pool_u16: np.ndarray, block_table: np.ndarray, seq_ids: np.ndarray,

@@ -355,3 +355,50 @@ def test_repository_cache_row_is_576_elements():
     assert kb.kv_bytes_per_token(kb.mla_elems_latent_rope(), 1) == 1152
     assert per_token == 45 * 1024
     assert kb.cache_bytes(262144, per_token) / kb.GiB == 11.25
+
+
+# ------------------------------------------------------------------ kv_a_proj_with_mqa
+
+def test_kv_projection_selection_weights_copy_hidden_dims():
+    """A weight whose rows are unit vectors selects hidden dims: the first 512
+    selected dims land in c_kv and the last 64 in the rope key, in row order."""
+    rng = np.random.default_rng(31)
+    hidden = rng.standard_normal((5, om.HIDDEN))
+    pick = rng.permutation(om.HIDDEN)[:576]
+    W = np.zeros((576, om.HIDDEN))
+    W[np.arange(576), pick] = 1.0
+    c, k = om.kv_a_projection(hidden, W)
+    assert np.array_equal(c, hidden[:, pick[:512]])
+    assert np.array_equal(k, hidden[:, pick[512:]])
+
+
+def test_kv_projection_zero_weight_gives_the_bias():
+    rng = np.random.default_rng(32)
+    bias = rng.standard_normal(576)
+    c, k = om.kv_a_projection(rng.standard_normal((3, om.HIDDEN)), np.zeros((576, om.HIDDEN)), bias)
+    assert np.array_equal(c, np.broadcast_to(bias[:512], (3, 512)))
+    assert np.array_equal(k, np.broadcast_to(bias[512:], (3, 64)))
+
+
+def test_kv_projection_differences_of_hidden_pairs():
+    """Row j = e_{2j} - e_{2j+1}: output j is hidden[2j] - hidden[2j+1]."""
+    rng = np.random.default_rng(33)
+    hidden = rng.integers(-1000, 1000, (4, om.HIDDEN)).astype(np.float64)
+    W = np.zeros((576, om.HIDDEN))
+    j = np.arange(576)
+    W[j, 2 * j] = 1.0
+    W[j, 2 * j + 1] = -1.0
+    c, k = om.kv_a_projection(hidden, W)
+    want = hidden[:, 0:1152:2] - hidden[:, 1:1152:2]
+    assert np.array_equal(np.concatenate([c, k], axis=1), want)
+
+
+def test_kv_projection_is_linear_in_the_hidden_state():
+    rng = np.random.default_rng(34)
+    W = rng.standard_normal((576, om.HIDDEN)) / 60.0
+    h1, h2 = rng.standard_normal((2, 3, om.HIDDEN))
+    c1, k1 = om.kv_a_projection(h1, W)
+    c2, k2 = om.kv_a_projection(h2, W)
+    c3, k3 = om.kv_a_projection(2.5 * h1 - h2, W)
+    assert np.allclose(c3, 2.5 * c1 - c2, rtol=0, atol=1e-10)
+    assert np.allclose(k3, 2.5 * k1 - k2, rtol=0, atol=1e-10)
