@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--impl", default="xmla", choices=["xmla", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--with-producer", action="store_true",
+                    help="the step starts from the new tokens' hidden states: "
+                         "kv_a_proj_with_mqa + RoPE + append (xmla_kv_produce), then decode")
     return ap.parse_args()
 
 
@@ -279,11 +282,13 @@ def run_xmla(args, wl):
         inp = workloads.layer_inputs(wl, layer, dev)
         prefix, new = session.split_prefix(wl, inp)
         st = session.build_layer(cfg, wl, prefix, dev)
-        layers.append({"st": st, "q": inp.q.clone(), "k_new": new.k_pe.clone(),
-                       "c_new": new.c_kv.clone(), "pos": new.positions.clone(),
-                       "sid": new.seq_ids.clone(),
-                       "out": torch.empty((wl.batch, wl.q_len, 32, 128), dtype=torch.bfloat16,
-                                          device=dev)})
+        L = {"st": st, "q": inp.q.clone(), "k_new": new.k_pe.clone(),
+             "c_new": new.c_kv.clone(), "pos": new.positions.clone(),
+             "sid": new.seq_ids.clone(),
+             "out": torch.empty((wl.batch, wl.q_len, 32, 128), dtype=torch.bfloat16, device=dev)}
+        if args.with_producer:
+            L["hidden"], L["W_kva"] = workloads.producer_inputs(wl, layer, dev)
+        layers.append(L)
         del inp, prefix, new
     torch.cuda.synchronize()
     dec = session.Decoder(wl.batch, wl.q_len, wl.max_seqlen, dev)
@@ -296,8 +301,12 @@ def run_xmla(args, wl):
 
     def step(events=True):
         for L, ev in zip(layers, ev_attn):
-            dec.step(cfg, L["st"], L["q"], L["c_new"], L["k_new"], L["pos"], L["sid"], scale,
-                     out=L["out"], events=ev if events else None)
+            if args.with_producer:
+                dec.step_from_hidden(cfg, L["st"], L["q"], L["hidden"], L["W_kva"], L["pos"],
+                                     L["sid"], scale, out=L["out"], events=ev if events else None)
+            else:
+                dec.step(cfg, L["st"], L["q"], L["c_new"], L["k_new"], L["pos"], L["sid"], scale,
+                         out=L["out"], events=ev if events else None)
 
     # eager warm-up (loads modules), then capture the step twice: `graph` is what
     # is timed; `graph_k` also records CUDA events around the split-K kernel
@@ -367,7 +376,8 @@ def run_xmla(args, wl):
     status = dec.check_status()
 
     # ---- end to end through the API: pinned host inputs in, result out, every step
-    h_in = [{k: L[k].cpu().pin_memory() for k in ("q", "k_new", "c_new", "pos", "sid")}
+    step_inputs = ("q", "hidden", "pos", "sid") if args.with_producer else ("q", "k_new", "c_new", "pos", "sid")
+    h_in = [{k: L[k].cpu().pin_memory() for k in step_inputs}
             for L in layers]
     h_out = [torch.empty_like(L["out"], device="cpu").pin_memory() for L in layers]
     h2d = sum(t.numel() * t.element_size() for d in h_in for t in d.values())
@@ -398,7 +408,8 @@ def run_xmla(args, wl):
     achieved = cache_bytes_layer / (attn_mean_ms * 1e-3) / 1e9
     ksha = kernel_sources_sha()
     traffic = traffic_record(ksha, wl.name)
-    # per layer and step: prologue (append + q absorb), split-K attention, combine
+    # per layer and step: prologue (append or producer + q absorb), split-K
+    # attention, combine
     launches = 3 * wl.layers * args.steps
 
     if rank == 0:
@@ -407,7 +418,9 @@ def run_xmla(args, wl):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(wl, world),
+            "config": dict(workload_config(wl, world), **(
+                {"step": "hidden states in: kv_a_proj_with_mqa + RoPE + append, then decode"}
+                if args.with_producer else {})),
             "attended_tokens_per_s": round(tokens_step * args.steps / (total_ms * 1e-3), 1),
             "pct_of_hbm_peak": round(100.0 * gbs / (peak * world), 2),
             "roofline": {"bound": "hbm", "kernel": f"mla_decode_kernel<{32 if wl.q_len == 1 else 64}>",

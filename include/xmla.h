@@ -129,6 +129,30 @@ xmla_status xmla_cache_append(void* pool, int64_t num_blocks, const int32_t* blo
                               const xmla_yarn_cfg* rope_cfg, int64_t T, int32_t* status_dev,
                               void* stream);
 
+/* Produce and append the cache rows of T tokens from their hidden states
+ * ([P5] MLA section: kv_a_proj_with_mqa = Linear(hidden_size, 512 + 64)
+ * compresses a token into the cached latent and rope key; hidden size 3584 from
+ * the model summary page "Xing4.0", architecture paragraph; [P1] section 一:
+ * attention_bias false).  For i < T:
+ *   y = hidden[i] . W_kva^T (+ bias), each of the 576 outputs rounded to bf16;
+ *   c_kv = y[0:512], k_raw = y[512:576];
+ *   pool[block_table[seq_ids[i]*max_blocks + positions[i]/64]][positions[i] % 64]
+ *       = [c_kv | k_rot]
+ * where k_rot is the YaRN RoPE of k_raw at positions[i] with rope_cfg (float64
+ * angle, one bf16 rounding, as xmla_rope_yarn), or k_raw when rope_cfg is NULL.
+ * Accumulation in fp32.
+ *   hidden: device bf16 [T, 3584], 16-byte aligned;
+ *   W_kva: device bf16 [576, 3584] (Linear weight layout), 16-byte aligned;
+ *   bias: device bf16 [576] or NULL (no bias);
+ *   pool, block_table, max_blocks, batch, seq_ids, positions, status_dev: as in
+ *   xmla_cache_append (rows out of range are skipped and reported).
+ * T == 0 is a no-op.  Errors: XMLA_ERR_INVALID_ARG, XMLA_ERR_SHAPE, XMLA_ERR_CUDA. */
+xmla_status xmla_kv_produce(const void* hidden, const void* W_kva, const void* bias, int64_t T,
+                            const xmla_yarn_cfg* rope_cfg, void* pool, int64_t num_blocks,
+                            const int32_t* block_table, int32_t max_blocks, int32_t batch,
+                            const int32_t* seq_ids, const int64_t* positions,
+                            int32_t* status_dev, void* stream);
+
 /* Bytes of device workspace xmla_decode needs for these sizes on a device with
  * num_sms SMs (num_splits = 0 picks the split count automatically, > 0 forces
  * it).  Returns 0 for unsupported sizes. */
@@ -213,6 +237,25 @@ xmla_status xmla_decode_step(const xmla_yarn_cfg* cfg, const void* q, const void
                              int32_t num_splits, void* workspace, size_t workspace_bytes,
                              int32_t* status_dev, void* out, void* stream, void* attn_start,
                              void* attn_stop);
+
+/* One decode step from the new tokens' hidden states: xmla_kv_produce (the
+ * kv_a_proj_with_mqa projection, RoPE of the rope key with cfg, append) and then
+ * xmla_decode_profiled, with the producer's blocks inside the first kernel of
+ * the decode chain beside the query absorb.  Arguments as in those two calls
+ * (hidden [T, 3584], W_kva [576, 3584], bias [576] or NULL); T >= 0.  A new row
+ * must not share its cache slot with another row of the same call.  Errors:
+ * the union of theirs. */
+xmla_status xmla_decode_step_from_hidden(const xmla_yarn_cfg* cfg, const void* q,
+                                         const void* W_UK, const void* W_UV, const void* hidden,
+                                         const void* W_kva, const void* bias, void* pool,
+                                         int64_t num_blocks, const int32_t* block_table,
+                                         int32_t max_blocks, const int32_t* seqlens,
+                                         int32_t batch, int32_t q_len, int64_t max_seqlen,
+                                         const int32_t* seq_ids, const int64_t* positions,
+                                         int64_t T, float softmax_scale, int32_t num_splits,
+                                         void* workspace, size_t workspace_bytes,
+                                         int32_t* status_dev, void* out, void* stream,
+                                         void* attn_start, void* attn_stop);
 
 /* Size in bytes of the fixed device scratch used by xmla_decode_noalloc. */
 #define XMLA_NOALLOC_SCRATCH_BYTES (32u << 20)

@@ -15,6 +15,7 @@
 
 #include "append.cuh"
 #include "decode_chain.h"
+#include "produce.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -116,23 +117,32 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
                  qscale, tab);
 }
 
-// The first kernel of a decode step: the absorb blocks above, followed by
-// blocks that append the step's new cache rows (one thread per 16-byte piece).
-// Both halves only wait for the kernel launched before this one, so the
-// append and the absorb run side by side.
+// The first kernel of a decode step: the absorb blocks above, then the
+// producer's blocks when the step starts from hidden states (produce.cuh, 4
+// warps each; pa.T == 0 otherwise), then blocks that append the step's ready
+// cache rows (one thread per 16-byte piece).  All of them only wait for the
+// kernel launched before this one, so they run side by side.
 __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
     __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, float qscale, const RopeTable q_tab,
-    const AppendArgs ap, const RopeTable k_tab) {
+    const AppendArgs ap, const RopeTable k_tab, const ProduceArgs pa) {
   pdl_launch_dependents();
   if (blockIdx.x < kAbsorbBlocks) {
     q_absorb_block(blockIdx.x % kHeads, blockIdx.x / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
                    qscale, q_tab);
     return;
   }
+  const int prod_blocks = pa.T > 0 ? kProdBlocks : 0;
+  if (blockIdx.x < kAbsorbBlocks + prod_blocks) {
+    __shared__ ProduceSmem<kAbsorbThreads / 32> psm;
+    produce_block<kAbsorbThreads / 32>(blockIdx.x - kAbsorbBlocks, threadIdx.x, pa, k_tab, psm,
+                                       [] { __syncthreads(); }, [] { pdl_wait(); });
+    return;
+  }
   pdl_wait();
   const int64_t total = ap.T * kRowPieces;
-  const int64_t idx = (int64_t)(blockIdx.x - kAbsorbBlocks) * kAbsorbThreads + threadIdx.x;
+  const int64_t idx =
+      (int64_t)(blockIdx.x - kAbsorbBlocks - prod_blocks) * kAbsorbThreads + threadIdx.x;
   if (idx < total)
     append_piece(idx, ap.pool, ap.num_blocks, ap.block_table, ap.max_blocks, ap.batch, ap.seq_ids,
                  ap.positions, ap.c_kv, ap.k_pe, ap.status, ap.rotate, k_tab);
@@ -148,12 +158,17 @@ cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
 cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                                  const int32_t* seqlens, __nv_bfloat16* q_ext, int rows,
                                  int q_len, float qscale, const RopeTable& q_tab,
-                                 const AppendArgs& ap, const RopeTable& k_tab, cudaStream_t st) {
+                                 const AppendArgs& ap, const RopeTable& k_tab,
+                                 const ProduceArgs* pa, cudaStream_t st) {
   const int64_t append_blocks = (ap.T * kRowPieces + kAbsorbThreads - 1) / kAbsorbThreads;
   if (append_blocks > (1 << 20)) return cudaErrorInvalidValue;
-  return launch_pdl(step_prologue_kernel, dim3((unsigned)(kAbsorbBlocks + append_blocks)),
+  ProduceArgs none{};
+  const ProduceArgs& p = pa != nullptr ? *pa : none;
+  const int64_t prod_blocks = p.T > 0 ? kProdBlocks : 0;
+  return launch_pdl(step_prologue_kernel,
+                    dim3((unsigned)(kAbsorbBlocks + prod_blocks + append_blocks)),
                     dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, qscale,
-                    q_tab, ap, k_tab);
+                    q_tab, ap, k_tab, p);
 }
 
 // ---------------------------------------------------------------- combine + W_UV

@@ -15,6 +15,7 @@
 
 #include <cstdint>
 
+#include "produce.cuh"
 #include "split_kv.h"
 #include "xmla_device.cuh"
 #include "yarn.cuh"
@@ -44,11 +45,13 @@ struct AppendArgs {
   int rotate;
 };
 
-// q_absorb and the cache append of the same step in one launch.
+// q_absorb and the cache rows of the same step in one launch: ready rows are
+// appended (ap), rows from hidden states are produced (pa, nullable).
 cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                                  const int32_t* seqlens, __nv_bfloat16* q_ext, int rows,
                                  int q_len, float qscale, const RopeTable& q_tab,
-                                 const AppendArgs& ap, const RopeTable& k_tab, cudaStream_t st);
+                                 const AppendArgs& ap, const RopeTable& k_tab,
+                                 const ProduceArgs* pa, cudaStream_t st);
 
 // Merge of the splits and the W_UV product, written to out[rows, 32, 128].
 cudaError_t launch_combine(const float* part_o, const float* part_ml, const __nv_bfloat16* W_UV,

@@ -145,7 +145,7 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
                               int64_t max_seqlen, float softmax_scale, int32_t num_splits,
                               void* workspace, size_t workspace_bytes, int32_t* status_dev,
                               void* out, void* stream, void* attn_start, void* attn_stop,
-                              const AppendArgs* ap) {
+                              const AppendArgs* ap, const ProduceArgs* pa = nullptr) {
   if (q == nullptr || W_UK == nullptr || W_UV == nullptr || pool == nullptr ||
       block_table == nullptr || seqlens == nullptr || workspace == nullptr || out == nullptr)
     return XMLA_ERR_INVALID_ARG;
@@ -180,7 +180,7 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   const cudaError_t e0 =
       ap != nullptr
           ? launch_step_prologue((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
-                                 rows, q_len, qscale, tab, *ap, tab, st)
+                                 rows, q_len, qscale, tab, *ap, tab, pa, st)
           : launch_q_absorb((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
                             rows, q_len, qscale, tab, st);
   if (e0 != cudaSuccess) return XMLA_ERR_CUDA;
@@ -252,6 +252,33 @@ extern "C" xmla_status xmla_decode_step(const xmla_yarn_cfg* cfg, const void* q,
   return run_decode(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens, batch,
                     q_len, max_seqlen, softmax_scale, num_splits, workspace, workspace_bytes,
                     status_dev, out, stream, attn_start, attn_stop, &ap);
+}
+
+extern "C" xmla_status xmla_decode_step_from_hidden(
+    const xmla_yarn_cfg* cfg, const void* q, const void* W_UK, const void* W_UV,
+    const void* hidden, const void* W_kva, const void* bias, void* pool, int64_t num_blocks,
+    const int32_t* block_table, int32_t max_blocks, const int32_t* seqlens, int32_t batch,
+    int32_t q_len, int64_t max_seqlen, const int32_t* seq_ids, const int64_t* positions,
+    int64_t T, float softmax_scale, int32_t num_splits, void* workspace, size_t workspace_bytes,
+    int32_t* status_dev, void* out, void* stream, void* attn_start, void* attn_stop) {
+  if (T < 0) return XMLA_ERR_SHAPE;
+  if (T > 0 && (hidden == nullptr || W_kva == nullptr || seq_ids == nullptr || positions == nullptr))
+    return XMLA_ERR_INVALID_ARG;
+  if ((((uintptr_t)hidden) | ((uintptr_t)W_kva)) & 15u || ((uintptr_t)bias) & 1u)
+    return XMLA_ERR_INVALID_ARG;
+  AppendArgs ap{};  // no ready rows: the producer writes them
+  ap.pool = (uint4*)pool;
+  ap.num_blocks = num_blocks;
+  ap.block_table = block_table;
+  ap.max_blocks = max_blocks;
+  ap.batch = batch;
+  ap.status = status_dev;
+  const ProduceArgs pa{(const __nv_bfloat16*)hidden, (const __nv_bfloat16*)W_kva,
+                       (const __nv_bfloat16*)bias, T, (uint16_t*)pool, num_blocks, block_table,
+                       max_blocks, batch, seq_ids, positions, status_dev, 1};
+  return run_decode(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens, batch,
+                    q_len, max_seqlen, softmax_scale, num_splits, workspace, workspace_bytes,
+                    status_dev, out, stream, attn_start, attn_stop, &ap, &pa);
 }
 
 extern "C" xmla_status xmla_decode(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,

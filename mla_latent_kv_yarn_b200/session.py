@@ -152,5 +152,21 @@ class Decoder:
                               stream, ev[0], ev[1])
         return out
 
+    def step_from_hidden(self, cfg, st: LayerState, q: torch.Tensor, hidden: torch.Tensor,
+                         W_kva: torch.Tensor, new_pos: torch.Tensor, new_seq: torch.Tensor,
+                         softmax_scale: float, out=None, stream=None, events=None,
+                         bias: torch.Tensor | None = None) -> torch.Tensor:
+        """One decode step from the new tokens' hidden states: their cache rows
+        are produced (kv_a_proj_with_mqa, RoPE, append), then the layer attends."""
+        out = self.out if out is None else out
+        ev = events or (None, None)
+        xmla.xmla_decode_step_from_hidden(cfg, q, st.W_UK, st.W_UV, hidden, W_kva, bias, st.pool,
+                                          st.num_blocks, st.block_table, st.max_blocks,
+                                          st.seqlens, self.batch, self.q_len, self.max_seqlen,
+                                          new_seq, new_pos, hidden.shape[0], softmax_scale,
+                                          self.num_splits, self.workspace, self.ws_bytes,
+                                          self.status, out, stream, ev[0], ev[1])
+        return out
+
     def check_status(self) -> int:
         return int(self.status.item())

@@ -90,7 +90,8 @@ def custom(batch: int, q_len: int, seqlens, *, contiguous: bool = False, seed: i
                     seed=seed, heads=heads)
 
 
-_TENSOR_IDS = {"q": 1, "c_kv": 2, "k_pe": 3, "W_UK": 4, "W_UV": 5, "blocks": 6}
+_TENSOR_IDS = {"q": 1, "c_kv": 2, "k_pe": 3, "W_UK": 4, "W_UV": 5, "blocks": 6, "hidden": 7,
+               "W_kva": 8}
 
 
 def _gen(wl: Workload, layer: int, what: str, device) -> torch.Generator:
@@ -172,3 +173,16 @@ def new_token_rows(wl: Workload, offsets) -> list[int]:
     for s, n in enumerate(wl.seqlens):
         rows.extend(range(offsets[s] + n - wl.q_len, offsets[s] + n))
     return rows
+
+
+HIDDEN = 3584  # model hidden size: input width of kv_a_proj_with_mqa
+
+
+def producer_inputs(wl: Workload, layer: int = 0, device="cpu"):
+    """Hidden states of each sequence's q_len new tokens [B*q_len, 3584] (N(0,1))
+    and the layer's kv_a_proj_with_mqa weight [576, 3584] (N(0, 1/3584)), bf16."""
+    hidden = _normal_bf16((wl.batch * wl.q_len, HIDDEN), 1.0, _gen(wl, layer, "hidden", device),
+                          device)
+    W_kva = _normal_bf16((D_LATENT + D_ROPE, HIDDEN), HIDDEN ** -0.5,
+                         _gen(wl, layer, "W_kva", device), device)
+    return hidden, W_kva

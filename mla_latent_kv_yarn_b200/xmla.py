@@ -24,7 +24,8 @@ STATUS_NAMES = {
 # Every symbol include/xmla.h declares.
 EXPORTS = [
     "xmla_yarn_default", "xmla_yarn_inv_freq", "xmla_softmax_scale", "xmla_rope_yarn",
-    "xmla_cache_append", "xmla_decode_workspace_size", "xmla_decode_num_splits", "xmla_decode",
+    "xmla_cache_append", "xmla_kv_produce", "xmla_decode_workspace_size", "xmla_decode_num_splits",
+    "xmla_decode", "xmla_decode_step_from_hidden",
     "xmla_decode_profiled", "xmla_decode_step", "xmla_decode_noalloc",
     "xmla_selftest_wait_timeout",
     "xmla_status_string",
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.xmla_rope_yarn.restype = ctypes.c_int
         L.xmla_cache_append.argtypes = [vp, i64, vp, i32, i32, vp, vp, vp, vp, cfgp, i64, vp, vp]
         L.xmla_cache_append.restype = ctypes.c_int
+        L.xmla_kv_produce.argtypes = [vp, vp, vp, i64, cfgp, vp, i64, vp, i32, i32, vp, vp, vp, vp]
+        L.xmla_kv_produce.restype = ctypes.c_int
         L.xmla_decode_workspace_size.argtypes = [i32, i32, i64, i32, i32]
         L.xmla_decode_workspace_size.restype = sz
         L.xmla_decode_num_splits.argtypes = [i32, i32, i64, i32, i32]
@@ -85,6 +88,10 @@ def lib() -> ctypes.CDLL:
         L.xmla_decode_step.argtypes = [cfgp, vp, vp, vp, vp, i64, vp, i32, vp, i32, i32, i64, vp, vp,
                                        vp, vp, i64, f32, i32, vp, sz, vp, vp, vp, vp, vp]
         L.xmla_decode_step.restype = ctypes.c_int
+        L.xmla_decode_step_from_hidden.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, i64, vp, i32, vp,
+                                                   i32, i32, i64, vp, vp, i64, f32, i32, vp, sz,
+                                                   vp, vp, vp, vp, vp]
+        L.xmla_decode_step_from_hidden.restype = ctypes.c_int
         L.xmla_decode_noalloc.argtypes = [cfgp, vp, vp, vp, vp, i64, vp, i32, vp, i32, i32, i64, f32,
                                           i32, vp, vp, vp]
         L.xmla_decode_noalloc.restype = ctypes.c_int
@@ -152,6 +159,16 @@ def xmla_cache_append(pool: torch.Tensor, num_blocks: int, block_table: torch.Te
            "xmla_cache_append")
 
 
+def xmla_kv_produce(hidden, W_kva, bias, T, rope_cfg, pool, num_blocks, block_table, max_blocks,
+                    batch, seq_ids, positions, status=None, stream=None) -> None:
+    """kv_a_proj_with_mqa of T hidden states, RoPE of the rope key, append to the cache."""
+    cfg = None if rope_cfg is None else ctypes.byref(rope_cfg)
+    _check(lib().xmla_kv_produce(_ptr(hidden), _ptr(W_kva), _ptr(bias), int(T), cfg, _ptr(pool),
+                                 int(num_blocks), _ptr(block_table), int(max_blocks), int(batch),
+                                 _ptr(seq_ids), _ptr(positions), _ptr(status), _stream(stream)),
+           "xmla_kv_produce")
+
+
 def xmla_decode_workspace_size(batch: int, q_len: int, max_seqlen: int, num_sms: int,
                                num_splits: int = 0) -> int:
     return int(lib().xmla_decode_workspace_size(int(batch), int(q_len), int(max_seqlen),
@@ -206,6 +223,22 @@ def xmla_decode_step(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_bloc
                                   int(workspace_bytes), _ptr(status), _ptr(out), _stream(stream),
                                   ev[0], ev[1]),
            "xmla_decode_step")
+
+
+def xmla_decode_step_from_hidden(cfg, q, W_UK, W_UV, hidden, W_kva, bias, pool, num_blocks,
+                                 block_table, max_blocks, seqlens, batch, q_len, max_seqlen,
+                                 seq_ids, positions, T, softmax_scale, num_splits, workspace,
+                                 workspace_bytes, status, out, stream=None, attn_start=None,
+                                 attn_stop=None) -> None:
+    """Produce the step's T new cache rows from hidden states, then decode."""
+    ev = [None if e is None else (e.cuda_event if hasattr(e, "cuda_event") else int(e))
+          for e in (attn_start, attn_stop)]
+    _check(lib().xmla_decode_step_from_hidden(
+        ctypes.byref(cfg), _ptr(q), _ptr(W_UK), _ptr(W_UV), _ptr(hidden), _ptr(W_kva), _ptr(bias),
+        _ptr(pool), int(num_blocks), _ptr(block_table), int(max_blocks), _ptr(seqlens), int(batch),
+        int(q_len), int(max_seqlen), _ptr(seq_ids), _ptr(positions), int(T), float(softmax_scale),
+        int(num_splits), _ptr(workspace), int(workspace_bytes), _ptr(status), _ptr(out),
+        _stream(stream), ev[0], ev[1]), "xmla_decode_step_from_hidden")
 
 
 def xmla_decode_noalloc(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens,

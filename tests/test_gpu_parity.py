@@ -319,3 +319,98 @@ def test_workload_step_40l_b32_sampled_layers(layer):
     seqs = [int(np.argmax(wl.seqlens)), int(np.argmin(wl.seqlens)), 5, 17]
     gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, seqs=seqs, form="absorbed"),
                     f"step_40l_b32 layer {layer}", plain_max_abs=True)
+
+
+# ------------------------------------------------------------------ cache producer (kv_a_proj_with_mqa)
+
+def _bf16_ulp(v: np.ndarray) -> np.ndarray:
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 7.0)
+
+
+def _produce(T, seed, bias=True, rope=True):
+    cfg, ocfg = gc.cfgs()
+    g = torch.Generator().manual_seed(seed)
+    hidden = torch.randn((T, om.HIDDEN), generator=g).to(torch.bfloat16)
+    W = (torch.randn((576, om.HIDDEN), generator=g) / om.HIDDEN ** 0.5).to(torch.bfloat16)
+    b = (torch.randn(576, generator=g) * 0.5).to(torch.bfloat16) if bias else None
+    pos = torch.randperm(262144, generator=g)[:T].to(torch.int64)
+    pos[0] = 262143
+    logical = torch.unique(pos // 64)
+    bt = torch.full((1, 4096), -1, dtype=torch.int32)
+    bt[0, logical] = torch.randperm(logical.numel(), generator=g).to(torch.int32)
+    nblk = logical.numel()
+    pool = torch.zeros((nblk, 64, 576), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sid = torch.zeros(T, dtype=torch.int32)
+    xmla.xmla_kv_produce(hidden.cuda(), W.cuda(), None if b is None else b.cuda(), T,
+                         cfg if rope else None, pool, nblk, bt.cuda(), 4096, 1, sid.cuda(),
+                         pos.cuda(), status)
+    torch.cuda.synchronize()
+    rows = pool.cpu()[bt[0, pos // 64].long(), (pos % 64).long()]
+    c, k = om.kv_a_projection(gc.f64(hidden), gc.f64(W), None if b is None else gc.f64(b))
+    return int(status.item()), gc.f64(rows), c, k, pos, ocfg
+
+
+@pytest.mark.parametrize("T,bias", [(1, False), (5, True), (33, False)])
+def test_kv_produce_matches_the_projection_oracle(T, bias):
+    """The latent is the bf16 rounding of the projection (within one bf16 step of
+    the fp64 value, fp32 accumulation); the rope key is the rotation of the
+    bf16-rounded raw key (within two steps: one from the input, the rotation's
+    own rounding)."""
+    st, rows, c, k, pos, ocfg = _produce(T, 40 + T, bias)
+    assert st == 0
+    assert np.all(np.abs(rows[:, :512] - c) <= _bf16_ulp(c) * (1 + 1e-6))
+    k_bf16 = gc.f64(torch.from_numpy(k).to(torch.bfloat16))
+    want = om.rope(k_bf16, pos.numpy(), ocfg)
+    pair_mag = np.maximum(np.abs(np.concatenate([k_bf16[:, 32:], k_bf16[:, :32]], axis=1)),
+                          np.abs(k_bf16))
+    assert np.all(np.abs(rows[:, 512:] - want) <= 2 * _bf16_ulp(pair_mag) * (1 + 1e-6))
+
+
+def test_kv_produce_without_rope_stores_the_raw_key():
+    st, rows, c, k, _, _ = _produce(3, 77, bias=True, rope=False)
+    assert st == 0
+    assert np.all(np.abs(rows[:, 512:] - k) <= _bf16_ulp(k) * (1 + 1e-6))
+
+
+def test_kv_produce_reports_rows_out_of_range():
+    cfg, _ = gc.cfgs()
+    hidden = torch.ones((2, om.HIDDEN), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((576, om.HIDDEN), dtype=torch.bfloat16, device="cuda")
+    bt = torch.tensor([[0, 7]], dtype=torch.int32, device="cuda")  # block 7 outside a 1-block pool
+    pool = torch.zeros((1, 64, 576), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    xmla.xmla_kv_produce(hidden, W, None, 2, cfg, pool, 1, bt, 2, 1,
+                         torch.zeros(2, dtype=torch.int32, device="cuda"),
+                         torch.tensor([3, 70], dtype=torch.int64, device="cuda"), status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 5 and float(pool.float().abs().sum()) == 0.0
+
+
+@pytest.mark.parametrize("batch,q_len,seqlens", [(1, 1, [300]), (2, 4, [1000, 257]),
+                                                 (4, 1, [8, 16, 24, 40])])
+def test_step_from_hidden_matches_the_oracle(batch, q_len, seqlens):
+    """xmla_decode_step_from_hidden: the new tokens' cache rows come from their
+    hidden states (projection, bf16, RoPE, append), then the layer attends.  The
+    oracle builds the same rows from its own projection."""
+    wl = workloads.custom(batch, q_len, seqlens, seed=90 + sum(seqlens))
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    hidden, W_kva = workloads.producer_inputs(wl, 0, "cpu")
+    rows = torch.tensor(workloads.new_token_rows(wl, inp.offsets))
+    c, k = om.kv_a_projection(gc.f64(hidden), gc.f64(W_kva))
+    inp.c_kv[rows] = torch.from_numpy(c).to(torch.bfloat16)
+    inp.k_pe[rows] = torch.from_numpy(k).to(torch.bfloat16)
+    ref = gc.oracle_out(wl, inp, ocfg)
+
+    dev = torch.device("cuda")
+    prefix, new = session.split_prefix(wl, inp)
+    st = session.build_layer(cfg, wl, prefix, dev)
+    dec = session.Decoder(wl.batch, wl.q_len, wl.max_seqlen, dev)
+    out = dec.step_from_hidden(cfg, st, inp.q.to(dev), hidden.to(dev), W_kva.to(dev),
+                               new.positions.to(dev), new.seq_ids.to(dev),
+                               xmla.xmla_softmax_scale(cfg, 192)).clone()
+    torch.cuda.synchronize()
+    assert dec.check_status() == 0
+    gc.assert_close(out, ref, f"from hidden {batch}x{q_len} {seqlens}")
