@@ -34,6 +34,12 @@ constexpr int kAbsorbRows = 8;
 constexpr int kAbsorbThreads = 128;
 constexpr int kAbsorbBlocks = kHeads * (kDLatent / 64 + 1);
 
+// Shared memory of one absorb block: q_nope rows and the per-thread-group sums.
+struct AbsorbSmem {
+  float sq[kAbsorbRows][kDNope];
+  float part[16][kAbsorbRows][64];
+};
+
 // Block (h, cb) of the absorb; cb == 8 is the rope block.  Every block waits
 // (griddepcontrol.wait) before reading q or seqlens: a preceding kernel may
 // have written them, and the split-K kernel relies on that wait (its producer
@@ -42,9 +48,10 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
                                                const __nv_bfloat16* __restrict__ W_UK,
                                                const int32_t* seqlens,
                                                __nv_bfloat16* __restrict__ q_ext, int rows,
-                                               int q_len, float qscale, const RopeTable& tab) {
-  __shared__ float sq[kAbsorbRows][kDNope];
-  __shared__ float part[16][kAbsorbRows][64];
+                                               int q_len, float qscale, const RopeTable& tab,
+                                               AbsorbSmem& sm) {
+  auto& sq = sm.sq;
+  auto& part = sm.part;
   const int t = threadIdx.x;
   if (cb == kDLatent / 64) {
     pdl_wait();
@@ -112,9 +119,10 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
 __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
     __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, float qscale, const RopeTable tab) {
+  __shared__ AbsorbSmem sm;
   pdl_launch_dependents();
   q_absorb_block(blockIdx.x % kHeads, blockIdx.x / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
-                 qscale, tab);
+                 qscale, tab, sm);
 }
 
 // The first kernel of a decode step: the absorb blocks above, then the
@@ -126,17 +134,21 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
     __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, float qscale, const RopeTable q_tab,
     const AppendArgs ap, const RopeTable k_tab, const ProduceArgs pa) {
+  // one buffer for whichever role the block takes
+  __shared__ union {
+    AbsorbSmem absorb;
+    ProduceSmem<kAbsorbThreads / 32> produce;
+  } sm;
   pdl_launch_dependents();
   if (blockIdx.x < kAbsorbBlocks) {
     q_absorb_block(blockIdx.x % kHeads, blockIdx.x / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
-                   qscale, q_tab);
+                   qscale, q_tab, sm.absorb);
     return;
   }
   const int prod_blocks = pa.T > 0 ? kProdBlocks : 0;
   if (blockIdx.x < kAbsorbBlocks + prod_blocks) {
-    __shared__ ProduceSmem<kAbsorbThreads / 32> psm;
-    produce_block<kAbsorbThreads / 32>(blockIdx.x - kAbsorbBlocks, threadIdx.x, pa, k_tab, psm,
-                                       [] { __syncthreads(); }, [] { pdl_wait(); });
+    produce_block<kAbsorbThreads / 32>(blockIdx.x - kAbsorbBlocks, threadIdx.x, pa, k_tab,
+                                       sm.produce, [] { __syncthreads(); }, [] { pdl_wait(); });
     return;
   }
   pdl_wait();

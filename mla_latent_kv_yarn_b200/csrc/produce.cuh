@@ -78,6 +78,9 @@ __device__ __forceinline__ void produce_block(int blk, int t, const ProduceArgs&
   static_assert(kHidden % (kWarps * 8) == 0, "warps split the hidden dim in 16-byte vectors");
   constexpr int kWarpVec = kHidden / kWarps / 8;       // 16-byte vectors per warp and row
   constexpr int kLaneVec = (kWarpVec + 31) / 32;       // per lane (the last one partial)
+  // tokens whose hidden slices are loaded together: 4 when the weight slices
+  // leave room in the registers (8 warps), else 1
+  constexpr int kBatch = kLaneVec <= 2 ? 4 : 1;
   const int lane = t & 31, warp = t >> 5;
   const int v0 = warp * kWarpVec + lane;  // this lane's vectors: v0 + 32 u, u < kLaneVec
   uint4 w[kProdCols][kLaneVec];
@@ -92,36 +95,47 @@ __device__ __forceinline__ void produce_block(int blk, int t, const ProduceArgs&
 
   for (int64_t t0 = 0; t0 < a.T; t0 += kProdTok) {
     const int nt = (int)min((int64_t)kProdTok, a.T - t0);
-    for (int k = 0; k < nt; ++k) {
-      const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + (t0 + k) * kHidden);
-      uint4 h[kLaneVec];
+    // the hidden slices of kBatch tokens are requested together, then used
+    for (int k0 = 0; k0 < nt; k0 += kBatch) {
+      uint4 hb[kBatch][kLaneVec];
 #pragma unroll
-      for (int u = 0; u < kLaneVec; ++u)
-        h[u] = lane + 32 * u < kWarpVec ? hrow[v0 + 32 * u] : make_uint4(0u, 0u, 0u, 0u);
-      float acc[kProdCols];
+      for (int kk = 0; kk < kBatch; ++kk) {
+        const uint4* hrow = reinterpret_cast<const uint4*>(a.hidden + (t0 + k0 + kk) * kHidden);
 #pragma unroll
-      for (int j = 0; j < kProdCols; ++j) {
-        acc[j] = 0.f;
-#pragma unroll
-        for (int u = 0; u < kLaneVec; ++u) {
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&h[u]);
-          const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&w[j][u]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 hf = __bfloat1622float2(h2[e]);
-            const float2 wf = __bfloat1622float2(w2[e]);
-            acc[j] = fmaf(hf.x, wf.x, acc[j]);
-            acc[j] = fmaf(hf.y, wf.y, acc[j]);
-          }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+        for (int u = 0; u < kLaneVec; ++u)
+          hb[kk][u] = k0 + kk < nt && lane + 32 * u < kWarpVec ? hrow[v0 + 32 * u]
+                                                                : make_uint4(0u, 0u, 0u, 0u);
       }
-      if (lane < kProdCols) {
-        float v = acc[0];
 #pragma unroll
-        for (int i = 1; i < kProdCols; ++i) v = lane == i ? acc[i] : v;
-        sm.part[k][warp][lane] = v;
+      for (int kk = 0; kk < kBatch; ++kk) {
+        const int k = k0 + kk;
+        if (k >= nt) break;  // nt is the same for every thread of the block
+        const uint4* h = hb[kk];
+        float acc[kProdCols];
+#pragma unroll
+        for (int j = 0; j < kProdCols; ++j) {
+          acc[j] = 0.f;
+#pragma unroll
+          for (int u = 0; u < kLaneVec; ++u) {
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&h[u]);
+            const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&w[j][u]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 hf = __bfloat1622float2(h2[e]);
+              const float2 wf = __bfloat1622float2(w2[e]);
+              acc[j] = fmaf(hf.x, wf.x, acc[j]);
+              acc[j] = fmaf(hf.y, wf.y, acc[j]);
+            }
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+        }
+        if (lane < kProdCols) {
+          float v = acc[0];
+#pragma unroll
+          for (int i = 1; i < kProdCols; ++i) v = lane == i ? acc[i] : v;
+          sm.part[k][warp][lane] = v;
+        }
       }
     }
     sync();
