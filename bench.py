@@ -48,6 +48,11 @@ def parse_args():
     ap.add_argument("--impl", default="xmla", choices=["xmla", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--shards", type=int, default=0,
+                    help="sequence-parallel decode over this many page shards: with --gpus G "
+                         "(torchrun) each rank holds one shard and the partials are all-gathered "
+                         "over NCCL; on one GPU, rank 0's share is timed (its shard, the gathered "
+                         "partials' combine; the all-gather becomes a local copy)")
     ap.add_argument("--with-producer", action="store_true",
                     help="the step starts from the new tokens' hidden states: "
                          "kv_a_proj_with_mqa + RoPE + append (xmla_kv_produce), then decode")
@@ -453,12 +458,173 @@ def run_xmla(args, wl):
     return 0
 
 
+def run_shards(args, wl):
+    """Sequence-parallel decode (no append): every layer's pages are dealt out
+    over G shards; one timed step is, per layer, xmla_decode_shard on this
+    rank's pages, the all-gather of the partials, and xmla_combine_shards."""
+    import torch
+    import torch.distributed as dist
+
+    from mla_latent_kv_yarn_b200 import build, session, workloads, xmla
+    from mla_latent_kv_yarn_b200 import seq_parallel as sp
+
+    rank, world, local = dist_env()
+    G = args.shards
+    if world not in (1, G):
+        raise SystemExit(f"--shards {G} runs on one GPU (emulated rank 0) or on {G} GPUs")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    build.build()
+    cfg = xmla.xmla_yarn_default()
+    scale = xmla.xmla_softmax_scale(cfg, 192)
+    layers = []
+    for layer in range(wl.layers):
+        inp = workloads.layer_inputs(wl, layer, dev)
+        full = session.build_layer(cfg, wl, inp, dev)
+        sh = sp.ShardDecoder(wl.batch, wl.q_len, wl.max_seqlen, G, rank, dev)
+        st = sp.shard_layer(full, sh.page_lo, sh.page_hi)
+        if world == 1:
+            # the other ranks' partials, computed once: the combine reads all G
+            parts = []
+            for r in range(G):
+                o = sp.ShardDecoder(wl.batch, wl.q_len, wl.max_seqlen, G, r, dev)
+                o.decode_shard(cfg, sp.shard_layer(full, o.page_lo, o.page_hi), inp.q, scale)
+                parts.append(o.partial.clone())
+                del o
+            sh.gathered.copy_(torch.cat(parts))
+        layers.append({"st": st, "sh": sh, "q": inp.q.clone(), "W_UV": full.W_UV})
+        del inp, full
+        torch.cuda.empty_cache()
+    torch.cuda.synchronize()
+    P = layers[0]["sh"].partial_floats
+
+    def step():
+        for L in layers:
+            sh = L["sh"]
+            sh.decode_shard(cfg, L["st"], L["q"], scale)
+            if world > 1:
+                sh.gather()
+            else:
+                sh.gathered[:P].copy_(sh.partial)   # stands in for the all-gather
+            sh.combine(L["W_UV"])
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+    status = max(int(L["sh"].status.item()) for L in layers)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def flush_l2(i):
+        flush_w.fill_(i & 0xFF)
+        flush_r.sum()
+
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        flush_l2(i)
+        graph.replay()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms = []
+    for i in range(args.steps):
+        flush_l2(i + 1)
+        e0[i].record(stream)
+        graph.replay()
+        e1[i].record(stream)
+        e1[i].synchronize()
+        ms.append(e0[i].elapsed_time(e1[i]))
+    clk = clocks.stop()
+    torch.cuda.synchronize()
+    total_ms = max_over_ranks(sum(ms), dev)
+
+    # end to end: q in from pinned host memory, the output back, every step
+    h_q = [L["q"].cpu().pin_memory() for L in layers]
+    h_out = [torch.empty_like(L["sh"].out, device="cpu").pin_memory() for L in layers]
+    ee0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ee1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e2e_ms = []
+    for i in range(args.steps):
+        flush_l2(i + 7)
+        ee0[i].record(stream)
+        for L, h in zip(layers, h_q):
+            L["q"].copy_(h, non_blocking=True)
+        graph.replay()
+        for L, h in zip(layers, h_out):
+            h.copy_(L["sh"].out, non_blocking=True)
+        ee1[i].record(stream)
+        ee1[i].synchronize()
+        e2e_ms.append(ee0[i].elapsed_time(ee1[i]))
+    e2e_total = max_over_ranks(sum(e2e_ms), dev)
+
+    sh0 = layers[0]["sh"]
+    tokens_shard = sum(max(0, min(n, 64 * sh0.page_hi) - min(n, 64 * sh0.page_lo))
+                       for n in wl.seqlens)
+    # whole-job throughput: the cache of every layer, all shards together, per step
+    cache_bytes = sum(wl.seqlens) * ROW_BYTES * wl.layers
+    own_bytes = tokens_shard * ROW_BYTES * wl.layers
+    if rank == 0:
+        gbs = cache_bytes * args.steps / (total_ms * 1e-3) / 1e9
+        peak, peak_kind = measured_peaks()
+        line = {
+            "metric": METRIC, "value": round(gbs if world > 1 else
+                                             own_bytes * args.steps / (total_ms * 1e-3) / 1e9, 3),
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "strong" if world > 1 else "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": dict(workload_config(wl, world), **{
+                "seq_parallel": f"{G} page shards per sequence" + (
+                    "; one GPU: rank 0's shard timed, the all-gather replaced by a local copy "
+                    "(value = that shard's cache bytes per second)" if world == 1 else
+                    "; partials all-gathered over NCCL")}),
+            "pct_of_hbm_peak": round(100.0 * (gbs if world > 1 else own_bytes * args.steps /
+                                              (total_ms * 1e-3) / 1e9) / (peak * world), 2),
+            "e2e": {"value": round((cache_bytes if world > 1 else own_bytes) * args.steps /
+                                   (e2e_total * 1e-3) / 1e9, 3), "unit": "GB/s",
+                    "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_q),
+                    "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_out)},
+            "gpu_launches": 4 * wl.layers * args.steps,
+            "shard_pages": [sh0.page_lo, sh0.page_hi],
+            "partial_bytes_per_rank": sh0.partial_floats * 4,
+            "device_status": status,
+            "peak_source": peak_kind,
+        }
+        if clk is not None:
+            line["clocks"] = clk
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     from mla_latent_kv_yarn_b200 import workloads
     wl = workloads.workload(args.workload)
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.shards > 0:
+        return run_shards(args, wl)
     return run_xmla(args, wl)
 
 

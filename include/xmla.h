@@ -257,6 +257,59 @@ xmla_status xmla_decode_step_from_hidden(const xmla_yarn_cfg* cfg, const void* q
                                          int32_t* status_dev, void* out, void* stream,
                                          void* attn_start, void* attn_stop);
 
+/* ---- Sequence-parallel decode: one sequence's pages spread over G GPUs.
+ * ([P5] MLA section: the absorbed attention is a softmax-weighted sum of the
+ * cached latent rows, so it splits over any partition of a sequence's tokens
+ * and the parts merge exactly by their log-sum-exp.  [P1] "256K 长上下文真能
+ * 本地用：Xing4.0 原生长上下文的工程代价拆解", introduction: contexts of this
+ * size are usually run on several data-centre GPUs; [P3] "别把上下文开满：3.0
+ * Flash 256K 最稳背后的设置避坑" (another model), hardware paragraph: its
+ * longest contexts need a second GPU.)
+ *
+ * Rank g of G holds logical pages [page_lo, page_hi) of every sequence in its
+ * own pool (block_table is indexed by the logical page; entries outside the
+ * rank's range are not read).  Each rank calls xmla_decode_shard, the ranks
+ * all-gather their partials (rank order, one after another), and every rank
+ * (or one) calls xmla_combine_shards on the gathered buffer. */
+
+/* Floats of one rank's partial: batch * q_len * 32 * 514 (0 for bad sizes).
+ * Layout, with R = batch * q_len * 32 and row index (b * q_len + j) * 32 + h:
+ *   [R][512]  O, unnormalised, relative to M
+ *   [R][2]    (M, L): running maximum (log2 units, scale folded in) and sum
+ * A row that saw no token has M = -inf, L = 0, O = 0. */
+size_t xmla_shard_partial_floats(int32_t batch, int32_t q_len);
+
+/* Workspace bytes of xmla_decode_shard for a rank's page range; the split
+ * count is sized for page_hi - page_lo pages.  0 for unsupported sizes. */
+size_t xmla_decode_shard_workspace_size(int32_t batch, int32_t q_len, int64_t max_seqlen,
+                                        int64_t page_lo, int64_t page_hi, int32_t num_sms,
+                                        int32_t num_splits);
+
+/* One rank's part of a sequence-parallel decode: the query absorb, the
+ * split-K attention over the logical pages [page_lo, page_hi) of each
+ * sequence (clipped to the sequence; causal masking and the last-page
+ * handling use the global positions), and the merge of its splits into
+ * shard_partial (device, xmla_shard_partial_floats floats, 16-byte aligned,
+ * caller-owned, overwritten).  Other arguments as in xmla_decode; seqlens
+ * are the global sequence lengths.  Errors: those of xmla_decode;
+ * XMLA_ERR_SHAPE if page_lo < 0 or page_hi < page_lo. */
+xmla_status xmla_decode_shard(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
+                              const void* pool, int64_t num_blocks, const int32_t* block_table,
+                              int32_t max_blocks, const int32_t* seqlens, int32_t batch,
+                              int32_t q_len, int64_t max_seqlen, float softmax_scale,
+                              int64_t page_lo, int64_t page_hi, int32_t num_splits,
+                              void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                              float* shard_partial, void* stream);
+
+/* Merge of num_shards gathered partials (device, num_shards *
+ * xmla_shard_partial_floats floats, rank-major, 16-byte aligned) and the
+ * W_UV product: out[b, j, h, :] (bf16, [batch, q_len, 32, 128]) as
+ * xmla_decode writes it.  Errors: XMLA_ERR_INVALID_ARG (null or misaligned),
+ * XMLA_ERR_SHAPE (sizes, num_shards outside [1, 1024]), XMLA_ERR_UNSUPPORTED,
+ * XMLA_ERR_CUDA. */
+xmla_status xmla_combine_shards(const float* partials, int32_t num_shards, const void* W_UV,
+                                int32_t batch, int32_t q_len, void* out, void* stream);
+
 /* Size in bytes of the fixed device scratch used by xmla_decode_noalloc. */
 #define XMLA_NOALLOC_SCRATCH_BYTES (32u << 20)
 

@@ -227,10 +227,75 @@ __device__ __forceinline__ void fma4(float4& acc, float w, const float4& x) {
   acc.w = fmaf(w, x.w, acc.w);
 }
 
+// The merge of one group's splits (sub, sub + gpr, ...) of a row, for the
+// float4 q4 of a 64-dim slice: the first kCombineDepth split rows are loaded
+// together and merged against the group's maximum over its first 16 splits
+// (lane k of the 16-lane group loads (m, l) of the group's k-th split); later
+// splits are loaded one by one and merged online.  Splits with l = 0 (no
+// token) are skipped.  po / pml: the row's O slice and (m, l) of split 0;
+// splits are o_stride floats and ml_stride (m, l) pairs apart.
+__device__ __forceinline__ void merge_group(const float* po, const float2* pml, int64_t o_stride,
+                                            int64_t ml_stride, int nsplit, int sub, int gpr, int q4,
+                                            bool active, float& m_g, float& l_g, float4& acc) {
+  float4 v[kCombineDepth];
+#pragma unroll
+  for (int k = 0; k < kCombineDepth; ++k) {
+    const int s = sub + gpr * k;
+    v[k] = active && s < nsplit ? *reinterpret_cast<const float4*>(po + s * o_stride)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const int s_lane = sub + gpr * q4;  // the split whose (m, l) this lane loads
+  const float2 ml = active && s_lane < nsplit ? pml[(int64_t)s_lane * ml_stride]
+                                              : make_float2(-INFINITY, 0.f);
+
+  // group maximum over its first 16 splits (lanes of one group: 16 consecutive)
+  m_g = ml.y > 0.f ? ml.x : -INFINITY;
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) m_g = fmaxf(m_g, __shfl_xor_sync(0xffffffffu, m_g, o));
+  l_g = 0.f;
+  acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < kCombineDepth; ++k) {
+    const float mk = __shfl_sync(0xffffffffu, ml.x, k, 16);
+    const float lk = __shfl_sync(0xffffffffu, ml.y, k, 16);
+    if (lk > 0.f) {  // also false past the group's last split
+      const float w = ex2(mk - m_g);
+      l_g = fmaf(w, lk, l_g);
+      fma4(acc, w, v[k]);
+    }
+  }
+  // splits past the first kCombineDepth of the group (many splits per group only):
+  // loaded one by one, merged online
+  if (active) {
+    for (int s = sub + gpr * kCombineDepth; s < nsplit; s += gpr) {
+      const float2 x = pml[(int64_t)s * ml_stride];
+      if (x.y > 0.f) {
+        if (x.x > m_g) {
+          const float c = m_g == -INFINITY ? 0.f : ex2(m_g - x.x);
+          l_g *= c;
+          acc.x *= c;
+          acc.y *= c;
+          acc.z *= c;
+          acc.w *= c;
+          m_g = x.x;
+        }
+        const float w = ex2(x.x - m_g);
+        l_g = fmaf(w, x.y, l_g);
+        fma4(acc, w, *reinterpret_cast<const float4*>(po + s * o_stride));
+      }
+    }
+  }
+}
+
+// kStrided: splits are o_stride floats / ml_stride (m, l) pairs apart (the
+// gathered partials of a sequence-parallel decode); otherwise rows_per_cta
+// rows apart, as the split-K kernel writes them.
+template <bool kStrided>
 __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThreads, 3)
     combine_uv_kernel(const float* part_o, const float* part_ml,
                       const __nv_bfloat16* __restrict__ W_UV, __nv_bfloat16* __restrict__ out,
-                      int rows, int q_len, int groups, int nsplit, int rows_per_cta) {
+                      int rows, int q_len, int groups, int nsplit, int rows_per_cta,
+                      int64_t o_stride_arg, int64_t ml_stride_arg) {
   // part_o and part_ml are written by the kernel launched just before this one,
   // which lets this grid start early: they carry no __restrict__, so their loads
   // are not taken as invariant and stay behind the griddepcontrol.wait below.
@@ -277,58 +342,14 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThread
   }
   const float* po = part_o + base * kDLatent + slice * kSliceDims + 4 * q4;
   const float2* pml = reinterpret_cast<const float2*>(part_ml) + base;
-  const int o_stride = rows_per_cta * kDLatent;  // floats between splits (nsplit * o_stride < 2^31)
+  const int64_t o_stride = kStrided ? o_stride_arg : rows_per_cta * kDLatent;
+  const int64_t ml_stride = kStrided ? ml_stride_arg : rows_per_cta;
 
   pdl_wait();  // the split partials come from the decode kernel
 
-  float4 v[kCombineDepth];
-#pragma unroll
-  for (int k = 0; k < kCombineDepth; ++k) {
-    const int s = sub + gpr * k;
-    v[k] = active && s < nsplit ? *reinterpret_cast<const float4*>(po + s * o_stride)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  const int s_lane = sub + gpr * q4;  // the split whose (m, l) this lane loads
-  const float2 ml = active && s_lane < nsplit ? pml[(int64_t)s_lane * rows_per_cta]
-                                              : make_float2(-INFINITY, 0.f);
-
-  // group maximum over its first 16 splits (lanes of one group: 16 consecutive)
-  float m_g = ml.y > 0.f ? ml.x : -INFINITY;
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) m_g = fmaxf(m_g, __shfl_xor_sync(0xffffffffu, m_g, o));
-  float l_g = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int k = 0; k < kCombineDepth; ++k) {
-    const float mk = __shfl_sync(0xffffffffu, ml.x, k, 16);
-    const float lk = __shfl_sync(0xffffffffu, ml.y, k, 16);
-    if (lk > 0.f) {  // also false past the group's last split
-      const float w = ex2(mk - m_g);
-      l_g = fmaf(w, lk, l_g);
-      fma4(acc, w, v[k]);
-    }
-  }
-  // splits past the first kCombineDepth of the group (many splits per group only):
-  // loaded one by one, merged online
-  if (active) {
-    for (int s = sub + gpr * kCombineDepth; s < nsplit; s += gpr) {
-      const float2 x = pml[(int64_t)s * rows_per_cta];
-      if (x.y > 0.f) {
-        if (x.x > m_g) {
-          const float c = m_g == -INFINITY ? 0.f : ex2(m_g - x.x);
-          l_g *= c;
-          acc.x *= c;
-          acc.y *= c;
-          acc.z *= c;
-          acc.w *= c;
-          m_g = x.x;
-        }
-        const float w = ex2(x.x - m_g);
-        l_g = fmaf(w, x.y, l_g);
-        fma4(acc, w, *reinterpret_cast<const float4*>(po + s * o_stride));
-      }
-    }
-  }
+  float m_g, l_g;
+  float4 acc;
+  merge_group(po, pml, o_stride, ml_stride, nsplit, sub, gpr, q4, active, m_g, l_g, acc);
   acc_s[grp][q4] = acc;
   if (q4 == 0) {
     grp_m[grp] = m_g;
@@ -395,10 +416,97 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThread
 
 cudaError_t launch_combine(const float* part_o, const float* part_ml, const __nv_bfloat16* W_UV,
                            __nv_bfloat16* out, int rows, int q_len, int groups, int nsplit,
-                           int rows_per_cta, cudaStream_t st) {
+                           int rows_per_cta, cudaStream_t st, int64_t o_stride,
+                           int64_t ml_stride) {
   const int chunks = (rows + kCombineRows - 1) / kCombineRows;
-  return launch_pdl(combine_uv_kernel, dim3(kSlices * kHeads * chunks), dim3(kCombineThreads), 0,
-                    st, part_o, part_ml, W_UV, out, rows, q_len, groups, nsplit, rows_per_cta);
+  const dim3 grid(kSlices * kHeads * chunks);
+  if (o_stride == 0 && ml_stride == 0)
+    return launch_pdl(combine_uv_kernel<false>, grid, dim3(kCombineThreads), 0, st, part_o,
+                      part_ml, W_UV, out, rows, q_len, groups, nsplit, rows_per_cta, (int64_t)0,
+                      (int64_t)0);
+  return launch_pdl(combine_uv_kernel<true>, grid, dim3(kCombineThreads), 0, st, part_o, part_ml,
+                    W_UV, out, rows, q_len, groups, nsplit, rows_per_cta, o_stride, ml_stride);
+}
+
+// ---------------------------------------------------------------- merge of one shard's splits
+
+// One rank's share of a sequence-parallel decode: its splits are merged into
+// one partial per (query row, head) -- the running maximum M, the sum L and
+// the unnormalised O, all relative to M -- laid out as
+//   out[(r * 32 + h) * 512 + d]             O,  r = b * q_len + j
+//   out[R * 512 + (r * 32 + h) * 2 + {0,1}] M, L  (R = rows * 32)
+// so that the partials of G ranks, gathered one after another, are G splits
+// of the combine above (split stride R * 514 floats).  Blocks as in the
+// combine: (64-dim slice, head, chunk of up to 16 rows), 256 threads.
+__global__ void __launch_bounds__(kCombineThreads)
+    merge_splits_kernel(const float* part_o, const float* part_ml, float* __restrict__ out,
+                        int rows, int q_len, int groups, int nsplit, int rows_per_cta) {
+  __shared__ __align__(16) float4 acc_s[kCombineGroups][kSliceDims / 4];
+  __shared__ float grp_m[kCombineGroups], grp_l[kCombineGroups];
+  const int slice = blockIdx.x % kSlices;
+  const int cid = blockIdx.x / kSlices;
+  const int h = cid % kHeads;
+  const int chunk = cid / kHeads;
+  const int r0 = chunk * kCombineRows;
+  const int nr = min(kCombineRows, rows - r0);
+  const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  const int q4 = tid & 15;
+  const int grp = tid >> 4;
+  const int gpr = max(1, kCombineGroups / nr);
+  const int my_rr = grp / gpr;
+  const int sub = grp % gpr;
+  const bool active = my_rr < nr;
+  int64_t base = 0;
+  if (active) {
+    const int r = r0 + my_rr;
+    const int b = r / q_len, j = r % q_len;
+    const int ridx = j * kHeads + h;
+    base = ((int64_t)b * groups + ridx / rows_per_cta) * nsplit * rows_per_cta + ridx % rows_per_cta;
+  }
+  const float* po = part_o + base * kDLatent + slice * kSliceDims + 4 * q4;
+  const float2* pml = reinterpret_cast<const float2*>(part_ml) + base;
+  pdl_wait();  // the split partials come from the decode kernel
+  float m_g, l_g;
+  float4 acc;
+  merge_group(po, pml, (int64_t)rows_per_cta * kDLatent, rows_per_cta, nsplit, sub, gpr, q4,
+              active, m_g, l_g, acc);
+  acc_s[grp][q4] = acc;
+  if (q4 == 0) {
+    grp_m[grp] = m_g;
+    grp_l[grp] = l_g;
+  }
+  __syncthreads();
+  const int64_t R = (int64_t)rows * kHeads;
+  for (int e = tid; e < nr * kSliceDims; e += kCombineThreads) {
+    const int rr = e / kSliceDims, d = e % kSliceDims;
+    const int g0 = rr * gpr;
+    float M = -INFINITY;
+    for (int g = 0; g < gpr; ++g)
+      if (grp_l[g0 + g] > 0.f) M = fmaxf(M, grp_m[g0 + g]);
+    float L = 0.f, t = 0.f;
+    for (int g = 0; g < gpr; ++g) {
+      if (grp_l[g0 + g] > 0.f) {
+        const float w = ex2(grp_m[g0 + g] - M);
+        L = fmaf(w, grp_l[g0 + g], L);
+        t = fmaf(w, reinterpret_cast<const float*>(&acc_s[g0 + g][0])[d], t);
+      }
+    }
+    const int64_t row = (int64_t)(r0 + rr) * kHeads + h;
+    out[row * kDLatent + slice * kSliceDims + d] = t;
+    if (slice == 0 && d == 0) {
+      out[R * kDLatent + 2 * row] = M;
+      out[R * kDLatent + 2 * row + 1] = L;
+    }
+  }
+}
+
+cudaError_t launch_merge_splits(const float* part_o, const float* part_ml, float* out, int rows,
+                                int q_len, int groups, int nsplit, int rows_per_cta,
+                                cudaStream_t st) {
+  const int chunks = (rows + kCombineRows - 1) / kCombineRows;
+  return launch_pdl(merge_splits_kernel, dim3(kSlices * kHeads * chunks), dim3(kCombineThreads), 0,
+                    st, part_o, part_ml, out, rows, q_len, groups, nsplit, rows_per_cta);
 }
 
 }  // namespace xmla

@@ -54,8 +54,17 @@ cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_
                                  const ProduceArgs* pa, cudaStream_t st);
 
 // Merge of the splits and the W_UV product, written to out[rows, 32, 128].
+// Split s of a row is o_stride floats (O) and ml_stride (m, l) pairs after
+// split 0; 0 means the split-K kernel's layout (rows_per_cta rows apart).
 cudaError_t launch_combine(const float* part_o, const float* part_ml, const __nv_bfloat16* W_UV,
                            __nv_bfloat16* out, int rows, int q_len, int groups, int nsplit,
-                           int rows_per_cta, cudaStream_t st);
+                           int rows_per_cta, cudaStream_t st, int64_t o_stride = 0,
+                           int64_t ml_stride = 0);
+
+// Merge of the splits into one partial per (row, head) -- (M, L, unnormalised
+// O) -- for a sequence-parallel decode; layout in absorb_combine.cu.
+cudaError_t launch_merge_splits(const float* part_o, const float* part_ml, float* out, int rows,
+                                int q_len, int groups, int nsplit, int rows_per_cta,
+                                cudaStream_t st);
 
 }  // namespace xmla

@@ -126,7 +126,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int NR>
+// kRanged: the call covers the logical pages [p.page_lo, p.page_hi) of every
+// sequence (one rank's share of a sequence-parallel decode); otherwise all.
+template <int NR, bool kRanged>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tmap_pool,
                       const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p) {
@@ -162,9 +164,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     seqlen = 0;
   }
   const int64_t npages = (seqlen + kPage - 1) / kPage;
-  const int64_t pps = (npages + p.nsplit - 1) / p.nsplit;
-  const int64_t p_begin = (int64_t)split * pps;
-  const int64_t p_end = min(npages, p_begin + pps);
+  const int64_t p_lo = kRanged ? min(p.page_lo, npages) : 0;
+  const int64_t p_hi = kRanged ? min(p.page_hi, npages) : npages;
+  const int64_t pps = (p_hi - p_lo + p.nsplit - 1) / p.nsplit;
+  const int64_t p_begin = p_lo + (int64_t)split * pps;
+  const int64_t p_end = min(p_hi, p_begin + pps);
   const int n_pages = (int)max((int64_t)0, p_end - p_begin);
 
   // ---- setup (independent of the previous kernel's results)
@@ -573,7 +577,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
 }
 
-template <int NR>
+template <int NR, bool kRanged>
 static cudaError_t launch_decode(const CUtensorMap& tp, const CUtensorMap& tq, const DecodeParams& dp,
                                  int64_t items, cudaStream_t st) {
   using L = DecodeLayout<NR>;
@@ -582,20 +586,23 @@ static cudaError_t launch_decode(const CUtensorMap& tp, const CUtensorMap& tq, c
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<NR>,
+    cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<NR, kRanged>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  return launch_pdl(mla_decode_kernel<NR>, dim3((unsigned)items), dim3(kDecodeThreads), L::kSmem,
+  return launch_pdl(mla_decode_kernel<NR, kRanged>, dim3((unsigned)items), dim3(kDecodeThreads), L::kSmem,
                     st, tp, tq, dp);
 }
 
 
 cudaError_t launch_split_kv(int nr, const CUtensorMap& pool_map, const CUtensorMap& q_map,
                             const DecodeParams& dp, int64_t items, cudaStream_t st) {
-  if (nr == 32) return launch_decode<32>(pool_map, q_map, dp, items, st);
-  if (nr == 64) return launch_decode<64>(pool_map, q_map, dp, items, st);
+  const bool ranged = dp.page_lo != 0 || dp.page_hi != INT64_MAX;
+  if (nr == 32) return ranged ? launch_decode<32, true>(pool_map, q_map, dp, items, st)
+                              : launch_decode<32, false>(pool_map, q_map, dp, items, st);
+  if (nr == 64) return ranged ? launch_decode<64, true>(pool_map, q_map, dp, items, st)
+                              : launch_decode<64, false>(pool_map, q_map, dp, items, st);
   return cudaErrorInvalidValue;
 }
 

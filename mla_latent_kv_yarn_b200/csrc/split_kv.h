@@ -28,6 +28,11 @@ struct DecodeParams {
   int32_t q_len;
   int32_t groups;
   int32_t nsplit;
+  // logical pages of every sequence this call attends over: [page_lo, page_hi)
+  // clipped to the sequence (0 and INT64_MAX for the whole sequence); the
+  // splits partition that range
+  int64_t page_lo;
+  int64_t page_hi;
 };
 
 // Split-K attention over `items` work items; nr = rows per CTA (32 or 64).

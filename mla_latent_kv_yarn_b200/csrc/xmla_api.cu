@@ -40,15 +40,18 @@ struct Plan {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// span_pages: logical pages a call attends over at most (the split count is
+// sized for them); 0 = all pages of max_seqlen.
 static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_sms,
-                      int32_t num_splits, Plan* pl) {
+                      int32_t num_splits, Plan* pl, int64_t span_pages = 0) {
   if (B < 1 || q_len < 1 || q_len > kMaxQLen || max_seqlen < q_len ||
-      max_seqlen > (int64_t)0x7fffffff - kPage || num_sms < 1 || num_splits < 0)
+      max_seqlen > (int64_t)0x7fffffff - kPage || num_sms < 1 || num_splits < 0 || span_pages < 0)
     return false;
   Plan P;
   P.nr = q_len == 1 ? 32 : 64;
   P.groups = (q_len * 32 + P.nr - 1) / P.nr;
-  const int64_t max_pages = (max_seqlen + kPage - 1) / kPage;
+  int64_t max_pages = (max_seqlen + kPage - 1) / kPage;
+  if (span_pages > 0 && span_pages < max_pages) max_pages = span_pages;
   int64_t ns;
   if (num_splits > 0) {
     ns = num_splits;
@@ -145,7 +148,9 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
                               int64_t max_seqlen, float softmax_scale, int32_t num_splits,
                               void* workspace, size_t workspace_bytes, int32_t* status_dev,
                               void* out, void* stream, void* attn_start, void* attn_stop,
-                              const AppendArgs* ap, const ProduceArgs* pa = nullptr) {
+                              const AppendArgs* ap, const ProduceArgs* pa = nullptr,
+                              int64_t page_lo = 0, int64_t page_hi = INT64_MAX,
+                              float* shard_partial = nullptr) {
   if (q == nullptr || W_UK == nullptr || W_UV == nullptr || pool == nullptr ||
       block_table == nullptr || seqlens == nullptr || workspace == nullptr || out == nullptr)
     return XMLA_ERR_INVALID_ARG;
@@ -155,13 +160,15 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   if ((((uintptr_t)pool) & 15u) || (((uintptr_t)workspace) & 255u) || (((uintptr_t)q) & 15u) ||
       (((uintptr_t)W_UK) & 15u) || (((uintptr_t)W_UV) & 15u) || (((uintptr_t)out) & 15u))
     return XMLA_ERR_INVALID_ARG;
+  if (page_lo < 0 || page_hi < page_lo) return XMLA_ERR_SHAPE;
   if (num_blocks < 1 || num_blocks * kPage >= 0x7fffffffLL || max_blocks < 1 ||
       (int64_t)max_blocks * kPage < max_seqlen)
     return XMLA_ERR_SHAPE;
   int nsm = 0;
   if (!device_ok(&nsm)) return XMLA_ERR_UNSUPPORTED;
   Plan P;
-  if (!make_plan(batch, q_len, max_seqlen, nsm, num_splits, &P)) return XMLA_ERR_SHAPE;
+  const int64_t span = page_hi == INT64_MAX ? 0 : (page_hi > page_lo ? page_hi - page_lo : 1);
+  if (!make_plan(batch, q_len, max_seqlen, nsm, num_splits, &P, span)) return XMLA_ERR_SHAPE;
   if (workspace_bytes < P.bytes) return XMLA_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
   uint8_t* ws = (uint8_t*)workspace;
@@ -199,9 +206,16 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   dp.q_len = q_len;
   dp.groups = P.groups;
   dp.nsplit = P.nsplit;
+  dp.page_lo = page_lo;
+  dp.page_hi = page_hi;
   if (record_event(attn_start, st) != cudaSuccess) return XMLA_ERR_CUDA;
   if (launch_split_kv(P.nr, tmap_pool, tmap_q, dp, P.items, st) != cudaSuccess) return XMLA_ERR_CUDA;
   if (record_event(attn_stop, st) != cudaSuccess) return XMLA_ERR_CUDA;
+  if (shard_partial != nullptr) {
+    const cudaError_t em = launch_merge_splits(dp.part_o, dp.part_ml, shard_partial, rows, q_len,
+                                               P.groups, P.nsplit, P.nr, st);
+    return em == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+  }
   const cudaError_t e = launch_combine(dp.part_o, dp.part_ml, (const __nv_bfloat16*)W_UV,
                                        (__nv_bfloat16*)out, rows, q_len, P.groups, P.nsplit, P.nr,
                                        st);
@@ -291,6 +305,62 @@ extern "C" xmla_status xmla_decode(const xmla_yarn_cfg* cfg, const void* q, cons
   return xmla_decode_profiled(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_blocks, seqlens,
                               batch, q_len, max_seqlen, softmax_scale, num_splits, workspace,
                               workspace_bytes, status_dev, out, stream, nullptr, nullptr);
+}
+
+// ---------------------------------------------------------------- sequence-parallel decode
+
+extern "C" size_t xmla_shard_partial_floats(int32_t batch, int32_t q_len) {
+  if (batch < 1 || q_len < 1 || q_len > kMaxQLen) return 0;
+  return (size_t)batch * q_len * kHeads * (kDLatent + 2);
+}
+
+extern "C" size_t xmla_decode_shard_workspace_size(int32_t batch, int32_t q_len,
+                                                   int64_t max_seqlen, int64_t page_lo,
+                                                   int64_t page_hi, int32_t num_sms,
+                                                   int32_t num_splits) {
+  if (page_lo < 0 || page_hi < page_lo) return 0;
+  Plan P;
+  const int64_t span = page_hi > page_lo ? page_hi - page_lo : 1;
+  return make_plan(batch, q_len, max_seqlen, num_sms, num_splits, &P, span) ? P.bytes : 0;
+}
+
+extern "C" xmla_status xmla_decode_shard(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
+                                         const void* pool, int64_t num_blocks,
+                                         const int32_t* block_table, int32_t max_blocks,
+                                         const int32_t* seqlens, int32_t batch, int32_t q_len,
+                                         int64_t max_seqlen, float softmax_scale, int64_t page_lo,
+                                         int64_t page_hi, int32_t num_splits, void* workspace,
+                                         size_t workspace_bytes, int32_t* status_dev,
+                                         float* shard_partial, void* stream) {
+  if (shard_partial == nullptr) return XMLA_ERR_INVALID_ARG;
+  if (((uintptr_t)shard_partial) & 15u) return XMLA_ERR_INVALID_ARG;
+  if (page_lo < 0 || page_hi < page_lo) return XMLA_ERR_SHAPE;
+  // W_UV and out are not used: the shard ends with its merged partial
+  return run_decode(cfg, q, W_UK, W_UK, pool, num_blocks, block_table, max_blocks, seqlens, batch,
+                    q_len, max_seqlen, softmax_scale, num_splits, workspace, workspace_bytes,
+                    status_dev, shard_partial, stream, nullptr, nullptr, nullptr, nullptr,
+                    page_lo, page_hi, shard_partial);
+}
+
+extern "C" xmla_status xmla_combine_shards(const float* partials, int32_t num_shards,
+                                           const void* W_UV, int32_t batch, int32_t q_len,
+                                           void* out, void* stream) {
+  if (partials == nullptr || W_UV == nullptr || out == nullptr) return XMLA_ERR_INVALID_ARG;
+  if (batch < 1 || q_len < 1 || q_len > kMaxQLen || num_shards < 1 || num_shards > kMaxSplits)
+    return XMLA_ERR_SHAPE;
+  if ((((uintptr_t)partials) | ((uintptr_t)W_UV) | ((uintptr_t)out)) & 15u)
+    return XMLA_ERR_INVALID_ARG;
+  int nsm = 0;
+  if (!device_ok(&nsm)) return XMLA_ERR_UNSUPPORTED;
+  const int rows = batch * q_len;
+  const int64_t R = (int64_t)rows * kHeads;
+  // the gathered partials, read as num_shards splits of one row group holding
+  // every (row, head): row r*32 + h of a shard is at r*32 + h
+  const cudaError_t e = launch_combine(partials, partials + R * kDLatent,
+                                       (const __nv_bfloat16*)W_UV, (__nv_bfloat16*)out, rows, rows,
+                                       1, num_shards, (int)R, (cudaStream_t)stream,
+                                       R * (kDLatent + 2), R * (kDLatent + 2) / 2);
+  return e == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- decode without caller scratch

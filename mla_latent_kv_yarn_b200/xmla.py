@@ -27,6 +27,8 @@ EXPORTS = [
     "xmla_cache_append", "xmla_kv_produce", "xmla_decode_workspace_size", "xmla_decode_num_splits",
     "xmla_decode", "xmla_decode_step_from_hidden",
     "xmla_decode_profiled", "xmla_decode_step", "xmla_decode_noalloc",
+    "xmla_shard_partial_floats", "xmla_decode_shard_workspace_size", "xmla_decode_shard",
+    "xmla_combine_shards",
     "xmla_selftest_wait_timeout",
     "xmla_status_string",
 ]
@@ -95,6 +97,15 @@ def lib() -> ctypes.CDLL:
         L.xmla_decode_noalloc.argtypes = [cfgp, vp, vp, vp, vp, i64, vp, i32, vp, i32, i32, i64, f32,
                                           i32, vp, vp, vp]
         L.xmla_decode_noalloc.restype = ctypes.c_int
+        L.xmla_shard_partial_floats.argtypes = [i32, i32]
+        L.xmla_shard_partial_floats.restype = sz
+        L.xmla_decode_shard_workspace_size.argtypes = [i32, i32, i64, i64, i64, i32, i32]
+        L.xmla_decode_shard_workspace_size.restype = sz
+        L.xmla_decode_shard.argtypes = [cfgp, vp, vp, vp, i64, vp, i32, vp, i32, i32, i64, f32, i64,
+                                        i64, i32, vp, sz, vp, vp, vp]
+        L.xmla_decode_shard.restype = ctypes.c_int
+        L.xmla_combine_shards.argtypes = [vp, i32, vp, i32, i32, vp, vp]
+        L.xmla_combine_shards.restype = ctypes.c_int
         L.xmla_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
         L.xmla_selftest_wait_timeout.restype = ctypes.c_int
         L.xmla_status_string.argtypes = [ctypes.c_int]
@@ -252,6 +263,38 @@ def xmla_decode_noalloc(cfg, q, W_UK, W_UV, pool, num_blocks, block_table, max_b
                                      float(softmax_scale), int(num_splits), _ptr(status), _ptr(out),
                                      _stream(stream)),
            "xmla_decode_noalloc")
+
+
+def xmla_shard_partial_floats(batch: int, q_len: int) -> int:
+    return int(lib().xmla_shard_partial_floats(int(batch), int(q_len)))
+
+
+def xmla_decode_shard_workspace_size(batch: int, q_len: int, max_seqlen: int, page_lo: int,
+                                     page_hi: int, num_sms: int, num_splits: int = 0) -> int:
+    return int(lib().xmla_decode_shard_workspace_size(int(batch), int(q_len), int(max_seqlen),
+                                                      int(page_lo), int(page_hi), int(num_sms),
+                                                      int(num_splits)))
+
+
+def xmla_decode_shard(cfg, q, W_UK, pool, num_blocks, block_table, max_blocks, seqlens, batch,
+                      q_len, max_seqlen, softmax_scale, page_lo, page_hi, num_splits, workspace,
+                      workspace_bytes, status, shard_partial, stream=None) -> None:
+    """One rank's part of a sequence-parallel decode over logical pages
+    [page_lo, page_hi): its merged partial goes to shard_partial (fp32)."""
+    _check(lib().xmla_decode_shard(ctypes.byref(cfg), _ptr(q), _ptr(W_UK), _ptr(pool),
+                                   int(num_blocks), _ptr(block_table), int(max_blocks),
+                                   _ptr(seqlens), int(batch), int(q_len), int(max_seqlen),
+                                   float(softmax_scale), int(page_lo), int(page_hi),
+                                   int(num_splits), _ptr(workspace), int(workspace_bytes),
+                                   _ptr(status), _ptr(shard_partial), _stream(stream)),
+           "xmla_decode_shard")
+
+
+def xmla_combine_shards(partials, num_shards, W_UV, batch, q_len, out, stream=None) -> None:
+    """Merge of gathered shard partials (rank-major) and the W_UV product."""
+    _check(lib().xmla_combine_shards(_ptr(partials), int(num_shards), _ptr(W_UV), int(batch),
+                                     int(q_len), _ptr(out), _stream(stream)),
+           "xmla_combine_shards")
 
 
 def xmla_selftest_wait_timeout(status: torch.Tensor, timeout_ns: int, stream=None) -> None:

@@ -262,6 +262,65 @@ def mla_attention_absorbed(q: np.ndarray, c_kv: np.ndarray, k_pe_rot: np.ndarray
     return np.einsum("jhc,hcv->jhv", o_lat, W_UV)
 
 
+def attention_partial(q: np.ndarray, c_kv: np.ndarray, k_pe_rot: np.ndarray,
+                      W_UK: np.ndarray, cfg: YarnConfig, seqlen: int, t_lo: int,
+                      t_hi: int) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """The absorbed attention of one sequence over its cached tokens [t_lo, t_hi) only.
+
+    [P5] MLA section: the output is a softmax-weighted sum over the cached
+    latent rows; restricted to a subset of tokens it is described exactly by
+    (m, l, O): m the largest visible score of the subset, l = sum exp(S - m),
+    O = sum exp(S - m) c_kv[t] (natural-log units, scores S as in
+    mla_attention_absorbed).  q: [q_len, H, 192] (q_pe not rotated); c_kv,
+    k_pe_rot: rows [t_lo, t_hi) of the sequence ([t_hi - t_lo, 512] / [.., 64]);
+    seqlen: the sequence's full length (query j at seqlen - q_len + j).
+    Rows that see no token of the subset get m = -inf, l = 0, O = 0.
+    Returns m [q_len, H], l [q_len, H], O [q_len, H, 512].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    c_kv = np.asarray(c_kv, dtype=np.float64)
+    k_pe_rot = np.asarray(k_pe_rot, dtype=np.float64)
+    W_UK = np.asarray(W_UK, dtype=np.float64)
+    q_len, H, _ = q.shape
+    scale = softmax_scale(cfg, q.shape[-1])
+    qpos = _query_positions(seqlen, q_len)
+    q_rot = rope(q[..., D_NOPE:], qpos[:, None], cfg)
+    q_lat = np.einsum("jhd,hdc->jhc", q[..., :D_NOPE], W_UK)
+    S = scale * (q_lat.reshape(q_len * H, -1) @ c_kv.T
+                 + q_rot.reshape(q_len * H, -1) @ k_pe_rot.T)        # [q_len*H, n]
+    tpos = np.arange(t_lo, t_hi)
+    visible = np.repeat(tpos[None, :] <= qpos[:, None], H, axis=0)
+    S = np.where(visible, S, -np.inf)
+    m = S.max(axis=1) if S.shape[1] > 0 else np.full(q_len * H, -np.inf)
+    E = np.where(visible, np.exp(S - np.where(np.isfinite(m), m, 0.0)[:, None]), 0.0)
+    l = E.sum(axis=1)
+    O = E @ c_kv
+    return m.reshape(q_len, H), l.reshape(q_len, H), O.reshape(q_len, H, -1)
+
+
+def merge_partials(parts) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Exact merge of partials (m, l, O) of disjoint token subsets of one sequence.
+
+    With M = max m_i over parts that saw a token: l = sum exp(m_i - M) l_i and
+    O = sum exp(m_i - M) O_i (the log-sum-exp combination of softmax sums).
+    """
+    parts = list(parts)
+    ms = np.stack([np.asarray(p[0], dtype=np.float64) for p in parts])
+    ls = np.stack([np.asarray(p[1], dtype=np.float64) for p in parts])
+    Os = np.stack([np.asarray(p[2], dtype=np.float64) for p in parts])
+    seen = ls > 0
+    M = np.where(seen, ms, -np.inf).max(axis=0)
+    w = np.where(seen, np.exp(np.where(seen, ms, 0.0) - np.where(np.isfinite(M), M, 0.0)), 0.0)
+    return M, (w * ls).sum(axis=0), (w[..., None] * Os).sum(axis=0)
+
+
+def finish_partial(m: np.ndarray, l: np.ndarray, O: np.ndarray, W_UV: np.ndarray) -> np.ndarray:
+    """Output of a complete partial: out[j, h] = W_UV[h]^T (O[j, h] / l[j, h]).
+    Returns [q_len, H, 128]; rows with l = 0 give 0."""
+    o_lat = np.where(l[..., None] > 0, O / np.where(l > 0, l, 1.0)[..., None], 0.0)
+    return np.einsum("jhc,hcv->jhv", o_lat, np.asarray(W_UV, dtype=np.float64))
+
+
 HIDDEN = 3584  # model hidden size (the summary page's architecture paragraph)
 
 

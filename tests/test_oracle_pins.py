@@ -402,3 +402,81 @@ def test_kv_projection_is_linear_in_the_hidden_state():
     c3, k3 = om.kv_a_projection(2.5 * h1 - h2, W)
     assert np.allclose(c3, 2.5 * c1 - c2, rtol=0, atol=1e-10)
     assert np.allclose(k3, 2.5 * k1 - k2, rtol=0, atol=1e-10)
+
+
+# ---------------------------------------------------------------- partials of a split sequence
+
+def _partial_case(seed=5, N=150, q_len=3):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((q_len, om.N_HEADS, om.D_NOPE + om.D_ROPE))
+    c = rng.standard_normal((N, om.D_LATENT))
+    k = rng.standard_normal((N, om.D_ROPE))
+    W_UK = rng.standard_normal((om.N_HEADS, om.D_NOPE, om.D_LATENT)) / math.sqrt(om.D_LATENT)
+    W_UV = rng.standard_normal((om.N_HEADS, om.D_LATENT, om.D_V)) / math.sqrt(om.D_LATENT)
+    return q, c, k, W_UK, W_UV
+
+
+def test_partial_of_one_token_is_that_token():
+    # one visible token: l = exp(0) = 1 and O is its latent row; the difference of
+    # two tokens' m is their log-probability ratio under the expanded definition
+    q, c, k, W_UK, _ = _partial_case(q_len=1)
+    cfg = om.YarnConfig()
+    N = c.shape[0]
+    k_rot = om.rope(k, np.arange(N), cfg)
+    t = 41
+    m, l, O = om.attention_partial(q, c[t:t + 1], k_rot[t:t + 1], W_UK, cfg, N, t, t + 1)
+    assert np.all(l == 1.0)
+    assert np.array_equal(O, np.broadcast_to(c[t], O.shape))
+    m_u, _, _ = om.attention_partial(q, c[t + 1:t + 2], k_rot[t + 1:t + 2], W_UK, cfg, N,
+                                     t + 1, t + 2)
+    P = om.mla_attention_probs(q, c, k, W_UK, cfg)
+    assert np.abs(np.log(P[0, :, t] / P[0, :, t + 1]) - (m[0] - m_u[0])).max() < 1e-9
+
+
+def test_empty_and_fully_masked_partials_see_nothing():
+    q, c, k, W_UK, _ = _partial_case()
+    cfg = om.YarnConfig()
+    N = c.shape[0]
+    for lo, hi in [(10, 10), (N, N)]:
+        m, l, O = om.attention_partial(q, c[lo:hi], k[lo:hi], W_UK, cfg, N, lo, hi)
+        assert np.all(m == -np.inf) and np.all(l == 0) and np.all(O == 0)
+    # the last token is visible only to the last query (q_len = 3)
+    m, l, O = om.attention_partial(q, c[N - 1:], k[N - 1:], W_UK, cfg, N, N - 1, N)
+    assert np.all(l[:-1] == 0) and np.all(m[:-1] == -np.inf) and np.all(O[:-1] == 0)
+    assert np.all(l[-1] == 1)
+
+
+@pytest.mark.parametrize("cuts", [[70], [1, 2, 149], [64, 128], [30, 60, 90, 120]])
+def test_merged_partials_equal_the_expanded_definition(cuts):
+    # the partials of any partition of the tokens merge to the attention of the
+    # expanded (non-absorbed) definition, in either order of the parts
+    q, c, k, W_UK, W_UV = _partial_case()
+    cfg = om.YarnConfig()
+    N = c.shape[0]
+    k_rot = om.rope(k, np.arange(N), cfg)
+    edges = [0] + cuts + [N]
+    parts = [om.attention_partial(q, c[a:b], k_rot[a:b], W_UK, cfg, N, a, b)
+             for a, b in zip(edges[:-1], edges[1:])]
+    want = om.mla_attention_expanded(q, c, k, W_UK, W_UV, cfg)
+    for order in (parts, parts[::-1]):
+        got = om.finish_partial(*om.merge_partials(order), W_UV)
+        assert np.abs(got - want).max() < 1e-12
+
+
+def test_merge_is_associative_and_has_the_empty_part_as_identity():
+    q, c, k, W_UK, _ = _partial_case(seed=9)
+    cfg = om.YarnConfig()
+    N = c.shape[0]
+    a = om.attention_partial(q, c[:50], k[:50], W_UK, cfg, N, 0, 50)
+    b = om.attention_partial(q, c[50:90], k[50:90], W_UK, cfg, N, 50, 90)
+    d = om.attention_partial(q, c[90:], k[90:], W_UK, cfg, N, 90, N)
+    e = om.attention_partial(q, c[:0], k[:0], W_UK, cfg, N, 0, 0)
+    flat = om.merge_partials([a, b, d])
+    for x in (om.merge_partials([om.merge_partials([a, b]), d]),
+              om.merge_partials([a, om.merge_partials([b, d])])):
+        assert np.array_equal(x[0], flat[0])                 # the maximum is exact
+        assert np.allclose(x[1], flat[1], rtol=1e-14, atol=0)
+        assert np.allclose(x[2], flat[2], rtol=1e-13, atol=1e-13)
+    with_e = om.merge_partials([a, e])
+    assert np.array_equal(with_e[0], a[0]) and np.array_equal(with_e[1], a[1])
+    assert np.array_equal(with_e[2], a[2])
