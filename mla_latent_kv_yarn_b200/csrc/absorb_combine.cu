@@ -114,15 +114,128 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
   }
 }
 
+// ---------------------------------------------------------------- length-aware split plan
+
+// Sum (kMax false) or maximum over the 128 threads of a block, returned to all.
+template <bool kMax>
+__device__ __forceinline__ long long plan_reduce(long long v, long long* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const long long x = __shfl_xor_sync(0xffffffffu, v, o);
+    v = kMax ? max(v, x) : v + x;
+  }
+  __syncthreads();  // the previous call's readers are done with red
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  v = red[0];
+#pragma unroll
+  for (int k = 1; k < kAbsorbThreads / 32; ++k) v = kMax ? max(v, red[k]) : v + red[k];
+  return v;
+}
+
+// Shared memory of the plan kernel: pages per unit, reduction and scan slots.
+struct PlanSmem {
+  int w[kMaxPlanCtas];
+  long long red[kAbsorbThreads / 32];
+  int scan[kAbsorbThreads / 32];
+};
+
+// The plan of WorkPlanArgs, by one block of 128 threads.  Unit u = b * groups
+// + g has w_u = ceil(seqlen_b / 64) pages; T is the smallest page count per
+// CTA for which sum_u max(1, ceil(w_u / T)) CTAs fit in the grid (at least two
+// pages per CTA unless a unit has fewer), found by bisection: T = ceil(total /
+// (ctas - units)) always fits, and so does T = max_u w_u.  Unit u then gets
+// ns_u = max(1, ceil(w_u / T)) CTAs, consecutive in unit order, each a run of
+// ceil(w_u / ns_u) <= T pages; CTAs past the last unit get no work.  It runs
+// as one extra block of the first kernel of a decode call, side by side with
+// the absorb; the split-K kernel waits for that kernel and so finds the tables.
+__device__ __forceinline__ void work_plan_block(const WorkPlanArgs& a, PlanSmem& sm) {
+  int* w_s = sm.w;
+  long long* red = sm.red;
+  int* scan_s = sm.scan;
+  const int t = threadIdx.x;
+  const int units = a.batch * a.groups;  // < a.ctas <= kMaxPlanCtas = 2 * kAbsorbThreads
+  pdl_wait();                            // the lengths may come from the kernel launched before
+  long long tot = 0, wmax = 0;
+  for (int u = t; u < units; u += kAbsorbThreads) {
+    int64_t n = a.seqlens[u / a.groups];
+    if (n < 0 || n > a.max_seqlen) n = 0;  // the split-K kernel reports the bad length
+    const int w = (int)((n + kPage - 1) / kPage);
+    w_s[u] = w;
+    tot += w;
+    wmax = max(wmax, (long long)w);
+  }
+  tot = plan_reduce<false>(tot, red);
+  wmax = plan_reduce<true>(wmax, red);
+  const long long spare = a.ctas - units;
+  long long lo = max(max(1LL, (tot + a.ctas - 1) / a.ctas), min(2LL, wmax));
+  long long hi = max(lo, min(max(wmax, 1LL), max(1LL, (tot + spare - 1) / spare)));
+  while (lo < hi) {  // uniform across the block: every thread sees the same sums
+    const long long mid = (lo + hi) >> 1;
+    long long c = 0;
+    for (int u = t; u < units; u += kAbsorbThreads) c += max(1LL, (w_s[u] + mid - 1) / mid);
+    c = plan_reduce<false>(c, red);
+    if (c <= a.ctas) hi = mid;
+    else lo = mid + 1;
+  }
+  const long long T = lo;
+  // first CTA of each unit: exclusive prefix sum of ns_u, units 2t and 2t + 1 on thread t
+  const int u0 = 2 * t, u1 = 2 * t + 1;
+  const int ns0 = u0 < units ? (int)max(1LL, (w_s[u0] + T - 1) / T) : 0;
+  const int ns1 = u1 < units ? (int)max(1LL, (w_s[u1] + T - 1) / T) : 0;
+  const int v = ns0 + ns1;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+    if ((t & 31) >= o) incl += x;
+  }
+  if ((t & 31) == 31) scan_s[t >> 5] = incl;
+  __syncthreads();
+  int before = 0, total = 0;
+#pragma unroll
+  for (int k = 0; k < kAbsorbThreads / 32; ++k) {
+    before += k < (t >> 5) ? scan_s[k] : 0;
+    total += scan_s[k];
+  }
+  const int first0 = before + incl - v;
+  auto emit = [&](int u, int first, int ns) {
+    const int w = w_s[u];
+    const int pps = (w + ns - 1) / ns;
+    a.unit_tab[u] = make_int2(first, ns);
+    for (int s = 0; s < ns; ++s)
+      a.work_tab[first + s] = make_int4(u, min(w, s * pps), min(w, (s + 1) * pps), 0);
+  };
+  if (ns0 > 0) emit(u0, first0, ns0);
+  if (ns1 > 0) emit(u1, first0 + ns0, ns1);
+  for (int k = total + t; k < a.ctas; k += kAbsorbThreads) a.work_tab[k] = make_int4(-1, 0, 0, 0);
+}
+
+static bool plan_ok(const WorkPlanArgs& plan) {
+  return plan.ctas > plan.batch * plan.groups && plan.ctas <= kMaxPlanCtas;
+}
+
 // q and seqlens carry no __restrict__ so that their loads stay behind the
 // griddepcontrol.wait (a preceding kernel may have written them).
+// kPlan: block kAbsorbBlocks computes the length-aware plan (batch > 1).
+template <bool kPlan>
 __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
-    __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, float qscale, const RopeTable tab) {
-  __shared__ AbsorbSmem sm;
+    __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, float qscale, const RopeTable tab,
+    const WorkPlanArgs plan) {
+  __shared__ union {
+    AbsorbSmem absorb;
+    PlanSmem plan;
+  } sm;
   pdl_launch_dependents();
+  if constexpr (kPlan) {
+    if (blockIdx.x == kAbsorbBlocks) {
+      work_plan_block(plan, sm.plan);
+      return;
+    }
+  }
   q_absorb_block(blockIdx.x % kHeads, blockIdx.x / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
-                 qscale, tab, sm);
+                 qscale, tab, sm.absorb);
 }
 
 // The first kernel of a decode step: the absorb blocks above, then the
@@ -130,14 +243,18 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
 // warps each; pa.T == 0 otherwise), then blocks that append the step's ready
 // cache rows (one thread per 16-byte piece).  All of them only wait for the
 // kernel launched before this one, so they run side by side.
+// kPlan: block kAbsorbBlocks computes the length-aware plan (batch > 1); the
+// producer and append blocks follow it.
+template <bool kPlan>
 __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
     __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, float qscale, const RopeTable q_tab,
-    const AppendArgs ap, const RopeTable k_tab, const ProduceArgs pa) {
+    const AppendArgs ap, const RopeTable k_tab, const ProduceArgs pa, const WorkPlanArgs plan) {
   // one buffer for whichever role the block takes
   __shared__ union {
     AbsorbSmem absorb;
     ProduceSmem<kAbsorbThreads / 32> produce;
+    PlanSmem plan;
   } sm;
   pdl_launch_dependents();
   if (blockIdx.x < kAbsorbBlocks) {
@@ -145,16 +262,25 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
                    qscale, q_tab, sm.absorb);
     return;
   }
+  constexpr int kPlanBlocks = kPlan ? 1 : 0;
+  if constexpr (kPlan) {
+    if (blockIdx.x == kAbsorbBlocks) {
+      work_plan_block(plan, sm.plan);
+      return;
+    }
+  }
   const int prod_blocks = pa.T > 0 ? kProdBlocks : 0;
-  if (blockIdx.x < kAbsorbBlocks + prod_blocks) {
-    produce_block<kAbsorbThreads / 32>(blockIdx.x - kAbsorbBlocks, threadIdx.x, pa, k_tab,
-                                       sm.produce, [] { __syncthreads(); }, [] { pdl_wait(); });
+  if (blockIdx.x < kAbsorbBlocks + kPlanBlocks + prod_blocks) {
+    produce_block<kAbsorbThreads / 32>(blockIdx.x - kAbsorbBlocks - kPlanBlocks, threadIdx.x, pa,
+                                       k_tab, sm.produce, [] { __syncthreads(); },
+                                       [] { pdl_wait(); });
     return;
   }
   pdl_wait();
   const int64_t total = ap.T * kRowPieces;
   const int64_t idx =
-      (int64_t)(blockIdx.x - kAbsorbBlocks - prod_blocks) * kAbsorbThreads + threadIdx.x;
+      (int64_t)(blockIdx.x - kAbsorbBlocks - kPlanBlocks - prod_blocks) * kAbsorbThreads +
+      threadIdx.x;
   if (idx < total)
     append_piece(idx, ap.pool, ap.num_blocks, ap.block_table, ap.max_blocks, ap.batch, ap.seq_ids,
                  ap.positions, ap.c_kv, ap.k_pe, ap.status, ap.rotate, k_tab);
@@ -162,25 +288,39 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
 
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
-                            float qscale, const RopeTable& tab, cudaStream_t st) {
-  return launch_pdl(q_absorb_kernel, dim3(kAbsorbBlocks), dim3(kAbsorbThreads), 0, st, q, W_UK,
-                    seqlens, q_ext, rows, q_len, qscale, tab);
+                            float qscale, const RopeTable& tab, const WorkPlanArgs* plan,
+                            cudaStream_t st) {
+  if (plan != nullptr) {
+    if (!plan_ok(*plan)) return cudaErrorInvalidValue;
+    return launch_pdl(q_absorb_kernel<true>, dim3(kAbsorbBlocks + 1), dim3(kAbsorbThreads), 0, st,
+                      q, W_UK, seqlens, q_ext, rows, q_len, qscale, tab, *plan);
+  }
+  return launch_pdl(q_absorb_kernel<false>, dim3(kAbsorbBlocks), dim3(kAbsorbThreads), 0, st, q,
+                    W_UK, seqlens, q_ext, rows, q_len, qscale, tab, WorkPlanArgs{});
 }
 
 cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                                  const int32_t* seqlens, __nv_bfloat16* q_ext, int rows,
                                  int q_len, float qscale, const RopeTable& q_tab,
                                  const AppendArgs& ap, const RopeTable& k_tab,
-                                 const ProduceArgs* pa, cudaStream_t st) {
+                                 const ProduceArgs* pa, const WorkPlanArgs* plan,
+                                 cudaStream_t st) {
   const int64_t append_blocks = (ap.T * kRowPieces + kAbsorbThreads - 1) / kAbsorbThreads;
   if (append_blocks > (1 << 20)) return cudaErrorInvalidValue;
   ProduceArgs none{};
   const ProduceArgs& p = pa != nullptr ? *pa : none;
   const int64_t prod_blocks = p.T > 0 ? kProdBlocks : 0;
-  return launch_pdl(step_prologue_kernel,
+  if (plan != nullptr) {
+    if (!plan_ok(*plan)) return cudaErrorInvalidValue;
+    return launch_pdl(step_prologue_kernel<true>,
+                      dim3((unsigned)(kAbsorbBlocks + 1 + prod_blocks + append_blocks)),
+                      dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, qscale,
+                      q_tab, ap, k_tab, p, *plan);
+  }
+  return launch_pdl(step_prologue_kernel<false>,
                     dim3((unsigned)(kAbsorbBlocks + prod_blocks + append_blocks)),
                     dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, qscale,
-                    q_tab, ap, k_tab, p);
+                    q_tab, ap, k_tab, p, WorkPlanArgs{});
 }
 
 // ---------------------------------------------------------------- combine + W_UV
@@ -289,13 +429,15 @@ __device__ __forceinline__ void merge_group(const float* po, const float2* pml, 
 
 // kStrided: splits are o_stride floats / ml_stride (m, l) pairs apart (the
 // gathered partials of a sequence-parallel decode); otherwise rows_per_cta
-// rows apart, as the split-K kernel writes them.
-template <bool kStrided>
+// rows apart, as the split-K kernel writes them.  kTable: the splits of a
+// (sequence, row group) unit are those unit_tab gives (length-aware plan),
+// read after the wait; otherwise nsplit per unit, unit after unit.
+template <bool kStrided, bool kTable>
 __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThreads, 3)
     combine_uv_kernel(const float* part_o, const float* part_ml,
                       const __nv_bfloat16* __restrict__ W_UV, __nv_bfloat16* __restrict__ out,
                       int rows, int q_len, int groups, int nsplit, int rows_per_cta,
-                      int64_t o_stride_arg, int64_t ml_stride_arg) {
+                      int64_t o_stride_arg, int64_t ml_stride_arg, const int2* unit_tab) {
   // part_o and part_ml are written by the kernel launched just before this one,
   // which lets this grid start early: they carry no __restrict__, so their loads
   // are not taken as invariant and stay behind the griddepcontrol.wait below.
@@ -334,11 +476,13 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThread
   const int sub = grp % gpr;
   const bool active = my_rr < nr;
   int64_t base = 0;  // partial row of split 0; split s is s * rows_per_cta rows further
+  int unit = 0, ridx = 0;
   if (active) {
     const int r = r0 + my_rr;  // r = b*q_len + j
     const int b = r / q_len, j = r % q_len;
-    const int ridx = j * kHeads + h;
-    base = ((int64_t)b * groups + ridx / rows_per_cta) * nsplit * rows_per_cta + ridx % rows_per_cta;
+    ridx = j * kHeads + h;
+    unit = b * groups + ridx / rows_per_cta;
+    base = (int64_t)unit * nsplit * rows_per_cta + ridx % rows_per_cta;
   }
   const float* po = part_o + base * kDLatent + slice * kSliceDims + 4 * q4;
   const float2* pml = reinterpret_cast<const float2*>(part_ml) + base;
@@ -347,9 +491,18 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThread
 
   pdl_wait();  // the split partials come from the decode kernel
 
+  int ns = nsplit;
+  if constexpr (kTable) {
+    // the plan was written by the first kernel of the call, complete before the decode kernel
+    const int2 ut = active ? unit_tab[unit] : make_int2(0, 0);
+    ns = ut.y;
+    base = (int64_t)ut.x * rows_per_cta + ridx % rows_per_cta;
+    po = part_o + base * kDLatent + slice * kSliceDims + 4 * q4;
+    pml = reinterpret_cast<const float2*>(part_ml) + base;
+  }
   float m_g, l_g;
   float4 acc;
-  merge_group(po, pml, o_stride, ml_stride, nsplit, sub, gpr, q4, active, m_g, l_g, acc);
+  merge_group(po, pml, o_stride, ml_stride, ns, sub, gpr, q4, active, m_g, l_g, acc);
   acc_s[grp][q4] = acc;
   if (q4 == 0) {
     grp_m[grp] = m_g;
@@ -417,15 +570,22 @@ __global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThread
 cudaError_t launch_combine(const float* part_o, const float* part_ml, const __nv_bfloat16* W_UV,
                            __nv_bfloat16* out, int rows, int q_len, int groups, int nsplit,
                            int rows_per_cta, cudaStream_t st, int64_t o_stride,
-                           int64_t ml_stride) {
+                           int64_t ml_stride, const int2* unit_tab) {
   const int chunks = (rows + kCombineRows - 1) / kCombineRows;
   const dim3 grid(kSlices * kHeads * chunks);
-  if (o_stride == 0 && ml_stride == 0)
-    return launch_pdl(combine_uv_kernel<false>, grid, dim3(kCombineThreads), 0, st, part_o,
+  const bool strided = o_stride != 0 || ml_stride != 0;
+  if (strided && unit_tab != nullptr) return cudaErrorInvalidValue;
+  if (unit_tab != nullptr)
+    return launch_pdl(combine_uv_kernel<false, true>, grid, dim3(kCombineThreads), 0, st, part_o,
                       part_ml, W_UV, out, rows, q_len, groups, nsplit, rows_per_cta, (int64_t)0,
-                      (int64_t)0);
-  return launch_pdl(combine_uv_kernel<true>, grid, dim3(kCombineThreads), 0, st, part_o, part_ml,
-                    W_UV, out, rows, q_len, groups, nsplit, rows_per_cta, o_stride, ml_stride);
+                      (int64_t)0, unit_tab);
+  if (!strided)
+    return launch_pdl(combine_uv_kernel<false, false>, grid, dim3(kCombineThreads), 0, st, part_o,
+                      part_ml, W_UV, out, rows, q_len, groups, nsplit, rows_per_cta, (int64_t)0,
+                      (int64_t)0, unit_tab);
+  return launch_pdl(combine_uv_kernel<true, false>, grid, dim3(kCombineThreads), 0, st, part_o,
+                    part_ml, W_UV, out, rows, q_len, groups, nsplit, rows_per_cta, o_stride,
+                    ml_stride, unit_tab);
 }
 
 // ---------------------------------------------------------------- merge of one shard's splits

@@ -24,10 +24,29 @@ namespace xmla {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Length-aware split plan of a batch, computed on the device by one extra
+// block of the first kernel of the call (after its griddepcontrol.wait, from
+// the sequence lengths): every (sequence, row group) unit u gets ns_u >= 1 of
+// the `ctas` split-K CTAs and its pages are divided evenly over them, with the
+// largest share per CTA as small as the CTA count allows.  unit_tab[u] =
+// {first CTA, ns_u}; work_tab[k] as in DecodeParams.
+constexpr int kMaxPlanCtas = 256;
+struct WorkPlanArgs {
+  const int32_t* seqlens;
+  int64_t max_seqlen;
+  int32_t batch;
+  int32_t groups;
+  int32_t ctas;  // split-K grid size, units < ctas <= kMaxPlanCtas
+  int4* work_tab;
+  int2* unit_tab;
+};
+
 // q_ext[r, h] for rows r = b*q_len + j; qscale = softmax scale * log2 e.
+// plan (nullable): also compute the length-aware plan.
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
-                            float qscale, const RopeTable& tab, cudaStream_t st);
+                            float qscale, const RopeTable& tab, const WorkPlanArgs* plan,
+                            cudaStream_t st);
 
 // The new tokens of a decode step, appended by step_prologue_kernel.
 struct AppendArgs {
@@ -46,20 +65,24 @@ struct AppendArgs {
 };
 
 // q_absorb and the cache rows of the same step in one launch: ready rows are
-// appended (ap), rows from hidden states are produced (pa, nullable).
+// appended (ap), rows from hidden states are produced (pa, nullable); plan
+// (nullable) as for launch_q_absorb.
 cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                                  const int32_t* seqlens, __nv_bfloat16* q_ext, int rows,
                                  int q_len, float qscale, const RopeTable& q_tab,
                                  const AppendArgs& ap, const RopeTable& k_tab,
-                                 const ProduceArgs* pa, cudaStream_t st);
+                                 const ProduceArgs* pa, const WorkPlanArgs* plan,
+                                 cudaStream_t st);
 
 // Merge of the splits and the W_UV product, written to out[rows, 32, 128].
 // Split s of a row is o_stride floats (O) and ml_stride (m, l) pairs after
 // split 0; 0 means the split-K kernel's layout (rows_per_cta rows apart).
+// unit_tab (non-null, split-K layout only): the splits of unit u are the
+// unit_tab[u].y work items from unit_tab[u].x on, as the plan above made them.
 cudaError_t launch_combine(const float* part_o, const float* part_ml, const __nv_bfloat16* W_UV,
                            __nv_bfloat16* out, int rows, int q_len, int groups, int nsplit,
                            int rows_per_cta, cudaStream_t st, int64_t o_stride = 0,
-                           int64_t ml_stride = 0);
+                           int64_t ml_stride = 0, const int2* unit_tab = nullptr);
 
 // Merge of the splits into one partial per (row, head) -- (M, L, unnormalised
 // O) -- for a sequence-parallel decode; layout in absorb_combine.cu.

@@ -126,9 +126,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// kRanged: the call covers the logical pages [p.page_lo, p.page_hi) of every
-// sequence (one rank's share of a sequence-parallel decode); otherwise all.
-template <int NR, bool kRanged>
+// How a CTA finds its pages.
+enum WorkMode : int {
+  kWorkSplit = 0,   // split (blockIdx % nsplit) of every sequence's pages
+  kWorkRanged = 1,  // the same over the logical pages [p.page_lo, p.page_hi) of every sequence
+                    // (one rank's share of a sequence-parallel decode)
+  kWorkTable = 2,   // entry blockIdx of p.work_tab (written by the preceding kernel)
+};
+
+template <int NR, int kMode>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tmap_pool,
                       const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p) {
@@ -151,25 +157,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
   // ---- work item
   const int item = blockIdx.x;
-  const int split = item % p.nsplit;
-  const int bg = item / p.nsplit;
-  const int g = bg % p.groups;
-  const int b = bg / p.groups;
-  const int j0 = g * (NR / 32);
-  const int jn = min(p.q_len - j0, NR / 32);
-  const int nrows = jn * 32;
-  int64_t seqlen = p.seqlens[b];
-  if (seqlen < p.q_len || seqlen > p.max_seqlen) {
-    if (threadIdx.x == 0) record_status(p.status, XMLA_ERR_DEVICE_OOB);
-    seqlen = 0;
+  int b = 0, g = 0;
+  int64_t seqlen = 0, npages = 0, p_begin = 0, p_end = 0;
+  if constexpr (kMode != kWorkTable) {
+    const int split = item % p.nsplit;
+    const int bg = item / p.nsplit;
+    g = bg % p.groups;
+    b = bg / p.groups;
+    seqlen = p.seqlens[b];
+    if (seqlen < p.q_len || seqlen > p.max_seqlen) {
+      if (threadIdx.x == 0) record_status(p.status, XMLA_ERR_DEVICE_OOB);
+      seqlen = 0;
+    }
+    npages = (seqlen + kPage - 1) / kPage;
+    const int64_t p_lo = kMode == kWorkRanged ? min(p.page_lo, npages) : 0;
+    const int64_t p_hi = kMode == kWorkRanged ? min(p.page_hi, npages) : npages;
+    const int64_t pps = (p_hi - p_lo + p.nsplit - 1) / p.nsplit;
+    p_begin = p_lo + (int64_t)split * pps;
+    p_end = min(p_hi, p_begin + pps);
   }
-  const int64_t npages = (seqlen + kPage - 1) / kPage;
-  const int64_t p_lo = kRanged ? min(p.page_lo, npages) : 0;
-  const int64_t p_hi = kRanged ? min(p.page_hi, npages) : npages;
-  const int64_t pps = (p_hi - p_lo + p.nsplit - 1) / p.nsplit;
-  const int64_t p_begin = p_lo + (int64_t)split * pps;
-  const int64_t p_end = min(p_hi, p_begin + pps);
-  const int n_pages = (int)max((int64_t)0, p_end - p_begin);
 
   // ---- setup (independent of the previous kernel's results)
   if (threadIdx.x == 0) {
@@ -203,6 +209,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + L::kOffTmem);
+  if constexpr (kMode == kWorkTable) {
+    // the table comes from the kernel launched before this one
+    pdl_wait();
+    const int4 e = p.work_tab[item];
+    if (e.x >= 0 && e.x < p.batch * p.groups) {
+      g = e.x % p.groups;
+      b = e.x / p.groups;
+      seqlen = p.seqlens[b];
+      if (seqlen < p.q_len || seqlen > p.max_seqlen) {
+        if (threadIdx.x == 0) record_status(p.status, XMLA_ERR_DEVICE_OOB);
+        seqlen = 0;
+      }
+      npages = (seqlen + kPage - 1) / kPage;
+      p_begin = min((int64_t)e.y, npages);
+      p_end = min((int64_t)e.z, npages);
+    }
+  }
+  const int j0 = g * (NR / 32);
+  const int jn = min(p.q_len - j0, NR / 32);
+  const int nrows = jn * 32;
+  const int n_pages = (int)max((int64_t)0, p_end - p_begin);
   const int32_t qrow0 = (int32_t)(((int64_t)b * p.q_len + j0) * 32);
   pdl_launch_dependents();
 
@@ -577,7 +604,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
 }
 
-template <int NR, bool kRanged>
+template <int NR, int kMode>
 static cudaError_t launch_decode(const CUtensorMap& tp, const CUtensorMap& tq, const DecodeParams& dp,
                                  int64_t items, cudaStream_t st) {
   using L = DecodeLayout<NR>;
@@ -586,23 +613,31 @@ static cudaError_t launch_decode(const CUtensorMap& tp, const CUtensorMap& tq, c
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<NR, kRanged>,
+    cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<NR, kMode>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  return launch_pdl(mla_decode_kernel<NR, kRanged>, dim3((unsigned)items), dim3(kDecodeThreads), L::kSmem,
-                    st, tp, tq, dp);
+  return launch_pdl(mla_decode_kernel<NR, kMode>, dim3((unsigned)items), dim3(kDecodeThreads),
+                    L::kSmem, st, tp, tq, dp);
 }
 
 
 cudaError_t launch_split_kv(int nr, const CUtensorMap& pool_map, const CUtensorMap& q_map,
                             const DecodeParams& dp, int64_t items, cudaStream_t st) {
-  const bool ranged = dp.page_lo != 0 || dp.page_hi != INT64_MAX;
-  if (nr == 32) return ranged ? launch_decode<32, true>(pool_map, q_map, dp, items, st)
-                              : launch_decode<32, false>(pool_map, q_map, dp, items, st);
-  if (nr == 64) return ranged ? launch_decode<64, true>(pool_map, q_map, dp, items, st)
-                              : launch_decode<64, false>(pool_map, q_map, dp, items, st);
+  const int mode = dp.work_tab != nullptr                          ? kWorkTable
+                   : (dp.page_lo != 0 || dp.page_hi != INT64_MAX) ? kWorkRanged
+                                                                  : kWorkSplit;
+  if (nr == 32) {
+    if (mode == kWorkTable) return launch_decode<32, kWorkTable>(pool_map, q_map, dp, items, st);
+    if (mode == kWorkRanged) return launch_decode<32, kWorkRanged>(pool_map, q_map, dp, items, st);
+    return launch_decode<32, kWorkSplit>(pool_map, q_map, dp, items, st);
+  }
+  if (nr == 64) {
+    if (mode == kWorkTable) return launch_decode<64, kWorkTable>(pool_map, q_map, dp, items, st);
+    if (mode == kWorkRanged) return launch_decode<64, kWorkRanged>(pool_map, q_map, dp, items, st);
+    return launch_decode<64, kWorkSplit>(pool_map, q_map, dp, items, st);
+  }
   return cudaErrorInvalidValue;
 }
 

@@ -13,7 +13,8 @@ namespace xmla {
 constexpr int kMaxSplits = 1024;
 
 // Arguments of the split-K attention kernel.  Partial results are laid out
-// per work item (sequence b, row group g, split s) in that order.
+// per work item: (sequence b, row group g, split s) in that order, or, with a
+// work table, in the order of the table's entries.
 struct DecodeParams {
   const int32_t* block_table;
   const int32_t* seqlens;
@@ -33,6 +34,11 @@ struct DecodeParams {
   // splits partition that range
   int64_t page_lo;
   int64_t page_hi;
+  // non-null: a work table written on the device by the first kernel of the
+  // call (length-aware plan, batch > 1): entry k = {unit b * groups + g,
+  // first logical page, end page, 0} of CTA k, unit -1 for an idle CTA.  The
+  // kernel reads it after griddepcontrol.wait; nsplit and page_lo/hi are unused.
+  const int4* work_tab;
 };
 
 // Split-K attention over `items` work items; nr = rows per CTA (32 or 64).

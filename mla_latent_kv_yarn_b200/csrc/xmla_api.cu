@@ -33,17 +33,22 @@ __global__ void wait_timeout_selftest_kernel(int32_t* status, uint64_t limit_ns)
 struct Plan {
   int nr;       // rows per CTA (32 or 64)
   int groups;   // row groups per sequence
-  int nsplit;   // KV splits per (sequence, group)
+  int nsplit;   // KV splits per (sequence, group) when every sequence has max_seqlen tokens
+  bool table;   // splits planned on the device from the actual lengths (WorkPlanArgs)
   int64_t items;
-  size_t off_qext, off_o, off_ml, bytes;
+  size_t off_qext, off_o, off_ml, off_wtab, off_utab, bytes;
 };
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // span_pages: logical pages a call attends over at most (the split count is
-// sized for them); 0 = all pages of max_seqlen.
+// sized for them); 0 = all pages of max_seqlen.  allow_table: a batch of
+// several sequences with automatic splits gets the length-aware plan: one
+// CTA per SM, the pages of each sequence divided over them in proportion to
+// its length by the first kernel of the call.
 static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_sms,
-                      int32_t num_splits, Plan* pl, int64_t span_pages = 0) {
+                      int32_t num_splits, Plan* pl, int64_t span_pages = 0,
+                      bool allow_table = true) {
   if (B < 1 || q_len < 1 || q_len > kMaxQLen || max_seqlen < q_len ||
       max_seqlen > (int64_t)0x7fffffff - kPage || num_sms < 1 || num_splits < 0 || span_pages < 0)
     return false;
@@ -64,13 +69,18 @@ static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_
   if (ns < 1) ns = 1;
   if (ns > kMaxSplits) return false;
   P.nsplit = (int)ns;
-  P.items = (int64_t)B * P.groups * P.nsplit;
+  const int64_t units = (int64_t)B * P.groups;
+  P.table = allow_table && num_splits == 0 && span_pages == 0 && B > 1 && units < num_sms &&
+            num_sms <= kMaxPlanCtas;
+  P.items = P.table ? num_sms : units * P.nsplit;
   if (P.items > 0x7fffffff) return false;
   const size_t qext = (size_t)B * q_len * kHeads * kDRow * 2;
   P.off_qext = 0;
   P.off_o = align_up(qext, 1024);
   P.off_ml = align_up(P.off_o + (size_t)P.items * P.nr * kDLatent * 4, 1024);
-  P.bytes = align_up(P.off_ml + (size_t)P.items * P.nr * 2 * 4, 1024);
+  P.off_wtab = align_up(P.off_ml + (size_t)P.items * P.nr * 2 * 4, 1024);
+  P.off_utab = align_up(P.off_wtab + (P.table ? (size_t)P.items * 16 : 0), 256);
+  P.bytes = align_up(P.off_utab + (P.table ? (size_t)units * 8 : 0), 1024);
   *pl = P;
   return true;
 }
@@ -168,7 +178,8 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   if (!device_ok(&nsm)) return XMLA_ERR_UNSUPPORTED;
   Plan P;
   const int64_t span = page_hi == INT64_MAX ? 0 : (page_hi > page_lo ? page_hi - page_lo : 1);
-  if (!make_plan(batch, q_len, max_seqlen, nsm, num_splits, &P, span)) return XMLA_ERR_SHAPE;
+  if (!make_plan(batch, q_len, max_seqlen, nsm, num_splits, &P, span, shard_partial == nullptr))
+    return XMLA_ERR_SHAPE;
   if (workspace_bytes < P.bytes) return XMLA_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
   uint8_t* ws = (uint8_t*)workspace;
@@ -181,15 +192,26 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
 
   const float qscale = softmax_scale * kLog2e;
   const RopeTable tab = make_rope_table(cfg);
+  WorkPlanArgs plan{};
+  if (P.table) {
+    plan.seqlens = seqlens;
+    plan.max_seqlen = max_seqlen;
+    plan.batch = batch;
+    plan.groups = P.groups;
+    plan.ctas = (int32_t)P.items;
+    plan.work_tab = (int4*)(ws + P.off_wtab);
+    plan.unit_tab = (int2*)(ws + P.off_utab);
+  }
   // Every kernel of the chain waits (griddepcontrol.wait) for its predecessor
   // before reading anything a kernel of this step may have written, so once
   // the first kernel completes all earlier work on the stream has landed.
   const cudaError_t e0 =
       ap != nullptr
           ? launch_step_prologue((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
-                                 rows, q_len, qscale, tab, *ap, tab, pa, st)
+                                 rows, q_len, qscale, tab, *ap, tab, pa,
+                                 P.table ? &plan : nullptr, st)
           : launch_q_absorb((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
-                            rows, q_len, qscale, tab, st);
+                            rows, q_len, qscale, tab, P.table ? &plan : nullptr, st);
   if (e0 != cudaSuccess) return XMLA_ERR_CUDA;
 
   DecodeParams dp;
@@ -208,6 +230,7 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   dp.nsplit = P.nsplit;
   dp.page_lo = page_lo;
   dp.page_hi = page_hi;
+  dp.work_tab = P.table ? plan.work_tab : nullptr;
   if (record_event(attn_start, st) != cudaSuccess) return XMLA_ERR_CUDA;
   if (launch_split_kv(P.nr, tmap_pool, tmap_q, dp, P.items, st) != cudaSuccess) return XMLA_ERR_CUDA;
   if (record_event(attn_stop, st) != cudaSuccess) return XMLA_ERR_CUDA;
@@ -218,7 +241,7 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   }
   const cudaError_t e = launch_combine(dp.part_o, dp.part_ml, (const __nv_bfloat16*)W_UV,
                                        (__nv_bfloat16*)out, rows, q_len, P.groups, P.nsplit, P.nr,
-                                       st);
+                                       st, 0, 0, P.table ? plan.unit_tab : nullptr);
   return e == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
 }
 

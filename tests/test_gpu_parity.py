@@ -207,6 +207,96 @@ def test_decode_theta_1e7():
     gc.assert_close(out, gc.oracle_out(wl, inp, ocfg), "theta 1e7")
 
 
+# ------------------------------------------------------------------ length-aware split plan
+
+# A batch of several sequences with automatic splits is planned on the device:
+# the first kernel of the call gives each (sequence, row group) unit a share of
+# the SM-count CTAs in proportion to its pages.  Lengths far apart put most
+# CTAs on one sequence and one CTA on each short one.
+PLAN_CASES = [
+    # batch, q_len, seqlens
+    (2, 1, [3000, 100]),
+    (6, 1, [1, 64, 65, 2500, 700, 129]),
+    (3, 4, [2200, 300, 4]),
+    (5, 8, [1200, 70, 640, 65, 999]),
+]
+
+
+def _plan_tables(dec: session.Decoder):
+    """The work and unit tables the first kernel left in the decoder's
+    workspace (layout of the library's workspace plan: q_ext, split O, split
+    (m, l), then the two tables)."""
+    def up(x, a):
+        return (x + a - 1) // a * a
+    nr = 32 if dec.q_len == 1 else 64
+    groups = (dec.q_len * 32 + nr - 1) // nr
+    items = dec.sms
+    off_o = up(dec.batch * dec.q_len * 32 * 576 * 2, 1024)
+    off_ml = up(off_o + items * nr * 512 * 4, 1024)
+    off_w = up(off_ml + items * nr * 2 * 4, 1024)
+    off_u = up(off_w + items * 16, 256)
+    ws = dec.workspace
+    work = ws[off_w:off_w + items * 16].view(torch.int32).view(items, 4).cpu().numpy()
+    unit = ws[off_u:off_u + dec.batch * groups * 8].view(torch.int32).view(-1, 2).cpu().numpy()
+    return work, unit, groups
+
+
+@pytest.mark.parametrize("batch,q_len,seqlens", PLAN_CASES)
+def test_length_aware_plan_matches_expanded_oracle(batch, q_len, seqlens):
+    wl = workloads.custom(batch, q_len, seqlens, seed=90 + sum(seqlens))
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg)
+    assert dec.check_status() == 0
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg), f"plan {batch}x{q_len} {seqlens}")
+
+
+@pytest.mark.parametrize("batch,q_len,seed", [(40, 1, 1), (147, 1, 2), (20, 4, 3)])
+def test_length_aware_plan_partitions_every_page_once(batch, q_len, seed):
+    """The tables: every page of every unit in exactly one CTA's run, runs of a
+    unit consecutive and in page order, no more CTAs than SMs, and the largest
+    run the smallest that fits (found here by brute force); then the output
+    against the (absorbed, pinned to the expanded) oracle."""
+    rng = np.random.default_rng(seed)
+    seqlens = [int(x) for x in rng.integers(200, 900, size=batch)]
+    seqlens[0] = 6000
+    wl = workloads.custom(batch, q_len, seqlens, seed=300 + seed)
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg)
+    assert dec.check_status() == 0
+    work, unit, groups = _plan_tables(dec)
+    C = dec.sms
+    w = [(seqlens[u // groups] + 63) // 64 for u in range(batch * groups)]
+    covered = 0
+    for u, (first, ns) in enumerate(unit):
+        assert ns >= 1
+        runs = work[first:first + ns]
+        assert (runs[:, 0] == u).all()
+        assert runs[0, 1] == 0 and runs[-1, 2] == w[u]
+        assert (runs[1:, 1] == runs[:-1, 2]).all() and (runs[:, 2] > runs[:, 1]).all()
+        covered += ns
+    assert covered <= C and (work[covered:, 0] == -1).all()
+    assert (unit[:, 0] == np.cumsum([0] + list(unit[:-1, 1]))).all()   # unit after unit
+    tot, wmax = sum(w), max(w)
+    T = next(t for t in range(max(1, -(-tot // C), min(2, wmax)), wmax + 2)
+             if sum(max(1, -(-x // t)) for x in w) <= C)
+    assert int((work[:covered, 2] - work[:covered, 1]).max()) == T
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, form="absorbed"), f"plan B={batch}")
+
+
+def test_length_aware_plan_is_deterministic():
+    wl = workloads.custom(3, 2, [4000, 90, 1500], seed=77)
+    cfg, _ = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    a, dec, st = gc.gpu_step(wl, inp, cfg)
+    q = inp.q.cuda().clone()
+    for _ in range(2):
+        b = dec.decode(cfg, st, q, xmla.xmla_softmax_scale(cfg)).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_decode_is_deterministic_and_split_count_only_changes_rounding():
     wl = workloads.custom(1, 1, [9000], seed=23)
     cfg, ocfg = gc.cfgs()
