@@ -40,6 +40,13 @@ struct AbsorbSmem {
   float part[16][kAbsorbRows][64];
 };
 
+// Row of q_ext holding head h of query row r (r = b*q_len + j): split, each
+// row group of 32 heads is followed by its low halves (part 1), q = hi + lo
+// with hi = bf16(q) and lo = bf16(q - hi); otherwise one bf16 row.
+__device__ __forceinline__ int64_t q_ext_row(int64_t r, int h, int part, int split) {
+  return split ? (2 * r + part) * kHeads + h : r * kHeads + h;
+}
+
 // Block (h, cb) of the absorb; cb == 8 is the rope block.  Every block waits
 // (griddepcontrol.wait) before reading q or seqlens: a preceding kernel may
 // have written them, and the split-K kernel relies on that wait (its producer
@@ -48,8 +55,8 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
                                                const __nv_bfloat16* __restrict__ W_UK,
                                                const int32_t* seqlens,
                                                __nv_bfloat16* __restrict__ q_ext, int rows,
-                                               int q_len, float qscale, const RopeTable& tab,
-                                               AbsorbSmem& sm) {
+                                               int q_len, int split, float qscale,
+                                               const RopeTable& tab, AbsorbSmem& sm) {
   auto& sq = sm.sq;
   auto& part = sm.part;
   const int t = threadIdx.x;
@@ -63,9 +70,16 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
       double y1, y2;
       rope_pair((double)__bfloat162float(x[i]), (double)__bfloat162float(x[i + kPairs]), pos, i,
                 tab, &y1, &y2);
-      __nv_bfloat16* o = q_ext + ((int64_t)r * kHeads + h) * kDRow + kDLatent;
-      o[i] = __double2bfloat16(y1 * (double)qscale);
-      o[i + kPairs] = __double2bfloat16(y2 * (double)qscale);
+      const double v1 = y1 * (double)qscale, v2 = y2 * (double)qscale;
+      const __nv_bfloat16 h1 = __double2bfloat16(v1), h2 = __double2bfloat16(v2);
+      __nv_bfloat16* o = q_ext + q_ext_row(r, h, 0, split) * kDRow + kDLatent;
+      o[i] = h1;
+      o[i + kPairs] = h2;
+      if (split) {  // the low halves, one block of 32 rows further
+        __nv_bfloat16* ol = q_ext + q_ext_row(r, h, 1, split) * kDRow + kDLatent;
+        ol[i] = __double2bfloat16(v1 - (double)__bfloat162float(h1));
+        ol[i + kPairs] = __double2bfloat16(v2 - (double)__bfloat162float(h2));
+      }
     }
     return;
   }
@@ -109,7 +123,12 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
       float s = 0.f;
 #pragma unroll
       for (int k = 0; k < 16; ++k) s += part[k][r][col];
-      q_ext[((int64_t)(r0 + r) * kHeads + h) * kDRow + cb * 64 + col] = __float2bfloat16_rn(s * qscale);
+      const float v = s * qscale;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      q_ext[q_ext_row(r0 + r, h, 0, split) * kDRow + cb * 64 + col] = hi;
+      if (split)
+        q_ext[q_ext_row(r0 + r, h, 1, split) * kDRow + cb * 64 + col] =
+            __float2bfloat16_rn(v - __bfloat162float(hi));
     }
   }
 }
@@ -221,8 +240,8 @@ static bool plan_ok(const WorkPlanArgs& plan) {
 template <bool kPlan>
 __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
-    __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, float qscale, const RopeTable tab,
-    const WorkPlanArgs plan) {
+    __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, int split, float qscale,
+    const RopeTable tab, const WorkPlanArgs plan) {
   __shared__ union {
     AbsorbSmem absorb;
     PlanSmem plan;
@@ -235,7 +254,7 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
     }
   }
   q_absorb_block(blockIdx.x % kHeads, blockIdx.x / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
-                 qscale, tab, sm.absorb);
+                 split, qscale, tab, sm.absorb);
 }
 
 // The first kernel of a decode step: the absorb blocks above, then the
@@ -248,8 +267,9 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
 template <bool kPlan>
 __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
-    __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, float qscale, const RopeTable q_tab,
-    const AppendArgs ap, const RopeTable k_tab, const ProduceArgs pa, const WorkPlanArgs plan) {
+    __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, int split, float qscale,
+    const RopeTable q_tab, const AppendArgs ap, const RopeTable k_tab, const ProduceArgs pa,
+    const WorkPlanArgs plan) {
   // one buffer for whichever role the block takes
   __shared__ union {
     AbsorbSmem absorb;
@@ -259,7 +279,7 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
   pdl_launch_dependents();
   if (blockIdx.x < kAbsorbBlocks) {
     q_absorb_block(blockIdx.x % kHeads, blockIdx.x / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
-                   qscale, q_tab, sm.absorb);
+                   split, qscale, q_tab, sm.absorb);
     return;
   }
   constexpr int kPlanBlocks = kPlan ? 1 : 0;
@@ -288,20 +308,20 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
 
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
-                            float qscale, const RopeTable& tab, const WorkPlanArgs* plan,
-                            cudaStream_t st) {
+                            int split, float qscale, const RopeTable& tab,
+                            const WorkPlanArgs* plan, cudaStream_t st) {
   if (plan != nullptr) {
     if (!plan_ok(*plan)) return cudaErrorInvalidValue;
     return launch_pdl(q_absorb_kernel<true>, dim3(kAbsorbBlocks + 1), dim3(kAbsorbThreads), 0, st,
-                      q, W_UK, seqlens, q_ext, rows, q_len, qscale, tab, *plan);
+                      q, W_UK, seqlens, q_ext, rows, q_len, split, qscale, tab, *plan);
   }
   return launch_pdl(q_absorb_kernel<false>, dim3(kAbsorbBlocks), dim3(kAbsorbThreads), 0, st, q,
-                    W_UK, seqlens, q_ext, rows, q_len, qscale, tab, WorkPlanArgs{});
+                    W_UK, seqlens, q_ext, rows, q_len, split, qscale, tab, WorkPlanArgs{});
 }
 
 cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                                  const int32_t* seqlens, __nv_bfloat16* q_ext, int rows,
-                                 int q_len, float qscale, const RopeTable& q_tab,
+                                 int q_len, int split, float qscale, const RopeTable& q_tab,
                                  const AppendArgs& ap, const RopeTable& k_tab,
                                  const ProduceArgs* pa, const WorkPlanArgs* plan,
                                  cudaStream_t st) {
@@ -314,13 +334,13 @@ cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_
     if (!plan_ok(*plan)) return cudaErrorInvalidValue;
     return launch_pdl(step_prologue_kernel<true>,
                       dim3((unsigned)(kAbsorbBlocks + 1 + prod_blocks + append_blocks)),
-                      dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, qscale,
-                      q_tab, ap, k_tab, p, *plan);
+                      dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, split,
+                      qscale, q_tab, ap, k_tab, p, *plan);
   }
   return launch_pdl(step_prologue_kernel<false>,
                     dim3((unsigned)(kAbsorbBlocks + prod_blocks + append_blocks)),
-                    dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, qscale,
-                    q_tab, ap, k_tab, p, WorkPlanArgs{});
+                    dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, split,
+                    qscale, q_tab, ap, k_tab, p, WorkPlanArgs{});
 }
 
 // ---------------------------------------------------------------- combine + W_UV

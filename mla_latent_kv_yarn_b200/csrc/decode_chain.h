@@ -42,11 +42,12 @@ struct WorkPlanArgs {
 };
 
 // q_ext[r, h] for rows r = b*q_len + j; qscale = softmax scale * log2 e.
-// plan (nullable): also compute the length-aware plan.
+// split: each query row as a hi and a lo bf16 row (the split-K kernel's
+// split_q layout).  plan (nullable): also compute the length-aware plan.
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
-                            float qscale, const RopeTable& tab, const WorkPlanArgs* plan,
-                            cudaStream_t st);
+                            int split, float qscale, const RopeTable& tab,
+                            const WorkPlanArgs* plan, cudaStream_t st);
 
 // The new tokens of a decode step, appended by step_prologue_kernel.
 struct AppendArgs {
@@ -69,7 +70,7 @@ struct AppendArgs {
 // (nullable) as for launch_q_absorb.
 cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                                  const int32_t* seqlens, __nv_bfloat16* q_ext, int rows,
-                                 int q_len, float qscale, const RopeTable& q_tab,
+                                 int q_len, int split, float qscale, const RopeTable& q_tab,
                                  const AppendArgs& ap, const RopeTable& k_tab,
                                  const ProduceArgs* pa, const WorkPlanArgs* plan,
                                  cudaStream_t st);

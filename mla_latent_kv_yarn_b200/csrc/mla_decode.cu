@@ -37,12 +37,21 @@ constexpr int kDecodeThreads = 32 * kSoftmaxWarp0 + kSoftmaxThreads;
 
 // ---------------------------------------------------------------- shared-memory plan
 
-template <int NR>
+// kSplitQ (32 rows only): q_ext comes as two bf16 rows per query row, hi and
+// lo = bf16(q - hi), so the QK product carries ~16 bits of the query: the
+// product runs with N = 64 (rows hi 0..31, lo 32..63) and the softmax adds
+// the two halves of S.  Otherwise q_ext is a single bf16 row each.  The split
+// needs 36 KB more of shared memory, taken from the page ring.
+template <int NR, bool kSplitQ_ = false>
 struct DecodeLayout {
   static_assert(NR == 32 || NR == 64, "rows per CTA");
-  static constexpr int kLatSlots = NR == 32 ? 9 : 7;   // 16 KB: latent dims 128m..128m+127 of a page
-  static constexpr int kRopeSlots = NR == 32 ? 4 : 2;  // 8 KB: rope dims of a page
-  static constexpr uint32_t kQChunk = NR * 128;        // one 64-column chunk of q_ext
+  static_assert(NR == 32 || !kSplitQ_, "the split query needs 32 rows per CTA");
+  static constexpr bool kSplitQ = kSplitQ_;
+  static constexpr int kQRows = kSplitQ ? 2 * NR : NR;  // B rows of the QK product
+  // 16 KB latent slots (dims 128m..128m+127 of a page) and 8 KB rope slots
+  static constexpr int kLatSlots = NR == 32 ? (kSplitQ ? 8 : 9) : 7;
+  static constexpr int kRopeSlots = NR == 32 && !kSplitQ ? 4 : 2;
+  static constexpr uint32_t kQChunk = kQRows * 128;    // one 64-column chunk of q_ext
   // P^T is stored MN-major: one row of NR bf16 per token, 64 B (64-byte swizzle)
   // for 32 rows or 128 B (128-byte swizzle) for 64 rows.
   static constexpr uint32_t kPRow = NR * 2;
@@ -78,10 +87,11 @@ struct DecodeLayout {
   static constexpr uint32_t kSmem = kBytes + 1024;  // slack for 1024-byte alignment
   static_assert(kSmem <= 232448, "shared memory per CTA");
   static_assert(kOffP % 1024 == 0 && kOffLat % 1024 == 0 && kOffRope % 1024 == 0, "alignment");
-  // tensor memory columns: O^T at [0, 4 NR), S^T buffers at [4 NR, 5 NR) and [5 NR, 6 NR)
+  // tensor memory columns: O^T at [0, 4 NR), S^T buffers of kSCols columns after it
   static constexpr uint32_t kColO = 0;
   static constexpr uint32_t kColS = 4 * NR;
-  static constexpr uint32_t kTmemCols = 6 * NR <= 256 ? 256 : 512;
+  static constexpr uint32_t kSCols = kQRows;  // columns of one S^T buffer
+  static constexpr uint32_t kTmemCols = 4 * NR + 2 * kSCols <= 256 ? 256 : 512;
 };
 
 
@@ -134,11 +144,11 @@ enum WorkMode : int {
   kWorkTable = 2,   // entry blockIdx of p.work_tab (written by the preceding kernel)
 };
 
-template <int NR, int kMode>
+template <int NR, int kMode, bool kSplitQ>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tmap_pool,
                       const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p) {
-  using L = DecodeLayout<NR>;
+  using L = DecodeLayout<NR, kSplitQ>;
   extern __shared__ uint8_t smem_raw[];
   uint32_t base = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
@@ -230,7 +240,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int jn = min(p.q_len - j0, NR / 32);
   const int nrows = jn * 32;
   const int n_pages = (int)max((int64_t)0, p_end - p_begin);
-  const int32_t qrow0 = (int32_t)(((int64_t)b * p.q_len + j0) * 32);
+  const int32_t qrow0 = (int32_t)(((int64_t)b * p.q_len + j0) * (L::kSplitQ ? 64 : 32));
   pdl_launch_dependents();
 
   if (warp == 0) {
@@ -324,7 +334,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // blocks in mbarrier try_wait, which suspends the thread instead of
     // spinning, so neither steals issue slots from the softmax warps.
     if (lane == 0 && n_pages > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(64, NR, false, false);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(64, L::kQRows, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, NR, true, true);
       // descriptor bases; operands are reached by adding (byte offset >> 4)
       const uint64_t d_lat_k = smem_desc_sw128(base + L::kOffLat, 16, 1024);     // page, K-major
@@ -345,7 +355,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             if (!(ok = wait(L::kBarSFree + sb, (uint32_t)(((i - 2) >> 1) & 1)))) break;
             tc_fence_after();
           }
-          const uint32_t t_s = tmem_base + L::kColS + sb * NR;
+          const uint32_t t_s = tmem_base + L::kColS + sb * L::kSCols;
           for (int m = 0; m < 4 && ok; ++m) {
             const int f = 4 * i + m;
             const int s = f % L::kLatSlots;
@@ -428,14 +438,26 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (named_bar_or(1, kSoftmaxThreads, !ok)) { ok = false; break; }
       tc_fence_after();
       float sv[kV];
+      if constexpr (L::kSplitQ) {
+        float lo[16];
+        tmem_ld16x64b_x16(t_lane + L::kColS + sb * L::kSCols, sv);
+        tmem_ld16x64b_x16(t_lane + L::kColS + sb * L::kSCols + NR, lo);
+        tc_wait_ld();
 #pragma unroll
-      for (int c = 0; c < NR / 32; ++c) {
-        float tmp[16];
-        tmem_ld16x64b_x16(t_lane + L::kColS + sb * NR + 32 * c, tmp);
+        for (int k = 0; k < 16; ++k) {
+          asm volatile("" : "+f"(sv[k]), "+f"(lo[k]));  // defined only after the wait
+          sv[k] += lo[k];
+        }
+      } else {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) sv[16 * c + k] = tmp[k];
+        for (int c = 0; c < NR / 32; ++c) {
+          float tmp[16];
+          tmem_ld16x64b_x16(t_lane + L::kColS + sb * NR + 32 * c, tmp);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) sv[16 * c + k] = tmp[k];
+        }
+        tc_wait_ld();
       }
-      tc_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(L::kBarSFree + sb));
 
@@ -604,40 +626,45 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
 }
 
-template <int NR, int kMode>
+template <int NR, int kMode, bool kSplitQ>
 static cudaError_t launch_decode(const CUtensorMap& tp, const CUtensorMap& tq, const DecodeParams& dp,
                                  int64_t items, cudaStream_t st) {
-  using L = DecodeLayout<NR>;
+  using L = DecodeLayout<NR, kSplitQ>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<NR, kMode>,
+    cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<NR, kMode, kSplitQ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  return launch_pdl(mla_decode_kernel<NR, kMode>, dim3((unsigned)items), dim3(kDecodeThreads),
-                    L::kSmem, st, tp, tq, dp);
+  return launch_pdl(mla_decode_kernel<NR, kMode, kSplitQ>, dim3((unsigned)items),
+                    dim3(kDecodeThreads), L::kSmem, st, tp, tq, dp);
 }
 
 
-cudaError_t launch_split_kv(int nr, const CUtensorMap& pool_map, const CUtensorMap& q_map,
-                            const DecodeParams& dp, int64_t items, cudaStream_t st) {
+template <int NR, bool kSplitQ>
+static cudaError_t launch_mode(int mode, const CUtensorMap& pool_map, const CUtensorMap& q_map,
+                               const DecodeParams& dp, int64_t items, cudaStream_t st) {
+  if (mode == kWorkTable)
+    return launch_decode<NR, kWorkTable, kSplitQ>(pool_map, q_map, dp, items, st);
+  if (mode == kWorkRanged)
+    return launch_decode<NR, kWorkRanged, kSplitQ>(pool_map, q_map, dp, items, st);
+  return launch_decode<NR, kWorkSplit, kSplitQ>(pool_map, q_map, dp, items, st);
+}
+
+cudaError_t launch_split_kv(int nr, bool split_q, const CUtensorMap& pool_map,
+                            const CUtensorMap& q_map, const DecodeParams& dp, int64_t items,
+                            cudaStream_t st) {
   const int mode = dp.work_tab != nullptr                          ? kWorkTable
                    : (dp.page_lo != 0 || dp.page_hi != INT64_MAX) ? kWorkRanged
                                                                   : kWorkSplit;
-  if (nr == 32) {
-    if (mode == kWorkTable) return launch_decode<32, kWorkTable>(pool_map, q_map, dp, items, st);
-    if (mode == kWorkRanged) return launch_decode<32, kWorkRanged>(pool_map, q_map, dp, items, st);
-    return launch_decode<32, kWorkSplit>(pool_map, q_map, dp, items, st);
-  }
-  if (nr == 64) {
-    if (mode == kWorkTable) return launch_decode<64, kWorkTable>(pool_map, q_map, dp, items, st);
-    if (mode == kWorkRanged) return launch_decode<64, kWorkRanged>(pool_map, q_map, dp, items, st);
-    return launch_decode<64, kWorkSplit>(pool_map, q_map, dp, items, st);
-  }
+  if (nr == 32)
+    return split_q ? launch_mode<32, true>(mode, pool_map, q_map, dp, items, st)
+                   : launch_mode<32, false>(mode, pool_map, q_map, dp, items, st);
+  if (nr == 64 && !split_q) return launch_mode<64, false>(mode, pool_map, q_map, dp, items, st);
   return cudaErrorInvalidValue;
 }
 

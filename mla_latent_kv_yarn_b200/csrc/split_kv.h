@@ -41,10 +41,12 @@ struct DecodeParams {
   const int4* work_tab;
 };
 
-// Split-K attention over `items` work items; nr = rows per CTA (32 or 64).
-// pool_map: 576-column rows of the cache pool, box 64 x 64; q_map: rows of
-// q_ext, box 64 x nr (both 128-byte swizzled).
-cudaError_t launch_split_kv(int nr, const CUtensorMap& pool_map, const CUtensorMap& q_map,
-                            const DecodeParams& dp, int64_t items, cudaStream_t st);
+// Split-K attention over `items` work items; nr = rows per CTA (32 or 64);
+// split_q (nr 32 only): q_ext holds a hi and a lo bf16 row per query row, 32
+// heads of hi then 32 of lo per query.  pool_map: 576-column rows of the cache
+// pool, box 64 x 64; q_map: rows of q_ext, box 64 x 64 (both 128-byte swizzled).
+cudaError_t launch_split_kv(int nr, bool split_q, const CUtensorMap& pool_map,
+                            const CUtensorMap& q_map, const DecodeParams& dp, int64_t items,
+                            cudaStream_t st);
 
 }  // namespace xmla

@@ -30,7 +30,16 @@ __global__ void wait_timeout_selftest_kernel(int32_t* status, uint64_t limit_ns)
 
 // ---------------------------------------------------------------- host plan
 
+// Up to this many tokens per sequence the query goes to the QK product as a hi
+// and a lo bf16 part (the split-K kernel's split_q layout, one query of 32
+// heads per CTA).  A short context is dominated by a few tokens and its output
+// is large (|out| up to ~4), so the ~2^-9 relative score error of a single
+// bf16 query reaches the 1e-2 output bound there; the split costs a shallower
+// page ring, which only long contexts, dominated by streaming, would notice.
+constexpr int64_t kSplitQMaxSeqlen = 4096;
+
 struct Plan {
+  bool split;   // hi/lo query (split_q)
   int nr;       // rows per CTA (32 or 64)
   int groups;   // row groups per sequence
   int nsplit;   // KV splits per (sequence, group) when every sequence has max_seqlen tokens
@@ -53,7 +62,8 @@ static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_
       max_seqlen > (int64_t)0x7fffffff - kPage || num_sms < 1 || num_splits < 0 || span_pages < 0)
     return false;
   Plan P;
-  P.nr = q_len == 1 ? 32 : 64;
+  P.split = max_seqlen <= kSplitQMaxSeqlen;
+  P.nr = P.split || q_len == 1 ? 32 : 64;
   P.groups = (q_len * 32 + P.nr - 1) / P.nr;
   int64_t max_pages = (max_seqlen + kPage - 1) / kPage;
   if (span_pages > 0 && span_pages < max_pages) max_pages = span_pages;
@@ -74,7 +84,8 @@ static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_
             num_sms <= kMaxPlanCtas;
   P.items = P.table ? num_sms : units * P.nsplit;
   if (P.items > 0x7fffffff) return false;
-  const size_t qext = (size_t)B * q_len * kHeads * kDRow * 2;
+  // q_ext: bf16 rows of 576; split, each row also has its low half
+  const size_t qext = (size_t)B * q_len * kHeads * kDRow * 2 * (P.split ? 2 : 1);
   P.off_qext = 0;
   P.off_o = align_up(qext, 1024);
   P.off_ml = align_up(P.off_o + (size_t)P.items * P.nr * kDLatent * 4, 1024);
@@ -188,7 +199,11 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
 
   CUtensorMap tmap_pool, tmap_q;
   if (!encode_rows576(&tmap_pool, pool, (uint64_t)num_blocks * kPage, kPage)) return XMLA_ERR_CUDA;
-  if (!encode_rows576(&tmap_q, q_ext, (uint64_t)rows * kHeads, (uint32_t)P.nr)) return XMLA_ERR_CUDA;
+  // the QK product's B tile: 64 rows (32 heads hi then lo when split, 32 heads of one query
+  // at 32 rows per CTA, else 2 queries x 32 heads)
+  if (!encode_rows576(&tmap_q, q_ext, (uint64_t)rows * kHeads * (P.split ? 2 : 1),
+                      P.split || P.nr == 64 ? 64 : 32))
+    return XMLA_ERR_CUDA;
 
   const float qscale = softmax_scale * kLog2e;
   const RopeTable tab = make_rope_table(cfg);
@@ -208,10 +223,11 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   const cudaError_t e0 =
       ap != nullptr
           ? launch_step_prologue((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
-                                 rows, q_len, qscale, tab, *ap, tab, pa,
+                                 rows, q_len, P.split ? 1 : 0, qscale, tab, *ap, tab, pa,
                                  P.table ? &plan : nullptr, st)
           : launch_q_absorb((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
-                            rows, q_len, qscale, tab, P.table ? &plan : nullptr, st);
+                            rows, q_len, P.split ? 1 : 0, qscale, tab,
+                            P.table ? &plan : nullptr, st);
   if (e0 != cudaSuccess) return XMLA_ERR_CUDA;
 
   DecodeParams dp;
@@ -232,7 +248,8 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   dp.page_hi = page_hi;
   dp.work_tab = P.table ? plan.work_tab : nullptr;
   if (record_event(attn_start, st) != cudaSuccess) return XMLA_ERR_CUDA;
-  if (launch_split_kv(P.nr, tmap_pool, tmap_q, dp, P.items, st) != cudaSuccess) return XMLA_ERR_CUDA;
+  if (launch_split_kv(P.nr, P.split, tmap_pool, tmap_q, dp, P.items, st) != cudaSuccess)
+    return XMLA_ERR_CUDA;
   if (record_event(attn_stop, st) != cudaSuccess) return XMLA_ERR_CUDA;
   if (shard_partial != nullptr) {
     const cudaError_t em = launch_merge_splits(dp.part_o, dp.part_ml, shard_partial, rows, q_len,
