@@ -42,15 +42,22 @@ constexpr int kDecodeThreads = 32 * kSoftmaxWarp0 + kSoftmaxThreads;
 // product runs with N = 64 (rows hi 0..31, lo 32..63) and the softmax adds
 // the two halves of S.  Otherwise q_ext is a single bf16 row each.  The split
 // needs 36 KB more of shared memory, taken from the page ring.
+// P^T buffers with 64 rows per CTA (two where shared memory allows)
+constexpr int kPBufs64 = 2;
+
 template <int NR, bool kSplitQ_ = false>
 struct DecodeLayout {
   static_assert(NR == 32 || NR == 64, "rows per CTA");
   static_assert(NR == 32 || !kSplitQ_, "the split query needs 32 rows per CTA");
   static constexpr bool kSplitQ = kSplitQ_;
   static constexpr int kQRows = kSplitQ ? 2 * NR : NR;  // B rows of the QK product
-  // 16 KB latent slots (dims 128m..128m+127 of a page) and 8 KB rope slots
-  static constexpr int kLatSlots = NR == 32 ? (kSplitQ ? 8 : 9) : 7;
-  static constexpr int kRopeSlots = NR == 32 && !kSplitQ ? 4 : 2;
+  // 16 KB latent slots (dims 128m..128m+127 of a page) and 8 KB rope slots.
+  // At least two pages of latent slots, so page i + 1 never waits for a slot
+  // of page i (whose PV needs page i's softmax); with 64 rows that leaves room
+  // for one rope slot, which the QK product then reads first and frees early.
+  static constexpr int kLatSlots = NR == 32 && !kSplitQ ? 9 : 8;
+  static constexpr int kRopeSlots = NR == 32 ? (kSplitQ ? 2 : 4) : 1;
+  static constexpr bool kRopeFirst = kRopeSlots == 1;
   static constexpr uint32_t kQChunk = kQRows * 128;    // one 64-column chunk of q_ext
   // P^T is stored MN-major: one row of NR bf16 per token, 64 B (64-byte swizzle)
   // for 32 rows or 128 B (128-byte swizzle) for 64 rows.
@@ -62,7 +69,8 @@ struct DecodeLayout {
   static constexpr uint32_t kRopeBytes = 8192;
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffP = kOffQ + 9 * kQChunk;
-  static constexpr uint32_t kOffLat = kOffP + 2 * kPBytes;
+  static constexpr int kPBufs = NR == 32 ? 2 : kPBufs64;
+  static constexpr uint32_t kOffLat = kOffP + kPBufs * kPBytes;
   static constexpr uint32_t kOffRope = kOffLat + kLatSlots * kLatBytes;
   static constexpr uint32_t kOffBars = kOffRope + kRopeSlots * kRopeBytes;
   // barrier indices
@@ -282,6 +290,21 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           blk = (int32_t)p.num_blocks;  // past the end: the tensor copy reads zeros
         }
         const int32_t y = blk * kPage;
+        auto issue_rope = [&]() {
+          if (!mbar_wait(bar(L::kBarRopeEmpty + ri), rph ^ 1u, abort_flag, p.status,
+                         p.wait_limit_ns))
+            return false;
+          mbar_arrive_expect_tx(bar(L::kBarRopeFull + ri), L::kRopeBytes);
+          tma_load_2d_hint(base + L::kOffRope + ri * L::kRopeBytes, &tmap_pool, kDLatent, y,
+                           bar(L::kBarRopeFull + ri), stream_policy);
+          ++rope_issued;
+          if (++ri == L::kRopeSlots) { ri = 0; rph ^= 1u; }
+          return true;
+        };
+        // the chunk the QK product reads first is requested first
+        if constexpr (L::kRopeFirst) {
+          if (!(ok = issue_rope())) break;
+        }
         for (int m = 0; m < 4; ++m) {
           if (!mbar_wait(bar(L::kBarLatEmpty + li), lph ^ 1u, abort_flag, p.status,
                          p.wait_limit_ns)) {
@@ -297,16 +320,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           if (++li == L::kLatSlots) { li = 0; lph ^= 1u; }
         }
         if (!ok) break;
-        if (!mbar_wait(bar(L::kBarRopeEmpty + ri), rph ^ 1u, abort_flag, p.status,
-                       p.wait_limit_ns)) {
-          ok = false;
-          break;
+        if constexpr (!L::kRopeFirst) {
+          if (!(ok = issue_rope())) break;
         }
-        mbar_arrive_expect_tx(bar(L::kBarRopeFull + ri), L::kRopeBytes);
-        tma_load_2d_hint(base + L::kOffRope + ri * L::kRopeBytes, &tmap_pool, kDLatent, y,
-                         bar(L::kBarRopeFull + ri), stream_policy);
-        ++rope_issued;
-        if (++ri == L::kRopeSlots) { ri = 0; rph ^= 1u; }
       }
       // Every copy issued must land before the CTA may exit: wait for the last
       // phase armed on each slot (immediate when the consumer already saw it).
@@ -356,6 +372,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             tc_fence_after();
           }
           const uint32_t t_s = tmem_base + L::kColS + sb * L::kSCols;
+          const int r = i % L::kRopeSlots;
+          if constexpr (L::kRopeFirst) {
+            // the rope chunk first: its single slot is refilled for the next page
+            // while this page's latent chunks go through
+            if (!(ok = wait(L::kBarRopeFull + r, (uint32_t)((i / L::kRopeSlots) & 1)))) break;
+            tc_fence_after();
+            const uint64_t ar = d_rope_k + ((r * L::kRopeBytes) >> 4);
+            const uint64_t bq = d_q + ((8 * L::kQChunk) >> 4);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc_mma_bf16(t_s, ar + ((k * 32) >> 4), bq + ((k * 32) >> 4), idesc_qk, k != 0 ? 1u : 0u);
+            tc_commit(bar(L::kBarRopeEmpty + r));
+          }
           for (int m = 0; m < 4 && ok; ++m) {
             const int f = 4 * i + m;
             const int s = f % L::kLatSlots;
@@ -368,26 +397,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 tc_mma_bf16(t_s, a0 + ((half * 8192 + k * 32) >> 4), bq + ((k * 32) >> 4), idesc_qk,
-                            (m | half | k) != 0 ? 1u : 0u);
+                            (L::kRopeFirst || (m | half | k) != 0) ? 1u : 0u);
             }
           }
           if (!ok) break;
-          const int r = i % L::kRopeSlots;
-          if (!(ok = wait(L::kBarRopeFull + r, (uint32_t)((i / L::kRopeSlots) & 1)))) break;
-          tc_fence_after();
-          const uint64_t ar = d_rope_k + ((r * L::kRopeBytes) >> 4);
-          const uint64_t bq = d_q + ((8 * L::kQChunk) >> 4);
+          if constexpr (!L::kRopeFirst) {
+            if (!(ok = wait(L::kBarRopeFull + r, (uint32_t)((i / L::kRopeSlots) & 1)))) break;
+            tc_fence_after();
+            const uint64_t ar = d_rope_k + ((r * L::kRopeBytes) >> 4);
+            const uint64_t bq = d_q + ((8 * L::kQChunk) >> 4);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_bf16(t_s, ar + ((k * 32) >> 4), bq + ((k * 32) >> 4), idesc_qk, 1u);
+            for (int k = 0; k < 4; ++k)
+              tc_mma_bf16(t_s, ar + ((k * 32) >> 4), bq + ((k * 32) >> 4), idesc_qk, 1u);
+          }
           tc_commit(bar(L::kBarSFull + sb));
-          tc_commit(bar(L::kBarRopeEmpty + r));
+          if constexpr (!L::kRopeFirst) tc_commit(bar(L::kBarRopeEmpty + r));
         }
       } else {
         for (int i = 0; i < n_pages && ok; ++i) {
           if (!(ok = wait(L::kBarPFull + (i & 1), (uint32_t)((i >> 1) & 1)))) break;
           tc_fence_after();
-          const uint64_t bp = d_p + (((i & 1) * L::kPBytes) >> 4);
+          const uint64_t bp = d_p + (((i % L::kPBufs) * L::kPBytes) >> 4);
 #pragma unroll 1
           for (int m = 0; m < 4; ++m) {
             const int s = (4 * i + m) % L::kLatSlots;
@@ -518,9 +548,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #pragma unroll
         for (int j = 0; j < kV; ++j) mr[j] = m_used[pr + 2 * j];
       }
-      if (i >= 2) {
-        // P buffer (i & 1) is free once the PV of page i - 2 has completed
-        const int pi = i - 2;
+      if (i >= L::kPBufs) {
+        // P buffer i % kPBufs is free once the PV of page i - kPBufs has completed
+        const int pi = i - L::kPBufs;
         const bool okw = mbar_wait(bar(L::kBarPvDone + (pi & 1)), (uint32_t)((pi >> 1) & 1),
                                    abort_flag, p.status, p.wait_limit_ns);
         if (named_bar_or(1, kSoftmaxThreads, !okw)) { ok = false; break; }
@@ -558,7 +588,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const float rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
         w[k] = pr == 0 ? pack_bf16x2(own, rcv) : pack_bf16x2(rcv, own);
       }
-      uint8_t* prow = smem + L::kOffP + sb * L::kPBytes + tok * L::kPRow;
+      uint8_t* prow = smem + L::kOffP + (i % L::kPBufs) * L::kPBytes + tok * L::kPRow;
 #pragma unroll
       for (int u = 0; u < kH / 4; ++u) {
         const int unit = pr * (kH / 4) + u;
