@@ -51,19 +51,24 @@ __device__ __forceinline__ int64_t q_ext_row(int64_t r, int h, int part, int spl
 // (griddepcontrol.wait) before reading q or seqlens: a preceding kernel may
 // have written them, and the split-K kernel relies on that wait (its producer
 // reads cache rows appended by the kernel before this one).
+template <bool kRowBlocks>
 __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat16* q,
                                                const __nv_bfloat16* __restrict__ W_UK,
                                                const int32_t* seqlens,
                                                __nv_bfloat16* __restrict__ q_ext, int rows,
                                                int q_len, int split, float qscale,
-                                               const RopeTable& tab, AbsorbSmem& sm) {
+                                               const RopeTable& tab, AbsorbSmem& sm,
+                                               int row_lo_arg, int row_hi_arg) {
+  // kRowBlocks: rows [row_lo, row_hi) of the query; otherwise all rows
+  const int row_lo = kRowBlocks ? row_lo_arg : 0;
+  const int row_hi = kRowBlocks ? row_hi_arg : rows;
   auto& sq = sm.sq;
   auto& part = sm.part;
   const int t = threadIdx.x;
   if (cb == kDLatent / 64) {
     pdl_wait();
     constexpr int kPairs = kDRope / 2;
-    for (int e = t; e < rows * kPairs; e += kAbsorbThreads) {
+    for (int e = row_lo * kPairs + t; e < row_hi * kPairs; e += kAbsorbThreads) {
       const int r = e / kPairs, i = e % kPairs;
       const int64_t pos = (int64_t)seqlens[r / q_len] - q_len + (r % q_len);
       const __nv_bfloat16* x = q + ((int64_t)r * kHeads + h) * kDQ + kDNope;
@@ -98,8 +103,8 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
     }
   }
   pdl_wait();
-  for (int r0 = 0; r0 < rows; r0 += kAbsorbRows) {
-    const int nr = min(kAbsorbRows, rows - r0);
+  for (int r0 = row_lo; r0 < row_hi; r0 += kAbsorbRows) {
+    const int nr = min(kAbsorbRows, row_hi - r0);
     __syncthreads();
     for (int e = t; e < nr * kDNope; e += kAbsorbThreads) {
       const int r = e / kDNope, d = e % kDNope;
@@ -236,8 +241,10 @@ static bool plan_ok(const WorkPlanArgs& plan) {
 
 // q and seqlens carry no __restrict__ so that their loads stay behind the
 // griddepcontrol.wait (a preceding kernel may have written them).
-// kPlan: block kAbsorbBlocks computes the length-aware plan (batch > 1).
-template <bool kPlan>
+// kPlan: one more block computes the length-aware plan (batch > 1).
+// kRowBlocks: every absorb block takes kAbsorbRows query rows (more rows than
+// that: kAbsorbBlocks blocks per kAbsorbRows rows); else all rows.
+template <bool kPlan, bool kRowBlocks>
 __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
     __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, int split, float qscale,
@@ -247,14 +254,19 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
     PlanSmem plan;
   } sm;
   pdl_launch_dependents();
+  const int absorb_blocks =
+      kRowBlocks ? kAbsorbBlocks * ((rows + kAbsorbRows - 1) / kAbsorbRows) : kAbsorbBlocks;
   if constexpr (kPlan) {
-    if (blockIdx.x == kAbsorbBlocks) {
+    if (blockIdx.x == absorb_blocks) {
       work_plan_block(plan, sm.plan);
       return;
     }
   }
-  q_absorb_block(blockIdx.x % kHeads, blockIdx.x / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
-                 split, qscale, tab, sm.absorb);
+  const int hb = kRowBlocks ? blockIdx.x % kAbsorbBlocks : blockIdx.x;
+  const int r_lo = kRowBlocks ? (blockIdx.x / kAbsorbBlocks) * kAbsorbRows : 0;
+  const int r_hi = kRowBlocks ? min(rows, r_lo + kAbsorbRows) : rows;
+  q_absorb_block<kRowBlocks>(hb % kHeads, hb / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
+                             split, qscale, tab, sm.absorb, r_lo, r_hi);
 }
 
 // The first kernel of a decode step: the absorb blocks above, then the
@@ -262,9 +274,9 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
 // warps each; pa.T == 0 otherwise), then blocks that append the step's ready
 // cache rows (one thread per 16-byte piece).  All of them only wait for the
 // kernel launched before this one, so they run side by side.
-// kPlan: block kAbsorbBlocks computes the length-aware plan (batch > 1); the
-// producer and append blocks follow it.
-template <bool kPlan>
+// kPlan: one more block computes the length-aware plan (batch > 1); the
+// producer and append blocks follow it.  kRowBlocks as for q_absorb_kernel.
+template <bool kPlan, bool kRowBlocks>
 __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
     __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, int split, float qscale,
@@ -277,21 +289,26 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
     PlanSmem plan;
   } sm;
   pdl_launch_dependents();
-  if (blockIdx.x < kAbsorbBlocks) {
-    q_absorb_block(blockIdx.x % kHeads, blockIdx.x / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
-                   split, qscale, q_tab, sm.absorb);
+  const int absorb_blocks =
+      kRowBlocks ? kAbsorbBlocks * ((rows + kAbsorbRows - 1) / kAbsorbRows) : kAbsorbBlocks;
+  if (blockIdx.x < absorb_blocks) {
+    const int hb = kRowBlocks ? blockIdx.x % kAbsorbBlocks : blockIdx.x;
+    const int r_lo = kRowBlocks ? (blockIdx.x / kAbsorbBlocks) * kAbsorbRows : 0;
+    const int r_hi = kRowBlocks ? min(rows, r_lo + kAbsorbRows) : rows;
+    q_absorb_block<kRowBlocks>(hb % kHeads, hb / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
+                               split, qscale, q_tab, sm.absorb, r_lo, r_hi);
     return;
   }
   constexpr int kPlanBlocks = kPlan ? 1 : 0;
   if constexpr (kPlan) {
-    if (blockIdx.x == kAbsorbBlocks) {
+    if (blockIdx.x == absorb_blocks) {
       work_plan_block(plan, sm.plan);
       return;
     }
   }
   const int prod_blocks = pa.T > 0 ? kProdBlocks : 0;
-  if (blockIdx.x < kAbsorbBlocks + kPlanBlocks + prod_blocks) {
-    produce_block<kAbsorbThreads / 32>(blockIdx.x - kAbsorbBlocks - kPlanBlocks, threadIdx.x, pa,
+  if (blockIdx.x < absorb_blocks + kPlanBlocks + prod_blocks) {
+    produce_block<kAbsorbThreads / 32>(blockIdx.x - absorb_blocks - kPlanBlocks, threadIdx.x, pa,
                                        k_tab, sm.produce, [] { __syncthreads(); },
                                        [] { pdl_wait(); });
     return;
@@ -299,7 +316,7 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
   pdl_wait();
   const int64_t total = ap.T * kRowPieces;
   const int64_t idx =
-      (int64_t)(blockIdx.x - kAbsorbBlocks - kPlanBlocks - prod_blocks) * kAbsorbThreads +
+      (int64_t)(blockIdx.x - absorb_blocks - kPlanBlocks - prod_blocks) * kAbsorbThreads +
       threadIdx.x;
   if (idx < total)
     append_piece(idx, ap.pool, ap.num_blocks, ap.block_table, ap.max_blocks, ap.batch, ap.seq_ids,
@@ -310,13 +327,18 @@ cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
                             int split, float qscale, const RopeTable& tab,
                             const WorkPlanArgs* plan, cudaStream_t st) {
+  const bool rb = rows > kAbsorbRows;
+  const unsigned absorb_blocks =
+      rb ? kAbsorbBlocks * (unsigned)((rows + kAbsorbRows - 1) / kAbsorbRows) : kAbsorbBlocks;
   if (plan != nullptr) {
     if (!plan_ok(*plan)) return cudaErrorInvalidValue;
-    return launch_pdl(q_absorb_kernel<true>, dim3(kAbsorbBlocks + 1), dim3(kAbsorbThreads), 0, st,
-                      q, W_UK, seqlens, q_ext, rows, q_len, split, qscale, tab, *plan);
+    return launch_pdl(rb ? q_absorb_kernel<true, true> : q_absorb_kernel<true, false>,
+                      dim3(absorb_blocks + 1), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens,
+                      q_ext, rows, q_len, split, qscale, tab, *plan);
   }
-  return launch_pdl(q_absorb_kernel<false>, dim3(kAbsorbBlocks), dim3(kAbsorbThreads), 0, st, q,
-                    W_UK, seqlens, q_ext, rows, q_len, split, qscale, tab, WorkPlanArgs{});
+  return launch_pdl(rb ? q_absorb_kernel<false, true> : q_absorb_kernel<false, false>,
+                    dim3(absorb_blocks), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext,
+                    rows, q_len, split, qscale, tab, WorkPlanArgs{});
 }
 
 cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
@@ -330,15 +352,18 @@ cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_
   ProduceArgs none{};
   const ProduceArgs& p = pa != nullptr ? *pa : none;
   const int64_t prod_blocks = p.T > 0 ? kProdBlocks : 0;
+  const bool rb = rows > kAbsorbRows;
+  const int64_t absorb_blocks =
+      rb ? (int64_t)kAbsorbBlocks * ((rows + kAbsorbRows - 1) / kAbsorbRows) : kAbsorbBlocks;
   if (plan != nullptr) {
     if (!plan_ok(*plan)) return cudaErrorInvalidValue;
-    return launch_pdl(step_prologue_kernel<true>,
-                      dim3((unsigned)(kAbsorbBlocks + 1 + prod_blocks + append_blocks)),
+    return launch_pdl(rb ? step_prologue_kernel<true, true> : step_prologue_kernel<true, false>,
+                      dim3((unsigned)(absorb_blocks + 1 + prod_blocks + append_blocks)),
                       dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, split,
                       qscale, q_tab, ap, k_tab, p, *plan);
   }
-  return launch_pdl(step_prologue_kernel<false>,
-                    dim3((unsigned)(kAbsorbBlocks + prod_blocks + append_blocks)),
+  return launch_pdl(rb ? step_prologue_kernel<false, true> : step_prologue_kernel<false, false>,
+                    dim3((unsigned)(absorb_blocks + prod_blocks + append_blocks)),
                     dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, split,
                     qscale, q_tab, ap, k_tab, p, WorkPlanArgs{});
 }
@@ -452,8 +477,10 @@ __device__ __forceinline__ void merge_group(const float* po, const float2* pml, 
 // rows apart, as the split-K kernel writes them.  kTable: the splits of a
 // (sequence, row group) unit are those unit_tab gives (length-aware plan),
 // read after the wait; otherwise nsplit per unit, unit after unit.
-template <bool kStrided, bool kTable>
-__global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThreads, 3)
+// kMinBlocks: CTAs per SM the kernel is compiled for: 3, or 4 when there are
+// more than kCombineRows rows, so that 512 CTAs (32 rows) still run in one wave.
+template <bool kStrided, bool kTable, int kMinBlocks>
+__global__ void __cluster_dims__(kSlices, 1, 1) __launch_bounds__(kCombineThreads, kMinBlocks)
     combine_uv_kernel(const float* part_o, const float* part_ml,
                       const __nv_bfloat16* __restrict__ W_UV, __nv_bfloat16* __restrict__ out,
                       int rows, int q_len, int groups, int nsplit, int rows_per_cta,
@@ -595,17 +622,18 @@ cudaError_t launch_combine(const float* part_o, const float* part_ml, const __nv
   const dim3 grid(kSlices * kHeads * chunks);
   const bool strided = o_stride != 0 || ml_stride != 0;
   if (strided && unit_tab != nullptr) return cudaErrorInvalidValue;
+  const bool wide = rows > kCombineRows;
   if (unit_tab != nullptr)
-    return launch_pdl(combine_uv_kernel<false, true>, grid, dim3(kCombineThreads), 0, st, part_o,
-                      part_ml, W_UV, out, rows, q_len, groups, nsplit, rows_per_cta, (int64_t)0,
-                      (int64_t)0, unit_tab);
+    return launch_pdl(wide ? combine_uv_kernel<false, true, 4> : combine_uv_kernel<false, true, 3>,
+                      grid, dim3(kCombineThreads), 0, st, part_o, part_ml, W_UV, out, rows, q_len,
+                      groups, nsplit, rows_per_cta, (int64_t)0, (int64_t)0, unit_tab);
   if (!strided)
-    return launch_pdl(combine_uv_kernel<false, false>, grid, dim3(kCombineThreads), 0, st, part_o,
-                      part_ml, W_UV, out, rows, q_len, groups, nsplit, rows_per_cta, (int64_t)0,
-                      (int64_t)0, unit_tab);
-  return launch_pdl(combine_uv_kernel<true, false>, grid, dim3(kCombineThreads), 0, st, part_o,
-                    part_ml, W_UV, out, rows, q_len, groups, nsplit, rows_per_cta, o_stride,
-                    ml_stride, unit_tab);
+    return launch_pdl(wide ? combine_uv_kernel<false, false, 4> : combine_uv_kernel<false, false, 3>,
+                      grid, dim3(kCombineThreads), 0, st, part_o, part_ml, W_UV, out, rows, q_len,
+                      groups, nsplit, rows_per_cta, (int64_t)0, (int64_t)0, unit_tab);
+  return launch_pdl(wide ? combine_uv_kernel<true, false, 4> : combine_uv_kernel<true, false, 3>,
+                    grid, dim3(kCombineThreads), 0, st, part_o, part_ml, W_UV, out, rows, q_len,
+                    groups, nsplit, rows_per_cta, o_stride, ml_stride, unit_tab);
 }
 
 // ---------------------------------------------------------------- merge of one shard's splits
