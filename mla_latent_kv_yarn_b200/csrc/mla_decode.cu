@@ -569,24 +569,28 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           dst[u] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      // probabilities (bf16-rounded, also summed in that precision)
-      float pb[kV];
+      // probabilities, rounded to bf16 in pairs (one conversion for rows j and
+      // kH + j of this thread) and summed in that precision (the rounded values
+      // are read back from the bits)
+      uint32_t x[kH];
 #pragma unroll
-      for (int j = 0; j < kV; ++j) {
-        const float pf = sv[j] == -INFINITY ? 0.f : ex2(sv[j] - mr[j]);
-        pb[j] = __bfloat162float(__float2bfloat16_rn(pf));
-        l_part[j] += pb[j];
+      for (int k = 0; k < kH; ++k) {
+        const float p0 = sv[k] == -INFINITY ? 0.f : ex2(sv[k] - mr[k]);
+        const float p1 = sv[kH + k] == -INFINITY ? 0.f : ex2(sv[kH + k] - mr[kH + k]);
+        x[k] = pack_bf16x2(p0, p1);
+        l_part[k] += __uint_as_float(x[k] << 16);
+        l_part[kH + k] += __uint_as_float(x[k] & 0xffff0000u);
       }
-      // The thread pair (t, t^2) holds the two row parities of one token: swap
-      // halves so that each owns kV consecutive rows, then write its 16-byte
-      // units of the token's P^T row (MN-major, swizzled as the PV operand).
+      // The thread pair (t, t^2) holds the two row parities of one token: each
+      // takes the partner's half it needs, so that it owns kV consecutive rows
+      // (pr 0: rows 0..kV-1 from the low halves, pr 1: the rest from the high
+      // halves), then writes its 16-byte units of the token's P^T row
+      // (MN-major, swizzled as the PV operand).
       uint32_t w[kH];
 #pragma unroll
       for (int k = 0; k < kH; ++k) {
-        const float own = pr == 0 ? pb[k] : pb[kH + k];
-        const float snd = pr == 0 ? pb[kH + k] : pb[k];
-        const float rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
-        w[k] = pr == 0 ? pack_bf16x2(own, rcv) : pack_bf16x2(rcv, own);
+        const uint32_t rcv = __shfl_xor_sync(0xffffffffu, x[k], 2);
+        w[k] = pr == 0 ? __byte_perm(x[k], rcv, 0x5410) : __byte_perm(rcv, x[k], 0x7632);
       }
       uint8_t* prow = smem + L::kOffP + (i % L::kPBufs) * L::kPBytes + tok * L::kPRow;
 #pragma unroll
