@@ -463,9 +463,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     bool ok = true;
     for (int i = 0; i < n_pages; ++i) {
       const int sb = i & 1;
+      // A timed-out wait is acted on at the page's one block-wide vote below,
+      // where all softmax threads leave together.
       ok = mbar_wait(bar(L::kBarSFull + sb), (uint32_t)((i >> 1) & 1), abort_flag, p.status,
                      p.wait_limit_ns);
-      if (named_bar_or(1, kSoftmaxThreads, !ok)) { ok = false; break; }
       tc_fence_after();
       float sv[kV];
       if constexpr (L::kSplitQ) {
@@ -500,7 +501,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         sv[j] = vis ? sv[j] : -INFINITY;
         exceed |= sv[j] > mr[j] + kLazyMax;
       }
-      if (named_bar_or(1, kSoftmaxThreads, exceed)) {
+      // P buffer i % kPBufs is free once the PV of page i - kPBufs has completed
+      bool okp = true;
+      if (i >= L::kPBufs) {
+        const int pi = i - L::kPBufs;
+        okp = mbar_wait(bar(L::kBarPvDone + (pi & 1)), (uint32_t)((pi >> 1) & 1), abort_flag,
+                        p.status, p.wait_limit_ns);
+      }
+      // one vote per page: nothing to do unless a row's maximum moved or a wait timed out
+      if (named_bar_or(1, kSoftmaxThreads, exceed || !ok || !okp)) {
+        if (named_bar_or(1, kSoftmaxThreads, !ok || !okp)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < NR / 32; ++c) {
           float tmp[16];
@@ -547,13 +557,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         named_bar_sync(1, kSoftmaxThreads);
 #pragma unroll
         for (int j = 0; j < kV; ++j) mr[j] = m_used[pr + 2 * j];
-      }
-      if (i >= L::kPBufs) {
-        // P buffer i % kPBufs is free once the PV of page i - kPBufs has completed
-        const int pi = i - L::kPBufs;
-        const bool okw = mbar_wait(bar(L::kBarPvDone + (pi & 1)), (uint32_t)((pi >> 1) & 1),
-                                   abort_flag, p.status, p.wait_limit_ns);
-        if (named_bar_or(1, kSoftmaxThreads, !okw)) { ok = false; break; }
       }
       if (p_begin + i == npages - 1 && (seqlen % kPage) != 0) {
         // Rows past the sequence end in its last block hold whatever the pool
