@@ -492,14 +492,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(L::kBarSFree + sb));
 
-      const int64_t tpos = (p_begin + i) * kPage + tok;
       bool exceed = false;
+      if ((p_begin + i + 1) * kPage - 1 <= qpos0 && jn == NR / 32) {
+        // every token of the page is visible to every row: no mask
 #pragma unroll
-      for (int j = 0; j < kV; ++j) {
-        const int jr = j >> 4;  // query of row pr + 2j within this CTA
-        const bool vis = jr < jn && tpos <= qpos0 + jr;
-        sv[j] = vis ? sv[j] : -INFINITY;
-        exceed |= sv[j] > mr[j] + kLazyMax;
+        for (int j = 0; j < kV; ++j) exceed |= sv[j] > mr[j] + kLazyMax;
+      } else {
+        const int64_t tpos = (p_begin + i) * kPage + tok;
+#pragma unroll
+        for (int j = 0; j < kV; ++j) {
+          const int jr = j >> 4;  // query of row pr + 2j within this CTA
+          const bool vis = jr < jn && tpos <= qpos0 + jr;
+          sv[j] = vis ? sv[j] : -INFINITY;
+          exceed |= sv[j] > mr[j] + kLazyMax;
+        }
       }
       // P buffer i % kPBufs is free once the PV of page i - kPBufs has completed
       bool okp = true;
