@@ -277,6 +277,27 @@ def traffic_record(kernel_src_sha: str, name: str):
     return None
 
 
+def roofline_line(wl, achieved, peak, peak_kind, traffic, cache_bytes, kernel_ms, flops, tpeak,
+                  tpeak_kind):
+    """The split-K kernel against the HBM roofline (decode: every cache byte read
+    once) and against the tensor roofline; a prefill chunk (q_len > 8) reads a
+    few MB many times from L2 and is bound by the tensor side, which then leads."""
+    tensor_achieved = flops / (kernel_ms * 1e-3) / 1e12
+    hbm = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+           "frac": round(achieved / peak, 4), "traffic": traffic,
+           "algorithmic_bytes_per_launch": cache_bytes, "peak_source": peak_kind}
+    tensor = {"bound": "tensor", "achieved": round(tensor_achieved, 2), "peak": tpeak,
+              "unit": "TFLOP/s", "frac": round(tensor_achieved / tpeak, 4),
+              "flops_per_launch": flops, "peak_source": tpeak_kind}
+    rows = 32 if wl.q_len == 1 or wl.q_len > 8 or wl.max_seqlen <= 4096 else 64
+    lead, other = (tensor, hbm) if wl.q_len > 8 else (hbm, tensor)
+    line = dict(lead, kernel=f"mla_decode_kernel<{rows}>", kernel_ms=round(kernel_ms, 5))
+    line[other["bound"]] = {k: v for k, v in other.items() if k != "bound"}
+    if lead is tensor:
+        line["traffic"] = traffic
+    return line
+
+
 def stage_tensors(tensors, dev):
     """One device buffer holding `tensors` back to back (each at a 256-byte
     boundary) and views into it carrying the same values, so that a step's
@@ -448,7 +469,10 @@ def run_xmla(args, wl):
     gbs = job_throughput(cache_bytes_layer * wl.layers, args.steps, total_ms, world)
     peak, peak_kind = measured_peaks()
     tpeak, tpeak_kind = measured_tensor_peak()
-    flops_layer = 2176 * 32 * wl.q_len * sum(wl.seqlens)
+    # 2176 flop per attended (query row, cache token) pair: QK over 576, PV over 512;
+    # query j of a sequence of n tokens attends n - q_len + j + 1 tokens (causal)
+    pairs = sum(wl.q_len * (n - wl.q_len) + wl.q_len * (wl.q_len + 1) // 2 for n in wl.seqlens)
+    flops_layer = 2176 * 32 * pairs
     attn_mean_ms = statistics.mean(attn_ms)
     achieved = cache_bytes_layer / (attn_mean_ms * 1e-3) / 1e9
     ksha = kernel_sources_sha()
@@ -468,17 +492,8 @@ def run_xmla(args, wl):
                 if args.with_producer else {})),
             "attended_tokens_per_s": round(tokens_step * args.steps / (total_ms * 1e-3), 1),
             "pct_of_hbm_peak": round(100.0 * gbs / (peak * world), 2),
-            "roofline": {"bound": "hbm", "kernel": f"mla_decode_kernel<{32 if wl.q_len == 1 else 64}>",
-                         "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "algorithmic_bytes_per_launch": cache_bytes_layer,
-                         "kernel_ms": round(attn_mean_ms, 5), "peak_source": peak_kind,
-                         # the same launch against the tensor roofline: 2176 flop per cache
-                         # token and query row (QK over 576, PV over 512)
-                         "tensor": {"achieved": round(flops_layer / (attn_mean_ms * 1e-3) / 1e12, 2),
-                                    "peak": tpeak, "unit": "TFLOP/s",
-                                    "frac": round(flops_layer / (attn_mean_ms * 1e-3) / 1e12 / tpeak, 4),
-                                    "flops_per_launch": flops_layer, "peak_source": tpeak_kind}},
+            "roofline": roofline_line(wl, achieved, peak, peak_kind, traffic, cache_bytes_layer,
+                                      attn_mean_ms, flops_layer, tpeak, tpeak_kind),
             "e2e": {"value": round(job_throughput(cache_bytes_layer * wl.layers, args.steps,
                                                   e2e_total, world), 3),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

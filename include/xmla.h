@@ -192,8 +192,12 @@ int32_t xmla_decode_num_splits(int32_t batch, int32_t q_len, int64_t max_seqlen,
  *      256-byte aligned; its contents on entry do not matter;
  *   status_dev: device int32 or NULL (see conventions);
  *   out: device bf16 [batch, q_len, 32, 128].
- * Supported: 1 <= batch, 1 <= q_len <= 8, q_len <= max_seqlen <= 2^31 - 64,
- * num_blocks*64 < 2^31.  Errors: XMLA_ERR_INVALID_ARG, XMLA_ERR_SHAPE,
+ * Supported: 1 <= batch, 1 <= q_len <= 65536, q_len <= max_seqlen <= 2^31 - 64,
+ * num_blocks*64 < 2^31.  A q_len of a few tokens is a decode step (speculative
+ * verification above 1); a long q_len is a chunk of a prompt (chunked
+ * prefill), attended causally in the same absorbed form: each query sees the
+ * cache up to its own position, and the pages past a CTA's last query are
+ * skipped.  Errors: XMLA_ERR_INVALID_ARG, XMLA_ERR_SHAPE,
  * XMLA_ERR_WORKSPACE, XMLA_ERR_CUDA, XMLA_ERR_UNSUPPORTED (not an sm_100
  * device); device errors via status_dev. */
 xmla_status xmla_decode(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,

@@ -247,6 +247,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int j0 = g * (NR / 32);
   const int jn = min(p.q_len - j0, NR / 32);
   const int nrows = jn * 32;
+  // causal: pages past this CTA's last query position hold nothing it may see
+  // (a prefill chunk's early queries; at decode sizes this is the last page)
+  p_end = min(p_end, (seqlen - p.q_len + j0 + jn - 1) / kPage + 1);
   const int n_pages = (int)max((int64_t)0, p_end - p_begin);
   const int32_t qrow0 = (int32_t)(((int64_t)b * p.q_len + j0) * (L::kSplitQ ? 64 : 32));
   pdl_launch_dependents();

@@ -30,13 +30,16 @@ __global__ void wait_timeout_selftest_kernel(int32_t* status, uint64_t limit_ns)
 
 // ---------------------------------------------------------------- host plan
 
-// Up to this many tokens per sequence the query goes to the QK product as a hi
-// and a lo bf16 part (the split-K kernel's split_q layout, one query of 32
-// heads per CTA).  A short context is dominated by a few tokens and its output
-// is large (|out| up to ~4), so the ~2^-9 relative score error of a single
-// bf16 query reaches the 1e-2 output bound there; the split costs a shallower
-// page ring, which only long contexts, dominated by streaming, would notice.
+// Up to this many tokens per sequence, and for every call with more than
+// kSplitQMinChunk new tokens (a prefill chunk, whose first queries see only a
+// few tokens), the query goes to the QK product as a hi and a lo bf16 part
+// (the split-K kernel's split_q layout, one query of 32 heads per CTA).  A
+// short context is dominated by a few tokens and its output is large (|out|
+// up to ~4), so the ~2^-9 relative score error of a single bf16 query reaches
+// the 1e-2 output bound there; the split costs a shallower page ring, which
+// only long decode contexts, dominated by streaming, would notice.
 constexpr int64_t kSplitQMaxSeqlen = 4096;
+constexpr int32_t kSplitQMinChunk = 8;
 
 struct Plan {
   bool split;   // hi/lo query (split_q)
@@ -62,7 +65,7 @@ static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_
       max_seqlen > (int64_t)0x7fffffff - kPage || num_sms < 1 || num_splits < 0 || span_pages < 0)
     return false;
   Plan P;
-  P.split = max_seqlen <= kSplitQMaxSeqlen;
+  P.split = max_seqlen <= kSplitQMaxSeqlen || q_len > kSplitQMinChunk;
   P.nr = P.split || q_len == 1 ? 32 : 64;
   P.groups = (q_len * 32 + P.nr - 1) / P.nr;
   int64_t max_pages = (max_seqlen + kPage - 1) / kPage;

@@ -20,7 +20,7 @@ constexpr int kDV = 128;
 constexpr int kDQ = kDNope + kDRope;      // 192
 constexpr int kDRow = kDLatent + kDRope;  // 576 bf16 per cache row
 constexpr int kPage = 64;                 // tokens per cache block
-constexpr int kMaxQLen = 8;
+constexpr int kMaxQLen = 65536;  // new tokens per sequence and call (decode steps to prefill chunks)
 
 // Default limit of one bounded wait inside a kernel (nanoseconds).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;

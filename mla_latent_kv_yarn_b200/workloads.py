@@ -19,6 +19,9 @@ latent 512 + rope 64 per token, nope 128, v 128):
   step_40l_b32    40 layers, B=32, q_len=1, N_s ~ U[8192, 65536], shuffled pages
   verify_q4_b8    B=8, q_len=4 (causal among the 4 new tokens), N=131072, shuffled
   decode_512k_b4  B=4, q_len=1, N=524288 (positions past 262144), shuffled
+and one more, outside those five:
+  prefill_4k      B=1, a 4096-token prompt attended as one chunk (q_len=4096, N=4096,
+                  causal), shuffled pages
 """
 from __future__ import annotations
 
@@ -63,10 +66,13 @@ class Workload:
 
 
 WORKLOAD_NAMES = ["decode_4k", "decode_256k", "step_40l_b32", "verify_q4_b8", "decode_512k_b4"]
+EXTRA_WORKLOADS = ["prefill_4k"]
 
 
 def workload(index_or_name) -> Workload:
-    """The five seeded workloads, by index 0..4 or by name."""
+    """The five seeded workloads, by index 0..4 or by name, and the extra ones by name."""
+    if index_or_name == "prefill_4k":
+        return Workload("prefill_4k", 1, 4096, [4096], seed=1234 + 5)
     idx = WORKLOAD_NAMES.index(index_or_name) if isinstance(index_or_name, str) else int(index_or_name)
     seed = 1234 + idx
     if idx == 0:

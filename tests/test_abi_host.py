@@ -65,7 +65,8 @@ def test_workspace_plan(x):
     # q_ext (32 x 576 bf16) + partial O (148 x 32 x 512 fp32) + (m, l), 1 KiB aligned pieces
     assert ws >= 148 * 32 * 512 * 4 + 148 * 32 * 8 + 32 * 576 * 2
     assert ws % 1024 == 0
-    assert x.xmla_decode_workspace_size(1, 9, 4096, 148) == 0      # q_len > 8
+    assert x.xmla_decode_workspace_size(1, 65537, 70000, 148) == 0  # q_len > 65536
+    assert x.xmla_decode_workspace_size(1, 4096, 4096, 148) > 0     # a prefill chunk
     assert x.xmla_decode_workspace_size(0, 1, 4096, 148) == 0
     assert x.xmla_decode_workspace_size(1, 4, 3, 148) == 0         # max_seqlen < q_len
 

@@ -305,6 +305,31 @@ def test_short_contexts(q_len, seed):
     gc.assert_close(out, gc.oracle_out(wl, inp, ocfg), f"short {seqlens}")
 
 
+# ------------------------------------------------------------------ prefill chunks
+
+# A long q_len is a chunk of a prompt: the chunk's tokens are appended and each
+# attends causally to the cache up to its own position (the first ones of a
+# fresh prompt see a handful of tokens).
+PREFILL_CASES = [
+    # batch, q_len, seqlens, oracle form
+    (1, 64, [64], "expanded"),             # a fresh 64-token prompt
+    (1, 200, [1000], "expanded"),          # a chunk on an 800-token prefix
+    (2, 130, [130, 700], "expanded"),      # one fresh prompt, one continued
+    (1, 96, [4500], "absorbed"),           # a chunk past 4096 tokens
+    (1, 1024, [1024], "absorbed"),
+]
+
+
+@pytest.mark.parametrize("batch,q_len,seqlens,form", PREFILL_CASES)
+def test_prefill_chunk_matches_the_oracle(batch, q_len, seqlens, form):
+    wl = workloads.custom(batch, q_len, seqlens, seed=400 + q_len + sum(seqlens))
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg)
+    assert dec.check_status() == 0
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, form=form), f"prefill {q_len} {seqlens}")
+
+
 def test_length_aware_plan_is_deterministic():
     wl = workloads.custom(3, 2, [4000, 90, 1500], seed=77)
     cfg, _ = gc.cfgs()

@@ -123,7 +123,7 @@ def test_combine_shards_rejects_bad_arguments():
     buf = torch.zeros(2 * xmla.xmla_shard_partial_floats(1, 1), dtype=torch.float32, device=dev)
     out = torch.empty((1, 1, 32, 128), dtype=torch.bfloat16, device=dev)
     for args, code in [((buf, 0, W, 1, 1, out), "XMLA_ERR_SHAPE"),
-                       ((buf, 2, W, 1, 9, out), "XMLA_ERR_SHAPE"),
+                       ((buf, 2, W, 1, 65537, out), "XMLA_ERR_SHAPE"),
                        ((buf[1:], 2, W, 1, 1, out), "XMLA_ERR_INVALID_ARG")]:
         with pytest.raises(xmla.XmlaError, match=code):
             xmla.xmla_combine_shards(*args)
