@@ -242,9 +242,27 @@ static bool plan_ok(const WorkPlanArgs& plan) {
 // q and seqlens carry no __restrict__ so that their loads stay behind the
 // griddepcontrol.wait (a preceding kernel may have written them).
 // kPlan: one more block computes the length-aware plan (batch > 1).
-// kRowBlocks: every absorb block takes kAbsorbRows query rows (more rows than
-// that: kAbsorbBlocks blocks per kAbsorbRows rows); else all rows.
-template <bool kPlan, bool kRowBlocks>
+// kRows: 0 = every absorb block takes all rows; 1 = kAbsorbRows query rows each
+// (kAbsorbBlocks blocks per kAbsorbRows rows); 2 = the same for the rope blocks
+// only (a prompt chunk, whose latent part the tensor-core absorb computes).
+template <int kRows>
+struct AbsorbGrid {
+  static constexpr int kPerRows = kRows == 2 ? kHeads : kAbsorbBlocks;
+  __device__ __forceinline__ static int blocks(int rows) {
+    return kRows ? kPerRows * ((rows + kAbsorbRows - 1) / kAbsorbRows) : kAbsorbBlocks;
+  }
+  // block -> (head, column block, first row, end row)
+  __device__ __forceinline__ static void map(int blk, int rows, int& h, int& cb, int& r_lo,
+                                             int& r_hi) {
+    const int hb = kRows ? blk % kPerRows : blk;
+    r_lo = kRows ? (blk / kPerRows) * kAbsorbRows : 0;
+    r_hi = kRows ? min(rows, r_lo + kAbsorbRows) : rows;
+    h = kRows == 2 ? hb : hb % kHeads;
+    cb = kRows == 2 ? kDLatent / 64 : hb / kHeads;
+  }
+};
+
+template <bool kPlan, int kRows>
 __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
     __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, int split, float qscale,
@@ -254,19 +272,18 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
     PlanSmem plan;
   } sm;
   pdl_launch_dependents();
-  const int absorb_blocks =
-      kRowBlocks ? kAbsorbBlocks * ((rows + kAbsorbRows - 1) / kAbsorbRows) : kAbsorbBlocks;
+  using G = AbsorbGrid<kRows>;
+  const int absorb_blocks = G::blocks(rows);
   if constexpr (kPlan) {
     if (blockIdx.x == absorb_blocks) {
       work_plan_block(plan, sm.plan);
       return;
     }
   }
-  const int hb = kRowBlocks ? blockIdx.x % kAbsorbBlocks : blockIdx.x;
-  const int r_lo = kRowBlocks ? (blockIdx.x / kAbsorbBlocks) * kAbsorbRows : 0;
-  const int r_hi = kRowBlocks ? min(rows, r_lo + kAbsorbRows) : rows;
-  q_absorb_block<kRowBlocks>(hb % kHeads, hb / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
-                             split, qscale, tab, sm.absorb, r_lo, r_hi);
+  int h, cb, r_lo, r_hi;
+  G::map(blockIdx.x, rows, h, cb, r_lo, r_hi);
+  q_absorb_block<kRows != 0>(h, cb, q, W_UK, seqlens, q_ext, rows, q_len, split, qscale, tab,
+                             sm.absorb, r_lo, r_hi);
 }
 
 // The first kernel of a decode step: the absorb blocks above, then the
@@ -275,8 +292,8 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
 // cache rows (one thread per 16-byte piece).  All of them only wait for the
 // kernel launched before this one, so they run side by side.
 // kPlan: one more block computes the length-aware plan (batch > 1); the
-// producer and append blocks follow it.  kRowBlocks as for q_absorb_kernel.
-template <bool kPlan, bool kRowBlocks>
+// producer and append blocks follow it.  kRows as for q_absorb_kernel.
+template <bool kPlan, int kRows>
 __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
     __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, int split, float qscale,
@@ -289,14 +306,13 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
     PlanSmem plan;
   } sm;
   pdl_launch_dependents();
-  const int absorb_blocks =
-      kRowBlocks ? kAbsorbBlocks * ((rows + kAbsorbRows - 1) / kAbsorbRows) : kAbsorbBlocks;
+  using G = AbsorbGrid<kRows>;
+  const int absorb_blocks = G::blocks(rows);
   if (blockIdx.x < absorb_blocks) {
-    const int hb = kRowBlocks ? blockIdx.x % kAbsorbBlocks : blockIdx.x;
-    const int r_lo = kRowBlocks ? (blockIdx.x / kAbsorbBlocks) * kAbsorbRows : 0;
-    const int r_hi = kRowBlocks ? min(rows, r_lo + kAbsorbRows) : rows;
-    q_absorb_block<kRowBlocks>(hb % kHeads, hb / kHeads, q, W_UK, seqlens, q_ext, rows, q_len,
-                               split, qscale, q_tab, sm.absorb, r_lo, r_hi);
+    int h, cb, r_lo, r_hi;
+    G::map(blockIdx.x, rows, h, cb, r_lo, r_hi);
+    q_absorb_block<kRows != 0>(h, cb, q, W_UK, seqlens, q_ext, rows, q_len, split, qscale, q_tab,
+                               sm.absorb, r_lo, r_hi);
     return;
   }
   constexpr int kPlanBlocks = kPlan ? 1 : 0;
@@ -326,19 +342,25 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
                             int split, float qscale, const RopeTable& tab,
-                            const WorkPlanArgs* plan, cudaStream_t st) {
-  const bool rb = rows > kAbsorbRows;
+                            const WorkPlanArgs* plan, bool rope_only, cudaStream_t st) {
+  const int mode = rope_only ? 2 : rows > kAbsorbRows ? 1 : 0;
+  const int64_t nrb = (rows + kAbsorbRows - 1) / kAbsorbRows;
   const unsigned absorb_blocks =
-      rb ? kAbsorbBlocks * (unsigned)((rows + kAbsorbRows - 1) / kAbsorbRows) : kAbsorbBlocks;
+      (unsigned)(mode == 2 ? kHeads * nrb : mode == 1 ? kAbsorbBlocks * nrb : kAbsorbBlocks);
+  auto kern = [&](bool with_plan) {
+    if (with_plan)
+      return mode == 2 ? q_absorb_kernel<true, 2> : mode == 1 ? q_absorb_kernel<true, 1>
+                                                              : q_absorb_kernel<true, 0>;
+    return mode == 2 ? q_absorb_kernel<false, 2> : mode == 1 ? q_absorb_kernel<false, 1>
+                                                             : q_absorb_kernel<false, 0>;
+  };
   if (plan != nullptr) {
     if (!plan_ok(*plan)) return cudaErrorInvalidValue;
-    return launch_pdl(rb ? q_absorb_kernel<true, true> : q_absorb_kernel<true, false>,
-                      dim3(absorb_blocks + 1), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens,
-                      q_ext, rows, q_len, split, qscale, tab, *plan);
+    return launch_pdl(kern(true), dim3(absorb_blocks + 1), dim3(kAbsorbThreads), 0, st, q, W_UK,
+                      seqlens, q_ext, rows, q_len, split, qscale, tab, *plan);
   }
-  return launch_pdl(rb ? q_absorb_kernel<false, true> : q_absorb_kernel<false, false>,
-                    dim3(absorb_blocks), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext,
-                    rows, q_len, split, qscale, tab, WorkPlanArgs{});
+  return launch_pdl(kern(false), dim3(absorb_blocks), dim3(kAbsorbThreads), 0, st, q, W_UK,
+                    seqlens, q_ext, rows, q_len, split, qscale, tab, WorkPlanArgs{});
 }
 
 cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
@@ -346,24 +368,30 @@ cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_
                                  int q_len, int split, float qscale, const RopeTable& q_tab,
                                  const AppendArgs& ap, const RopeTable& k_tab,
                                  const ProduceArgs* pa, const WorkPlanArgs* plan,
-                                 cudaStream_t st) {
+                                 bool rope_only, cudaStream_t st) {
   const int64_t append_blocks = (ap.T * kRowPieces + kAbsorbThreads - 1) / kAbsorbThreads;
   if (append_blocks > (1 << 20)) return cudaErrorInvalidValue;
   ProduceArgs none{};
   const ProduceArgs& p = pa != nullptr ? *pa : none;
   const int64_t prod_blocks = p.T > 0 ? kProdBlocks : 0;
-  const bool rb = rows > kAbsorbRows;
+  const int mode = rope_only ? 2 : rows > kAbsorbRows ? 1 : 0;
+  const int64_t nrb = (rows + kAbsorbRows - 1) / kAbsorbRows;
   const int64_t absorb_blocks =
-      rb ? (int64_t)kAbsorbBlocks * ((rows + kAbsorbRows - 1) / kAbsorbRows) : kAbsorbBlocks;
+      mode == 2 ? kHeads * nrb : mode == 1 ? (int64_t)kAbsorbBlocks * nrb : kAbsorbBlocks;
+  auto kern = [&](bool with_plan) {
+    if (with_plan)
+      return mode == 2 ? step_prologue_kernel<true, 2>
+                       : mode == 1 ? step_prologue_kernel<true, 1> : step_prologue_kernel<true, 0>;
+    return mode == 2 ? step_prologue_kernel<false, 2>
+                     : mode == 1 ? step_prologue_kernel<false, 1> : step_prologue_kernel<false, 0>;
+  };
   if (plan != nullptr) {
     if (!plan_ok(*plan)) return cudaErrorInvalidValue;
-    return launch_pdl(rb ? step_prologue_kernel<true, true> : step_prologue_kernel<true, false>,
-                      dim3((unsigned)(absorb_blocks + 1 + prod_blocks + append_blocks)),
+    return launch_pdl(kern(true), dim3((unsigned)(absorb_blocks + 1 + prod_blocks + append_blocks)),
                       dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, split,
                       qscale, q_tab, ap, k_tab, p, *plan);
   }
-  return launch_pdl(rb ? step_prologue_kernel<false, true> : step_prologue_kernel<false, false>,
-                    dim3((unsigned)(absorb_blocks + prod_blocks + append_blocks)),
+  return launch_pdl(kern(false), dim3((unsigned)(absorb_blocks + prod_blocks + append_blocks)),
                     dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, split,
                     qscale, q_tab, ap, k_tab, p, WorkPlanArgs{});
 }
@@ -707,6 +735,96 @@ __global__ void __launch_bounds__(kCombineThreads)
       out[R * kDLatent + 2 * row + 1] = L;
     }
   }
+}
+
+// ---------------------------------------------------------------- latent output of a prompt chunk
+
+// For the tensor-core W_UV product of a prompt chunk: the splits of each
+// (row, head) merged and normalised, o = sum_s 2^(m_s - M) O_s / L, written as
+// o_hi = bf16(o) and o_lo = bf16(o - o_hi) at [(r * 32 + h) * 512 + d].  Blocks
+// as in the combine (64-dim slice, head, chunk of up to 16 rows), 256 threads.
+template <bool kTable>
+__global__ void __launch_bounds__(kCombineThreads)
+    latent_out_kernel(const float* part_o, const float* part_ml, __nv_bfloat16* __restrict__ o_hi,
+                      __nv_bfloat16* __restrict__ o_lo, int rows, int q_len, int groups,
+                      int nsplit, int rows_per_cta, const int2* unit_tab) {
+  __shared__ __align__(16) float4 acc_s[kCombineGroups][kSliceDims / 4];
+  __shared__ float grp_m[kCombineGroups], grp_l[kCombineGroups];
+  const int slice = blockIdx.x % kSlices;
+  const int cid = blockIdx.x / kSlices;
+  const int h = cid % kHeads;
+  const int chunk = cid / kHeads;
+  const int r0 = chunk * kCombineRows;
+  const int nr = min(kCombineRows, rows - r0);
+  const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  const int q4 = tid & 15;
+  const int grp = tid >> 4;
+  const int gpr = max(1, kCombineGroups / nr);
+  const int my_rr = grp / gpr;
+  const int sub = grp % gpr;
+  const bool active = my_rr < nr;
+  int unit = 0, ridx = 0;
+  if (active) {
+    const int r = r0 + my_rr;
+    const int b = r / q_len, j = r % q_len;
+    ridx = j * kHeads + h;
+    unit = b * groups + ridx / rows_per_cta;
+  }
+  pdl_wait();  // the split partials come from the decode kernel
+  int64_t base = (int64_t)unit * nsplit * rows_per_cta + ridx % rows_per_cta;
+  int ns = nsplit;
+  if constexpr (kTable) {
+    const int2 ut = active ? unit_tab[unit] : make_int2(0, 0);
+    ns = ut.y;
+    base = (int64_t)ut.x * rows_per_cta + ridx % rows_per_cta;
+  }
+  const float* po = part_o + base * kDLatent + slice * kSliceDims + 4 * q4;
+  const float2* pml = reinterpret_cast<const float2*>(part_ml) + base;
+  float m_g, l_g;
+  float4 acc;
+  merge_group(po, pml, (int64_t)rows_per_cta * kDLatent, rows_per_cta, ns, sub, gpr, q4, active,
+              m_g, l_g, acc);
+  acc_s[grp][q4] = acc;
+  if (q4 == 0) {
+    grp_m[grp] = m_g;
+    grp_l[grp] = l_g;
+  }
+  __syncthreads();
+  for (int e = tid; e < nr * kSliceDims / 2; e += kCombineThreads) {
+    const int rr = e / (kSliceDims / 2), d = 2 * (e % (kSliceDims / 2));
+    const int g0 = rr * gpr;
+    float M = -INFINITY;
+    for (int g = 0; g < gpr; ++g)
+      if (grp_l[g0 + g] > 0.f) M = fmaxf(M, grp_m[g0 + g]);
+    float L = 0.f, t0 = 0.f, t1 = 0.f;
+    for (int g = 0; g < gpr; ++g) {
+      if (grp_l[g0 + g] > 0.f) {
+        const float w = ex2(grp_m[g0 + g] - M);
+        L = fmaf(w, grp_l[g0 + g], L);
+        t0 = fmaf(w, reinterpret_cast<const float*>(&acc_s[g0 + g][0])[d], t0);
+        t1 = fmaf(w, reinterpret_cast<const float*>(&acc_s[g0 + g][0])[d + 1], t1);
+      }
+    }
+    const float a = L > 0.f ? t0 / L : 0.f, c = L > 0.f ? t1 / L : 0.f;
+    const __nv_bfloat162 hv = __floats2bfloat162_rn(a, c);
+    const __nv_bfloat162 lv = __floats2bfloat162_rn(a - __low2float(hv), c - __high2float(hv));
+    const int64_t off = ((int64_t)(r0 + rr) * kHeads + h) * kDLatent + slice * kSliceDims + d;
+    *reinterpret_cast<__nv_bfloat162*>(o_hi + off) = hv;
+    *reinterpret_cast<__nv_bfloat162*>(o_lo + off) = lv;
+  }
+}
+
+cudaError_t launch_latent_out(const float* part_o, const float* part_ml, __nv_bfloat16* o_hi,
+                              __nv_bfloat16* o_lo, int rows, int q_len, int groups, int nsplit,
+                              int rows_per_cta, const int2* unit_tab, cudaStream_t st) {
+  const int chunks = (rows + kCombineRows - 1) / kCombineRows;
+  const dim3 grid(kSlices * kHeads * chunks);
+  if (unit_tab != nullptr)
+    return launch_pdl(latent_out_kernel<true>, grid, dim3(kCombineThreads), 0, st, part_o, part_ml,
+                      o_hi, o_lo, rows, q_len, groups, nsplit, rows_per_cta, unit_tab);
+  return launch_pdl(latent_out_kernel<false>, grid, dim3(kCombineThreads), 0, st, part_o, part_ml,
+                    o_hi, o_lo, rows, q_len, groups, nsplit, rows_per_cta, unit_tab);
 }
 
 cudaError_t launch_merge_splits(const float* part_o, const float* part_ml, float* out, int rows,

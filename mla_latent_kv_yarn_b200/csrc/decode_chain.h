@@ -44,10 +44,12 @@ struct WorkPlanArgs {
 // q_ext[r, h] for rows r = b*q_len + j; qscale = softmax scale * log2 e.
 // split: each query row as a hi and a lo bf16 row (the split-K kernel's
 // split_q layout).  plan (nullable): also compute the length-aware plan.
+// rope_only: only the rope columns (the latent part comes from
+// launch_absorb_gemm).
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
                             int split, float qscale, const RopeTable& tab,
-                            const WorkPlanArgs* plan, cudaStream_t st);
+                            const WorkPlanArgs* plan, bool rope_only, cudaStream_t st);
 
 // The new tokens of a decode step, appended by step_prologue_kernel.
 struct AppendArgs {
@@ -73,7 +75,7 @@ cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_
                                  int q_len, int split, float qscale, const RopeTable& q_tab,
                                  const AppendArgs& ap, const RopeTable& k_tab,
                                  const ProduceArgs* pa, const WorkPlanArgs* plan,
-                                 cudaStream_t st);
+                                 bool rope_only, cudaStream_t st);
 
 // Merge of the splits and the W_UV product, written to out[rows, 32, 128].
 // Split s of a row is o_stride floats (O) and ml_stride (m, l) pairs after
@@ -84,6 +86,33 @@ cudaError_t launch_combine(const float* part_o, const float* part_ml, const __nv
                            __nv_bfloat16* out, int rows, int q_len, int groups, int nsplit,
                            int rows_per_cta, cudaStream_t st, int64_t o_stride = 0,
                            int64_t ml_stride = 0, const int2* unit_tab = nullptr);
+
+// Per-head tensor-core products of a prompt chunk (head_gemm.cu).  Rows r =
+// b*q_len + j, R of them.
+struct HeadGemmParams {
+  int rows;                 // R
+  float scale;              // absorb: softmax scale * log2 e
+  __nv_bfloat16* q_ext;     // absorb: latent columns of the hi/lo query rows
+  __nv_bfloat16* out;       // W_UV: out[R, 32, 128]
+  int32_t* status;
+  uint64_t wait_limit_ns;
+};
+// q_lat = q_nope . W_UK[h] for every head, written scaled as hi/lo bf16 into
+// q_ext (split query layout).  q_map: the query [R, 32, 192] as a 3-D map, box
+// 64 x 1 x 128; wuk_map: W_UK as [4096, 512], box 64 x 128 (both 128-B swizzle).
+cudaError_t launch_absorb_gemm(const CUtensorMap& q_map, const CUtensorMap& wuk_map,
+                               const HeadGemmParams& p, cudaStream_t st);
+// out = (o_hi + o_lo) . W_UV[h] for every head.  ohi/olo_map: [R, 32, 512]
+// bf16 as 3-D maps, box 64 x 1 x 128; wuv_map: W_UV as [16384, 128], box 64 x 128.
+cudaError_t launch_uv_gemm(const CUtensorMap& ohi_map, const CUtensorMap& olo_map,
+                           const CUtensorMap& wuv_map, const HeadGemmParams& p, cudaStream_t st);
+
+// The merged latent output of every (row, head), normalised, as two bf16 parts
+// o_hi = bf16(o), o_lo = bf16(o - o_hi), each [rows, 32, 512]; unit_tab as for
+// launch_combine.
+cudaError_t launch_latent_out(const float* part_o, const float* part_ml, __nv_bfloat16* o_hi,
+                              __nv_bfloat16* o_lo, int rows, int q_len, int groups, int nsplit,
+                              int rows_per_cta, const int2* unit_tab, cudaStream_t st);
 
 // Merge of the splits into one partial per (row, head) -- (M, L, unnormalised
 // O) -- for a sequence-parallel decode; layout in absorb_combine.cu.

@@ -43,12 +43,13 @@ constexpr int32_t kSplitQMinChunk = 8;
 
 struct Plan {
   bool split;   // hi/lo query (split_q)
+  bool gemm;    // a prompt chunk: absorb and W_UV on the tensor cores (head_gemm.cu)
   int nr;       // rows per CTA (32 or 64)
   int groups;   // row groups per sequence
   int nsplit;   // KV splits per (sequence, group) when every sequence has max_seqlen tokens
   bool table;   // splits planned on the device from the actual lengths (WorkPlanArgs)
   int64_t items;
-  size_t off_qext, off_o, off_ml, off_wtab, off_utab, bytes;
+  size_t off_qext, off_o, off_ml, off_wtab, off_utab, off_olat, bytes;
 };
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -94,7 +95,11 @@ static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_
   P.off_ml = align_up(P.off_o + (size_t)P.items * P.nr * kDLatent * 4, 1024);
   P.off_wtab = align_up(P.off_ml + (size_t)P.items * P.nr * 2 * 4, 1024);
   P.off_utab = align_up(P.off_wtab + (P.table ? (size_t)P.items * 16 : 0), 256);
-  P.bytes = align_up(P.off_utab + (P.table ? (size_t)units * 8 : 0), 1024);
+  // a prompt chunk's merged latent output, hi and lo bf16 [rows, 32, 512] each
+  P.gemm = allow_table && q_len > kSplitQMinChunk;
+  P.off_olat = align_up(P.off_utab + (P.table ? (size_t)units * 8 : 0), 1024);
+  const size_t olat = P.gemm ? (size_t)B * q_len * kHeads * kDLatent * 2 : 0;
+  P.bytes = align_up(P.off_olat + 2 * olat, 1024);
   *pl = P;
   return true;
 }
@@ -120,6 +125,35 @@ static bool encode_rows576(CUtensorMap* m, const void* ptr, uint64_t rows, uint3
   cuuint64_t dims[2] = {(cuuint64_t)kDRow, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kDRow * 2};
   cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over a [rows, 32, cols] bf16 tensor (the query, cols 192, or o_lat,
+// cols 512), box 64 columns x 1 head x 128 rows, 128-byte swizzle: one box is a
+// 128-row K-major tile of one head.
+static bool encode_heads3d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)kHeads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * 2 * kHeads};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over a row-major [rows, cols] bf16 weight, box 64 columns x 128 rows,
+// 128-byte swizzle: one box is 128 K rows of 64 N columns (an MN-major tile).
+static bool encode_weight(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, 128};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -223,15 +257,38 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   // Every kernel of the chain waits (griddepcontrol.wait) for its predecessor
   // before reading anything a kernel of this step may have written, so once
   // the first kernel completes all earlier work on the stream has landed.
+  // A prompt chunk runs five kernels: the first does the rope columns of q_ext
+  // (and the append, the plan) while the tensor-core absorb fills the latent
+  // columns; after the split-K kernel the merged latent output goes out as
+  // hi/lo bf16 and the tensor-core W_UV product writes `out`.
+  HeadGemmParams gp{};
+  CUtensorMap tmap_qin, tmap_wuk, tmap_ohi, tmap_olo, tmap_wuv;
+  __nv_bfloat16* o_hi = (__nv_bfloat16*)(ws + P.off_olat);
+  __nv_bfloat16* o_lo = o_hi + (size_t)rows * kHeads * kDLatent;
+  if (P.gemm) {
+    if (!encode_heads3d(&tmap_qin, q, (uint64_t)rows, kDQ) ||
+        !encode_weight(&tmap_wuk, W_UK, (uint64_t)kHeads * kDNope, kDLatent) ||
+        !encode_heads3d(&tmap_ohi, o_hi, (uint64_t)rows, kDLatent) ||
+        !encode_heads3d(&tmap_olo, o_lo, (uint64_t)rows, kDLatent) ||
+        !encode_weight(&tmap_wuv, W_UV, (uint64_t)kHeads * kDLatent, kDV))
+      return XMLA_ERR_CUDA;
+    gp.rows = rows;
+    gp.scale = qscale;
+    gp.q_ext = q_ext;
+    gp.out = (__nv_bfloat16*)out;
+    gp.status = status_dev;
+    gp.wait_limit_ns = kWaitLimitNs;
+  }
   const cudaError_t e0 =
       ap != nullptr
           ? launch_step_prologue((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
                                  rows, q_len, P.split ? 1 : 0, qscale, tab, *ap, tab, pa,
-                                 P.table ? &plan : nullptr, st)
+                                 P.table ? &plan : nullptr, P.gemm, st)
           : launch_q_absorb((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
                             rows, q_len, P.split ? 1 : 0, qscale, tab,
-                            P.table ? &plan : nullptr, st);
+                            P.table ? &plan : nullptr, P.gemm, st);
   if (e0 != cudaSuccess) return XMLA_ERR_CUDA;
+  if (P.gemm && launch_absorb_gemm(tmap_qin, tmap_wuk, gp, st) != cudaSuccess) return XMLA_ERR_CUDA;
 
   DecodeParams dp;
   dp.block_table = block_table;
@@ -258,6 +315,13 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
     const cudaError_t em = launch_merge_splits(dp.part_o, dp.part_ml, shard_partial, rows, q_len,
                                                P.groups, P.nsplit, P.nr, st);
     return em == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+  }
+  if (P.gemm) {
+    if (launch_latent_out(dp.part_o, dp.part_ml, o_hi, o_lo, rows, q_len, P.groups, P.nsplit, P.nr,
+                          P.table ? plan.unit_tab : nullptr, st) != cudaSuccess)
+      return XMLA_ERR_CUDA;
+    return launch_uv_gemm(tmap_ohi, tmap_olo, tmap_wuv, gp, st) == cudaSuccess ? XMLA_OK
+                                                                               : XMLA_ERR_CUDA;
   }
   const cudaError_t e = launch_combine(dp.part_o, dp.part_ml, (const __nv_bfloat16*)W_UV,
                                        (__nv_bfloat16*)out, rows, q_len, P.groups, P.nsplit, P.nr,
