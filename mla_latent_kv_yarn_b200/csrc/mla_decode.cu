@@ -626,7 +626,55 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                  abort_flag, p.status, p.wait_limit_ns);
       have = !named_bar_or(1, kSoftmaxThreads, !okw);
     }
-    if (have) {
+    bool direct = false;
+    if constexpr (L::kSplitQ) direct = p.o_hi != nullptr;
+    if (have && direct) {
+      // one split per unit: normalise here and write the bf16 hi/lo latent
+      // output; the row sums come first, their reciprocals go to m_used
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < NR / 32; ++c) {
+        float tmp[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) tmp[k] = l_part[16 * c + k];
+        xpose_reduce16<false>(tmp, lane);
+        red[quarter * NR + pr + 2 * (16 * c + row_t)] = tmp[0];
+      }
+      named_bar_sync(1, kSoftmaxThreads);
+      if (tid < NR) {
+        const float l = red[tid] + red[NR + tid] + red[2 * NR + tid] + red[3 * NR + tid];
+        m_used[tid] = l > 0.f ? 1.f / l : 0.f;
+      }
+      named_bar_sync(1, kSoftmaxThreads);
+#pragma unroll 1
+      for (int m = 0; m < 4; ++m) {
+        const int d = 128 * m + 32 * quarter + lane;
+#pragma unroll
+        for (int c = 0; c < NR / 32; ++c) {
+          float o[32];
+          tmem_ld32(t_lane + L::kColO + m * NR + 32 * c, o);
+          tc_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const int n = 32 * c + k;
+            if (n < nrows) {
+              const float v = o[k] * m_used[n];
+              const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+              const int64_t off = (row0 + n) * kDLatent + d;
+              p.o_hi[off] = hv;
+              p.o_lo[off] = __float2bfloat16_rn(v - __bfloat162float(hv));
+            }
+          }
+        }
+      }
+    } else if (direct) {
+      pdl_wait();  // the previous step's W_UV product may still read these rows
+      const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+      for (int e = tid; e < nrows * kDLatent; e += kSoftmaxThreads) {
+        p.o_hi[row0 * kDLatent + e] = z;
+        p.o_lo[row0 * kDLatent + e] = z;
+      }
+    } else if (have) {
       tc_fence_after();
 #pragma unroll 1
       for (int m = 0; m < 4; ++m) {
@@ -658,6 +706,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         p.part_ml[(row0 + tid) * 2 + 1] = l;
       }
     } else if (tid < nrows) {
+      pdl_wait();  // the previous step's merge may still read this split's m, l
       p.part_ml[(row0 + tid) * 2 + 0] = -INFINITY;
       p.part_ml[(row0 + tid) * 2 + 1] = 0.f;
     }

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -39,6 +40,12 @@ struct DecodeParams {
   // first logical page, end page, 0} of CTA k, unit -1 for an idle CTA.  The
   // kernel reads it after griddepcontrol.wait; nsplit and page_lo/hi are unused.
   const int4* work_tab;
+  // non-null (split_q, one split per unit, no work table): the kernel writes
+  // the normalised latent output o = O / l itself as o_hi = bf16(o) and
+  // o_lo = bf16(o - o_hi) at [(r * 32 + h) * 512 + d] (r = b * q_len + j)
+  // instead of part_o / part_ml
+  __nv_bfloat16* o_hi;
+  __nv_bfloat16* o_lo;
 };
 
 // Split-K attention over `items` work items; nr = rows per CTA (32 or 64);

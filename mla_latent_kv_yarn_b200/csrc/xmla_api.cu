@@ -259,8 +259,9 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   // the first kernel completes all earlier work on the stream has landed.
   // A prompt chunk runs five kernels: the first does the rope columns of q_ext
   // (and the append, the plan) while the tensor-core absorb fills the latent
-  // columns; after the split-K kernel the merged latent output goes out as
-  // hi/lo bf16 and the tensor-core W_UV product writes `out`.
+  // columns; the latent output goes out as hi/lo bf16 (from the split-K
+  // kernel itself when every unit has one split, else from a merge kernel)
+  // and the tensor-core W_UV product writes `out`.
   HeadGemmParams gp{};
   CUtensorMap tmap_qin, tmap_wuk, tmap_ohi, tmap_olo, tmap_wuv;
   __nv_bfloat16* o_hi = (__nv_bfloat16*)(ws + P.off_olat);
@@ -307,6 +308,11 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   dp.page_lo = page_lo;
   dp.page_hi = page_hi;
   dp.work_tab = P.table ? plan.work_tab : nullptr;
+  // a prompt chunk with one split per unit needs no merge: the attention
+  // kernel writes the normalised hi/lo latent output the W_UV GEMM reads
+  const bool direct = P.gemm && P.split && P.nsplit == 1 && !P.table && shard_partial == nullptr;
+  dp.o_hi = direct ? o_hi : nullptr;
+  dp.o_lo = direct ? o_lo : nullptr;
   if (record_event(attn_start, st) != cudaSuccess) return XMLA_ERR_CUDA;
   if (launch_split_kv(P.nr, P.split, tmap_pool, tmap_q, dp, P.items, st) != cudaSuccess)
     return XMLA_ERR_CUDA;
@@ -317,7 +323,8 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
     return em == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
   }
   if (P.gemm) {
-    if (launch_latent_out(dp.part_o, dp.part_ml, o_hi, o_lo, rows, q_len, P.groups, P.nsplit, P.nr,
+    if (!direct &&
+        launch_latent_out(dp.part_o, dp.part_ml, o_hi, o_lo, rows, q_len, P.groups, P.nsplit, P.nr,
                           P.table ? plan.unit_tab : nullptr, st) != cudaSuccess)
       return XMLA_ERR_CUDA;
     return launch_uv_gemm(tmap_ohi, tmap_olo, tmap_wuv, gp, st) == cudaSuccess ? XMLA_OK

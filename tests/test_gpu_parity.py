@@ -317,6 +317,8 @@ PREFILL_CASES = [
     (2, 130, [130, 700], "expanded"),      # one fresh prompt, one continued
     (1, 96, [4500], "absorbed"),           # a chunk past 4096 tokens
     (1, 1024, [1024], "absorbed"),
+    (1, 16, [3000], "absorbed"),           # several splits per unit: merged before W_UV
+    (2, 12, [2000, 500], "absorbed"),      # length-aware plan, merged through the unit table
 ]
 
 
@@ -442,6 +444,27 @@ def test_workload_decode_512k_b4():
     out, dec, _ = gc.gpu_step(wl, inp, cfg)
     assert dec.check_status() == 0
     gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, seqs=[0, 3], form="absorbed"), "decode_512k_b4", plain_max_abs=True)
+
+
+def test_workload_prefill_4k_sampled_queries():
+    # query j of the chunk sits at position N - q_len + j and sees tokens 0..that
+    # position, which is the one-query case over the first position + 1 tokens
+    wl = workloads.workload("prefill_4k")
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cuda")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg)
+    assert dec.check_status() == 0
+    n, ql = wl.seqlens[0], wl.q_len
+    js = [0, 1, 63, 64, 127, 1000, 2047, 2048, 3071, 4000, ql - 1]
+    c, kp = gc.f64(inp.c_kv[:n]), gc.f64(inp.k_pe[:n])
+    kp_rot = om.rope(kp, np.arange(n), ocfg)
+    wk, wv = gc.f64(inp.W_UK), gc.f64(inp.W_UV)
+    ref = []
+    for j in js:
+        t = n - ql + j + 1
+        ref.append(om.mla_attention_absorbed(gc.f64(inp.q[0, j:j + 1]), c[:t], kp_rot[:t], wk, wv,
+                                             ocfg)[0])
+    gc.assert_close(out[:, js], {0: np.stack(ref)}, "prefill_4k sampled queries", plain_max_abs=True)
 
 
 @pytest.mark.parametrize("layer", [0, 39])
