@@ -380,3 +380,51 @@ def mla_decode_from_pool(q: np.ndarray, pool: np.ndarray, block_table: np.ndarra
         out[b] = mla_attention_absorbed(q[b], rows[:, :D_LATENT], rows[:, D_LATENT:],
                                         W_UK, W_UV, cfg)
     return out
+
+
+# ---------------------------------------------------------------- 8-bit latent cache
+#
+# [P1] section 三, 方案 A: a q8_0 KV cache ("--cache-type-k q8_0") halves the
+# bf16 cache bytes at a small precision cost.  The pages name the format only:
+# 8-bit codes with one scale per block of 32 values.  Reading taken here: the
+# 576 values of a cache row ([c_kv | rotated k_pe]) in 18 blocks of 32; each
+# block keeps a power-of-two scale 2^e, e the smallest integer with
+# 127 * 2^e >= the block's largest magnitude, clamped to [Q8_EMIN, Q8_EMAX];
+# codes are x / 2^e rounded to nearest (ties to even) and clamped to
+# [-127, 127].  A power of two (rather than q8_0's free fp16 scale) keeps every
+# dequantised value code * 2^e exact in fp16 and bf16, so the cache holds
+# exactly the values the attention consumes.
+
+Q8_BLOCK = 32                # values per scale block
+Q8_BLOCKS = (D_LATENT + D_ROPE) // Q8_BLOCK   # 18 blocks per cache row
+Q8_EMIN, Q8_EMAX = -14, 8    # scale exponent range
+
+
+def q8_block_exponent(amax: np.ndarray) -> np.ndarray:
+    """Smallest e with 127 * 2^e >= amax, clamped to [Q8_EMIN, Q8_EMAX].
+
+    Exact: with amax = m * 2^k (m in [0.5, 1)), 127 * 2^(k-7) = (127/128) 2^k is
+    enough iff m <= 127/128, and 127 * 2^(k-6) > 2^k always is.
+    """
+    amax = np.asarray(amax, dtype=np.float64)
+    m, k = np.frexp(amax)
+    e = np.where(m > 127.0 / 128.0, k - 6, k - 7)
+    e = np.where(amax > 0, e, Q8_EMIN)
+    return np.clip(e, Q8_EMIN, Q8_EMAX).astype(np.int64)
+
+
+def q8_quantize(rows: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Quantise cache rows [..., 576] -> (codes int8 [..., 576], exps int8 [..., 18])."""
+    x = np.asarray(rows, dtype=np.float64)
+    xb = x.reshape(x.shape[:-1] + (Q8_BLOCKS, Q8_BLOCK))
+    e = q8_block_exponent(np.max(np.abs(xb), axis=-1))
+    codes = np.clip(np.rint(xb / np.exp2(e.astype(np.float64))[..., None]), -127, 127)
+    return codes.reshape(x.shape).astype(np.int8), e.astype(np.int8)
+
+
+def q8_dequantize(codes: np.ndarray, exps: np.ndarray) -> np.ndarray:
+    """Values code * 2^e of quantised rows, float64 [..., 576]."""
+    c = np.asarray(codes, dtype=np.float64)
+    cb = c.reshape(c.shape[:-1] + (Q8_BLOCKS, Q8_BLOCK))
+    scale = np.exp2(np.asarray(exps, dtype=np.float64))[..., None]
+    return (cb * scale).reshape(c.shape)

@@ -480,3 +480,75 @@ def test_merge_is_associative_and_has_the_empty_part_as_identity():
     with_e = om.merge_partials([a, e])
     assert np.array_equal(with_e[0], a[0]) and np.array_equal(with_e[1], a[1])
     assert np.array_equal(with_e[2], a[2])
+
+
+# ---------------------------------------------------------------- 8-bit latent cache
+
+def _brute_exponent(amax: float) -> int:
+    # smallest e in range with 127 * 2^e >= amax, by search in exact rationals
+    from fractions import Fraction
+    a = Fraction(amax)
+    for e in range(om.Q8_EMIN, om.Q8_EMAX + 1):
+        if 127 * Fraction(2) ** e >= a:
+            return e
+    return om.Q8_EMAX
+
+
+def test_q8_exponent_matches_a_brute_force_search():
+    rng = np.random.default_rng(11)
+    amax = np.concatenate([
+        np.abs(rng.standard_normal(400)) * np.exp2(rng.integers(-20, 12, 400)),
+        # the boundaries: exactly 127 * 2^e, one ulp either side, powers of two
+        [127.0 * 2.0 ** e for e in range(-14, 9)],
+        [np.nextafter(127.0 * 2.0 ** e, np.inf) for e in range(-14, 9)],
+        [np.nextafter(127.0 * 2.0 ** e, 0.0) for e in range(-14, 9)],
+        [2.0 ** k for k in range(-20, 16)], [0.0, 1e-30, 1e6]])
+    got = om.q8_block_exponent(amax)
+    want = np.array([_brute_exponent(float(a)) for a in amax])
+    assert np.array_equal(got, want)
+
+
+def test_q8_round_trip_is_exact_on_representable_rows():
+    # a block of integers times 2^e whose largest magnitude lies in (63.5, 127]
+    # keeps exactly that exponent and comes back unchanged
+    rng = np.random.default_rng(12)
+    codes = rng.integers(-127, 128, (5, 576))
+    codes[:, ::32] = 127 * np.where(rng.random((5, 18)) < 0.5, 1, -1)
+    e = rng.integers(om.Q8_EMIN, om.Q8_EMAX + 1, (5, 18))
+    x = (codes.reshape(5, 18, 32) * np.exp2(e)[..., None]).reshape(5, 576)
+    c, ex = om.q8_quantize(x)
+    assert np.array_equal(ex, e) and np.array_equal(c, codes)
+    assert np.array_equal(om.q8_dequantize(c, ex), x)
+
+
+def test_q8_error_is_at_most_half_a_step():
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((64, 576)) * np.exp2(rng.integers(-6, 6, (64, 1)))
+    c, e = om.q8_quantize(x)
+    d = om.q8_dequantize(c, e)
+    step = np.repeat(np.exp2(e.astype(np.float64)), 32, axis=-1)
+    assert np.all(np.abs(d - x) <= 0.5 * step)
+    assert np.all(np.abs(c) <= 127)
+    # the exponent is the smallest that fits: one less would need a code > 127
+    amax = np.abs(x.reshape(64, 18, 32)).max(-1)
+    assert np.all(amax > 127 * np.exp2(e.astype(np.float64) - 1))
+
+
+def test_q8_ties_round_to_even_and_special_blocks():
+    x = np.zeros((1, 576))
+    x[0, 0] = 127.0          # block 0: e = 0
+    x[0, 1:5] = [2.5, 3.5, -2.5, -0.5]
+    x[0, 32] = 1e-9          # block 1: tiny, clamped to the smallest exponent
+    x[0, 64] = 1e9           # block 2: beyond the range, saturates
+    x[0, 65] = -1e9
+    c, e = om.q8_quantize(x)
+    assert e[0, 0] == 0 and list(c[0, 1:5]) == [2, 4, -2, 0]
+    assert e[0, 1] == om.Q8_EMIN and c[0, 32] == 0
+    assert e[0, 2] == om.Q8_EMAX and c[0, 64] == 127 and c[0, 65] == -127
+    assert e[0, 3] == om.Q8_EMIN and not c[0, 96:128].any()   # an all-zero block
+
+
+def test_q8_row_halves_the_cache_as_the_page_says():
+    # [P1] section 三, 方案 A: the q8_0 cache halves the bf16 one (12.5 GB -> ~6.3 GB).
+    # 576 one-byte codes + 18 exponent bytes against 576 bf16 values:
+    assert (576 + om.Q8_BLOCKS) / (576 * 2) == pytest.approx(6.3 / 12.5, rel=0.05)
