@@ -36,6 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "MLA decode: latent-KV HBM GB/s (% of B200 peak) and attended tokens/s"
 ROW_BYTES = 1152  # one cache row: [c_kv 512 | k_pe 64] bf16
+Q8_ROW_BYTES = 608  # one 8-bit cache row: 576 codes, 18 exponents, 14 pad bytes
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -48,6 +49,9 @@ def parse_args():
     ap.add_argument("--workload", default="decode_256k")
     ap.add_argument("--impl", default="xmla", choices=["xmla", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "q8"],
+                    help="q8: the 8-bit latent cache (int8 codes, a power-of-two scale per 32 "
+                         "values, 608 B per token; decode only)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--shards", type=int, default=0,
                     help="sequence-parallel decode over this many page shards: with --gpus G "
@@ -278,7 +282,7 @@ def traffic_record(kernel_src_sha: str, name: str):
 
 
 def roofline_line(wl, achieved, peak, peak_kind, traffic, cache_bytes, kernel_ms, flops, tpeak,
-                  tpeak_kind):
+                  tpeak_kind, q8=False):
     """The split-K kernel against the HBM roofline (decode: every cache byte read
     once) and against the tensor roofline; a prefill chunk (q_len > 8) reads a
     few MB many times from L2 and is bound by the tensor side, which then leads."""
@@ -291,7 +295,8 @@ def roofline_line(wl, achieved, peak, peak_kind, traffic, cache_bytes, kernel_ms
               "flops_per_launch": flops, "peak_source": tpeak_kind}
     rows = 32 if wl.q_len == 1 or wl.q_len > 8 or wl.max_seqlen <= 4096 else 64
     lead, other = (tensor, hbm) if wl.q_len > 8 else (hbm, tensor)
-    line = dict(lead, kernel=f"mla_decode_kernel<{rows}>", kernel_ms=round(kernel_ms, 5))
+    name = "mla_decode_q8_kernel" if q8 else f"mla_decode_kernel<{rows}>"
+    line = dict(lead, kernel=name, kernel_ms=round(kernel_ms, 5))
     line[other["bound"]] = {k: v for k, v in other.items() if k != "bound"}
     if lead is tensor:
         line["traffic"] = traffic
@@ -338,7 +343,7 @@ def run_xmla(args, wl):
     for layer in range(wl.layers):
         inp = workloads.layer_inputs(wl, layer, dev)
         prefix, new = session.split_prefix(wl, inp)
-        st = session.build_layer(cfg, wl, prefix, dev)
+        st = session.build_layer(cfg, wl, prefix, dev, cache=args.cache)
         L = {"st": st, "q": inp.q.clone(), "k_new": new.k_pe.clone(),
              "c_new": new.c_kv.clone(), "pos": new.positions.clone(),
              "sid": new.seq_ids.clone(),
@@ -357,7 +362,7 @@ def run_xmla(args, wl):
     for L, v in zip(layers, views):
         L["out"] = v
     torch.cuda.synchronize()
-    dec = session.Decoder(wl.batch, wl.q_len, wl.max_seqlen, dev)
+    dec = session.Decoder(wl.batch, wl.q_len, wl.max_seqlen, dev, cache=args.cache)
     ev_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in layers]
     for a, b in ev_attn:          # materialise the events before capture
@@ -463,7 +468,8 @@ def run_xmla(args, wl):
         e2e_ms.append(ee0[i].elapsed_time(ee1[i]))
     e2e_total = max_over_ranks(sum(e2e_ms), dev)
 
-    cache_bytes_layer = sum(wl.seqlens) * ROW_BYTES
+    q8 = args.cache == "q8"
+    cache_bytes_layer = sum(wl.seqlens) * (Q8_ROW_BYTES if q8 else ROW_BYTES)
     tokens_step = sum(wl.seqlens) * wl.layers * world
     bytes_step = cache_bytes_layer * wl.layers * world
     gbs = job_throughput(cache_bytes_layer * wl.layers, args.steps, total_ms, world)
@@ -476,24 +482,28 @@ def run_xmla(args, wl):
     attn_mean_ms = statistics.mean(attn_ms)
     achieved = cache_bytes_layer / (attn_mean_ms * 1e-3) / 1e9
     ksha = kernel_sources_sha()
-    traffic = traffic_record(ksha, wl.name)
+    traffic = None if q8 else traffic_record(ksha, wl.name)
     # per layer and step: prologue (append or producer + q absorb), split-K
-    # attention, combine
-    launches = 3 * wl.layers * args.steps
+    # attention, combine; on the 8-bit cache the append is a kernel of its own
+    launches = (4 if q8 else 3) * wl.layers * args.steps
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(gbs, 3), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16" if q8 else "bf16",
+            "data": "synthetic",
             "config": dict(workload_config(wl, world), **(
                 {"step": "hidden states in: kv_a_proj_with_mqa + RoPE + append, then decode"}
-                if args.with_producer else {})),
+                if args.with_producer else {}), **(
+                {"cache_row": "q8: 576 int8 codes + 18 power-of-two block exponents (32 values "
+                              "each), 608 B", "step": "8-bit append (quantise) + decode"}
+                if q8 else {})),
             "attended_tokens_per_s": round(tokens_step * args.steps / (total_ms * 1e-3), 1),
             "pct_of_hbm_peak": round(100.0 * gbs / (peak * world), 2),
             "roofline": roofline_line(wl, achieved, peak, peak_kind, traffic, cache_bytes_layer,
-                                      attn_mean_ms, flops_layer, tpeak, tpeak_kind),
+                                      attn_mean_ms, flops_layer, tpeak, tpeak_kind, q8),
             "e2e": {"value": round(job_throughput(cache_bytes_layer * wl.layers, args.steps,
                                                   e2e_total, world), 3),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -503,7 +513,7 @@ def run_xmla(args, wl):
         }
         if clk is not None:
             line["clocks"] = clk
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not q8:
             n, run, cores = oracle_sample(wl, args.cpu_seconds)
             t = run(n)
             line["cpu_baseline"] = {
@@ -684,6 +694,9 @@ def main():
     wl = workloads.workload(args.workload)
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.cache == "q8" and (args.with_producer or args.shards > 0 or wl.q_len > 8):
+        raise SystemExit("--cache q8 runs decode steps (q_len <= 8) without --with-producer "
+                         "or --shards")
     if args.shards > 0:
         return run_shards(args, wl)
     return run_xmla(args, wl)

@@ -221,6 +221,66 @@ xmla_status xmla_decode_profiled(const xmla_yarn_cfg* cfg, const void* q, const 
                                  int32_t* status_dev, void* out, void* stream, void* attn_start,
                                  void* attn_stop);
 
+/* ---- 8-bit latent cache ([P1] section 三, 方案 A: a q8_0 KV cache halves
+ * the bytes of the bf16 one at a small precision cost; the page names 8-bit
+ * codes with one scale per block of 32 values).
+ *
+ * Row layout (608 bytes per token, 16-byte aligned rows): bytes [0, 576) are
+ * int8 codes of [c_kv 512 | rotated k_pe 64]; bytes [576, 594) the int8
+ * exponents e of blocks 0..17 (block k = values [32k, 32k+32)); bytes
+ * [594, 608) zero.  Value = code * 2^e.  Quantisation of a bf16 row: e = the
+ * smallest integer with 127 * 2^e >= max |x| over the block, clamped to
+ * [-14, 8]; code = x / 2^e rounded to nearest (ties to even), clamped to
+ * [-127, 127].  The power-of-two scale keeps every value exact in f16.  A
+ * pool is [num_blocks, 64, 608] bytes, addressed through the block table as
+ * the bf16 pool. */
+
+/* Quantise and append T token rows: row i = [c_kv[i] | k_rot[i]] goes to
+ * block block_table[seq_ids[i]*max_blocks + positions[i]/64], row
+ * positions[i] % 64, of pool_q8, where k_rot is the YaRN RoPE of k_pe[i] at
+ * positions[i] rounded to bf16 (float64 angle, as xmla_rope_yarn), or k_pe[i]
+ * itself when rope_cfg is NULL.
+ *   pool_q8: device [num_blocks, 64, 608] bytes, 16-byte aligned;
+ *   c_kv: device bf16 [T, 512]; k_pe: device bf16 [T, 64], both 16-byte aligned;
+ *   other arguments as xmla_cache_append (rows out of range are skipped and
+ *   reported through status_dev).
+ * T == 0 is a no-op.  Errors: XMLA_ERR_INVALID_ARG, XMLA_ERR_SHAPE, XMLA_ERR_CUDA. */
+xmla_status xmla_cache_append_q8(void* pool_q8, int64_t num_blocks, const int32_t* block_table,
+                                 int32_t max_blocks, int32_t batch, const int32_t* seq_ids,
+                                 const int64_t* positions, const void* c_kv, const void* k_pe,
+                                 const xmla_yarn_cfg* rope_cfg, int64_t T, int32_t* status_dev,
+                                 void* stream);
+
+/* Workspace bytes and split count of xmla_decode_q8 (0 for unsupported sizes). */
+size_t xmla_decode_q8_workspace_size(int32_t batch, int32_t q_len, int64_t max_seqlen,
+                                     int32_t num_sms, int32_t num_splits);
+int32_t xmla_decode_q8_num_splits(int32_t batch, int32_t q_len, int64_t max_seqlen,
+                                  int32_t num_sms, int32_t num_splits);
+
+/* xmla_decode over an 8-bit pool: the same attention with c_kv and k_pe_rot
+ * the dequantised values code * 2^e of each cached row.  The products run on
+ * the tensor cores in f16 (the absorbed query rounded once to f16, the
+ * probabilities to f16, fp32 accumulation).  Arguments as xmla_decode except
+ * pool_q8 (device [num_blocks, 64, 608] bytes, 16-byte aligned) and the
+ * workspace size (xmla_decode_q8_workspace_size).  Supported: 1 <= q_len <= 8,
+ * other limits as xmla_decode.  Errors as xmla_decode. */
+xmla_status xmla_decode_q8(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
+                           const void* W_UV, const void* pool_q8, int64_t num_blocks,
+                           const int32_t* block_table, int32_t max_blocks, const int32_t* seqlens,
+                           int32_t batch, int32_t q_len, int64_t max_seqlen, float softmax_scale,
+                           int32_t num_splits, void* workspace, size_t workspace_bytes,
+                           int32_t* status_dev, void* out, void* stream);
+
+/* xmla_decode_q8 with CUDA events around its attention kernel, as
+ * xmla_decode_profiled. */
+xmla_status xmla_decode_q8_profiled(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
+                                    const void* W_UV, const void* pool_q8, int64_t num_blocks,
+                                    const int32_t* block_table, int32_t max_blocks,
+                                    const int32_t* seqlens, int32_t batch, int32_t q_len,
+                                    int64_t max_seqlen, float softmax_scale, int32_t num_splits,
+                                    void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                                    void* out, void* stream, void* attn_start, void* attn_stop);
+
 /* One decode step ([P5] MLA section; [P1] sections 一 and 二): append the
  * step's T new token rows to the cache, then attend.  The result is that of
  *   xmla_cache_append(pool, num_blocks, block_table, max_blocks, batch, seq_ids,

@@ -51,7 +51,8 @@ __device__ __forceinline__ int64_t q_ext_row(int64_t r, int h, int part, int spl
 // (griddepcontrol.wait) before reading q or seqlens: a preceding kernel may
 // have written them, and the split-K kernel relies on that wait (its producer
 // reads cache rows appended by the kernel before this one).
-template <bool kRowBlocks>
+// kF16: q_ext rows hold f16 values (one row per query row; split unused).
+template <bool kRowBlocks, bool kF16 = false>
 __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat16* q,
                                                const __nv_bfloat16* __restrict__ W_UK,
                                                const int32_t* seqlens,
@@ -76,6 +77,12 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
       rope_pair((double)__bfloat162float(x[i]), (double)__bfloat162float(x[i + kPairs]), pos, i,
                 tab, &y1, &y2);
       const double v1 = y1 * (double)qscale, v2 = y2 * (double)qscale;
+      if constexpr (kF16) {
+        __half* o = reinterpret_cast<__half*>(q_ext) + ((int64_t)r * kHeads + h) * kDRow + kDLatent;
+        o[i] = __double2half(v1);
+        o[i + kPairs] = __double2half(v2);
+        continue;
+      }
       const __nv_bfloat16 h1 = __double2bfloat16(v1), h2 = __double2bfloat16(v2);
       __nv_bfloat16* o = q_ext + q_ext_row(r, h, 0, split) * kDRow + kDLatent;
       o[i] = h1;
@@ -129,6 +136,11 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
 #pragma unroll
       for (int k = 0; k < 16; ++k) s += part[k][r][col];
       const float v = s * qscale;
+      if constexpr (kF16) {
+        reinterpret_cast<__half*>(q_ext)[((int64_t)(r0 + r) * kHeads + h) * kDRow + cb * 64 + col] =
+            __float2half_rn(v);
+        continue;
+      }
       const __nv_bfloat16 hi = __float2bfloat16_rn(v);
       q_ext[q_ext_row(r0 + r, h, 0, split) * kDRow + cb * 64 + col] = hi;
       if (split)
@@ -262,7 +274,7 @@ struct AbsorbGrid {
   }
 };
 
-template <bool kPlan, int kRows>
+template <bool kPlan, int kRows, bool kF16 = false>
 __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
     const __nv_bfloat16* q, const __nv_bfloat16* __restrict__ W_UK, const int32_t* seqlens,
     __nv_bfloat16* __restrict__ q_ext, int rows, int q_len, int split, float qscale,
@@ -282,8 +294,8 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
   }
   int h, cb, r_lo, r_hi;
   G::map(blockIdx.x, rows, h, cb, r_lo, r_hi);
-  q_absorb_block<kRows != 0>(h, cb, q, W_UK, seqlens, q_ext, rows, q_len, split, qscale, tab,
-                             sm.absorb, r_lo, r_hi);
+  q_absorb_block<kRows != 0, kF16>(h, cb, q, W_UK, seqlens, q_ext, rows, q_len, split, qscale,
+                                   tab, sm.absorb, r_lo, r_hi);
 }
 
 // The first kernel of a decode step: the absorb blocks above, then the
@@ -342,11 +354,24 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
                             int split, float qscale, const RopeTable& tab,
-                            const WorkPlanArgs* plan, bool rope_only, cudaStream_t st) {
+                            const WorkPlanArgs* plan, bool rope_only, cudaStream_t st,
+                            bool f16) {
   const int mode = rope_only ? 2 : rows > kAbsorbRows ? 1 : 0;
   const int64_t nrb = (rows + kAbsorbRows - 1) / kAbsorbRows;
   const unsigned absorb_blocks =
       (unsigned)(mode == 2 ? kHeads * nrb : mode == 1 ? kAbsorbBlocks * nrb : kAbsorbBlocks);
+  if (f16) {
+    if (mode == 2) return cudaErrorInvalidValue;
+    if (plan != nullptr) {
+      if (!plan_ok(*plan)) return cudaErrorInvalidValue;
+      return launch_pdl(mode == 1 ? q_absorb_kernel<true, 1, true> : q_absorb_kernel<true, 0, true>,
+                        dim3(absorb_blocks + 1), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens,
+                        q_ext, rows, q_len, 0, qscale, tab, *plan);
+    }
+    return launch_pdl(mode == 1 ? q_absorb_kernel<false, 1, true> : q_absorb_kernel<false, 0, true>,
+                      dim3(absorb_blocks), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext,
+                      rows, q_len, 0, qscale, tab, WorkPlanArgs{});
+  }
   auto kern = [&](bool with_plan) {
     if (with_plan)
       return mode == 2 ? q_absorb_kernel<true, 2> : mode == 1 ? q_absorb_kernel<true, 1>

@@ -46,10 +46,12 @@ struct WorkPlanArgs {
 // split_q layout).  plan (nullable): also compute the length-aware plan.
 // rope_only: only the rope columns (the latent part comes from
 // launch_absorb_gemm).
+// f16: q_ext holds f16 values (single rows) for the 8-bit cache's kernel.
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
                             int split, float qscale, const RopeTable& tab,
-                            const WorkPlanArgs* plan, bool rope_only, cudaStream_t st);
+                            const WorkPlanArgs* plan, bool rope_only, cudaStream_t st,
+                            bool f16 = false);
 
 // The new tokens of a decode step, appended by step_prologue_kernel.
 struct AppendArgs {
@@ -119,5 +121,19 @@ cudaError_t launch_latent_out(const float* part_o, const float* part_ml, __nv_bf
 cudaError_t launch_merge_splits(const float* part_o, const float* part_ml, float* out, int rows,
                                 int q_len, int groups, int nsplit, int rows_per_cta,
                                 cudaStream_t st);
+
+// Quantise and append T cache rows to the 8-bit pool ([num_blocks, 64, 608]
+// bytes, layout in q8_append.cu); rotate: RoPE the rope key with tab first.
+cudaError_t launch_cache_append_q8(uint8_t* pool, int64_t num_blocks, const int32_t* block_table,
+                                   int32_t max_blocks, int32_t batch, const int32_t* seq_ids,
+                                   const int64_t* positions, const __nv_bfloat16* c_kv,
+                                   const __nv_bfloat16* k_pe, int32_t* status, int rotate,
+                                   const RopeTable& tab, int64_t T, cudaStream_t st);
+
+// Split-K attention over the 8-bit pool (dp.pool_q8), 32 rows per CTA, f16
+// q_ext (q_map as for launch_split_kv with 32-row boxes); writes the same
+// partials as launch_split_kv.
+cudaError_t launch_split_kv_q8(const CUtensorMap& q_map, const DecodeParams& dp, int64_t items,
+                               cudaStream_t st);
 
 }  // namespace xmla

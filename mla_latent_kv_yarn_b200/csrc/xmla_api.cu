@@ -59,15 +59,16 @@ static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // several sequences with automatic splits gets the length-aware plan: one
 // CTA per SM, the pages of each sequence divided over them in proportion to
 // its length by the first kernel of the call.
+// q8: the 8-bit cache's kernel (32 rows per CTA, one f16 query row each).
 static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_sms,
                       int32_t num_splits, Plan* pl, int64_t span_pages = 0,
-                      bool allow_table = true) {
-  if (B < 1 || q_len < 1 || q_len > kMaxQLen || max_seqlen < q_len ||
+                      bool allow_table = true, bool q8 = false) {
+  if (B < 1 || q_len < 1 || q_len > (q8 ? kQ8MaxQLen : kMaxQLen) || max_seqlen < q_len ||
       max_seqlen > (int64_t)0x7fffffff - kPage || num_sms < 1 || num_splits < 0 || span_pages < 0)
     return false;
   Plan P;
-  P.split = max_seqlen <= kSplitQMaxSeqlen || q_len > kSplitQMinChunk;
-  P.nr = P.split || q_len == 1 ? 32 : 64;
+  P.split = !q8 && (max_seqlen <= kSplitQMaxSeqlen || q_len > kSplitQMinChunk);
+  P.nr = q8 || P.split || q_len == 1 ? 32 : 64;
   P.groups = (q_len * 32 + P.nr - 1) / P.nr;
   int64_t max_pages = (max_seqlen + kPage - 1) / kPage;
   if (span_pages > 0 && span_pages < max_pages) max_pages = span_pages;
@@ -96,7 +97,7 @@ static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_
   P.off_wtab = align_up(P.off_ml + (size_t)P.items * P.nr * 2 * 4, 1024);
   P.off_utab = align_up(P.off_wtab + (P.table ? (size_t)P.items * 16 : 0), 256);
   // a prompt chunk's merged latent output, hi and lo bf16 [rows, 32, 512] each
-  P.gemm = allow_table && q_len > kSplitQMinChunk;
+  P.gemm = !q8 && allow_table && q_len > kSplitQMinChunk;
   P.off_olat = align_up(P.off_utab + (P.table ? (size_t)units * 8 : 0), 1024);
   const size_t olat = P.gemm ? (size_t)B * q_len * kHeads * kDLatent * 2 : 0;
   P.bytes = align_up(P.off_olat + 2 * olat, 1024);
@@ -208,7 +209,7 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
                               void* out, void* stream, void* attn_start, void* attn_stop,
                               const AppendArgs* ap, const ProduceArgs* pa = nullptr,
                               int64_t page_lo = 0, int64_t page_hi = INT64_MAX,
-                              float* shard_partial = nullptr) {
+                              float* shard_partial = nullptr, bool q8 = false) {
   if (q == nullptr || W_UK == nullptr || W_UV == nullptr || pool == nullptr ||
       block_table == nullptr || seqlens == nullptr || workspace == nullptr || out == nullptr)
     return XMLA_ERR_INVALID_ARG;
@@ -226,7 +227,11 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   if (!device_ok(&nsm)) return XMLA_ERR_UNSUPPORTED;
   Plan P;
   const int64_t span = page_hi == INT64_MAX ? 0 : (page_hi > page_lo ? page_hi - page_lo : 1);
-  if (!make_plan(batch, q_len, max_seqlen, nsm, num_splits, &P, span, shard_partial == nullptr))
+  if (q8 && (ap != nullptr || pa != nullptr || shard_partial != nullptr || page_lo != 0 ||
+             page_hi != INT64_MAX))
+    return XMLA_ERR_INVALID_ARG;
+  if (!make_plan(batch, q_len, max_seqlen, nsm, num_splits, &P, span, shard_partial == nullptr,
+                 q8))
     return XMLA_ERR_SHAPE;
   if (workspace_bytes < P.bytes) return XMLA_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
@@ -235,7 +240,8 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   const int rows = batch * q_len;
 
   CUtensorMap tmap_pool, tmap_q;
-  if (!encode_rows576(&tmap_pool, pool, (uint64_t)num_blocks * kPage, kPage)) return XMLA_ERR_CUDA;
+  if (!q8 && !encode_rows576(&tmap_pool, pool, (uint64_t)num_blocks * kPage, kPage))
+    return XMLA_ERR_CUDA;
   // the QK product's B tile: 64 rows (32 heads hi then lo when split, 32 heads of one query
   // at 32 rows per CTA, else 2 queries x 32 heads)
   if (!encode_rows576(&tmap_q, q_ext, (uint64_t)rows * kHeads * (P.split ? 2 : 1),
@@ -287,7 +293,7 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
                                  P.table ? &plan : nullptr, P.gemm, st)
           : launch_q_absorb((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
                             rows, q_len, P.split ? 1 : 0, qscale, tab,
-                            P.table ? &plan : nullptr, P.gemm, st);
+                            P.table ? &plan : nullptr, P.gemm, st, q8);
   if (e0 != cudaSuccess) return XMLA_ERR_CUDA;
   if (P.gemm && launch_absorb_gemm(tmap_qin, tmap_wuk, gp, st) != cudaSuccess) return XMLA_ERR_CUDA;
 
@@ -313,9 +319,11 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   const bool direct = P.gemm && P.split && P.nsplit == 1 && !P.table && shard_partial == nullptr;
   dp.o_hi = direct ? o_hi : nullptr;
   dp.o_lo = direct ? o_lo : nullptr;
+  dp.pool_q8 = q8 ? (const uint8_t*)pool : nullptr;
   if (record_event(attn_start, st) != cudaSuccess) return XMLA_ERR_CUDA;
-  if (launch_split_kv(P.nr, P.split, tmap_pool, tmap_q, dp, P.items, st) != cudaSuccess)
-    return XMLA_ERR_CUDA;
+  const cudaError_t ea = q8 ? launch_split_kv_q8(tmap_q, dp, P.items, st)
+                            : launch_split_kv(P.nr, P.split, tmap_pool, tmap_q, dp, P.items, st);
+  if (ea != cudaSuccess) return XMLA_ERR_CUDA;
   if (record_event(attn_stop, st) != cudaSuccess) return XMLA_ERR_CUDA;
   if (shard_partial != nullptr) {
     const cudaError_t em = launch_merge_splits(dp.part_o, dp.part_ml, shard_partial, rows, q_len,
@@ -422,6 +430,73 @@ extern "C" xmla_status xmla_decode(const xmla_yarn_cfg* cfg, const void* q, cons
 }
 
 // ---------------------------------------------------------------- sequence-parallel decode
+
+// ---------------------------------------------------------------- 8-bit latent cache
+
+extern "C" size_t xmla_decode_q8_workspace_size(int32_t batch, int32_t q_len, int64_t max_seqlen,
+                                                int32_t num_sms, int32_t num_splits) {
+  Plan P;
+  return make_plan(batch, q_len, max_seqlen, num_sms, num_splits, &P, 0, true, true) ? P.bytes
+                                                                                      : 0;
+}
+
+extern "C" int32_t xmla_decode_q8_num_splits(int32_t batch, int32_t q_len, int64_t max_seqlen,
+                                             int32_t num_sms, int32_t num_splits) {
+  Plan P;
+  return make_plan(batch, q_len, max_seqlen, num_sms, num_splits, &P, 0, true, true) ? P.nsplit
+                                                                                      : 0;
+}
+
+extern "C" xmla_status xmla_cache_append_q8(void* pool_q8, int64_t num_blocks,
+                                            const int32_t* block_table, int32_t max_blocks,
+                                            int32_t batch, const int32_t* seq_ids,
+                                            const int64_t* positions, const void* c_kv,
+                                            const void* k_pe, const xmla_yarn_cfg* rope_cfg,
+                                            int64_t T, int32_t* status_dev, void* stream) {
+  if (T < 0 || num_blocks < 1 || max_blocks < 1 || batch < 1) return XMLA_ERR_SHAPE;
+  if (T == 0) return XMLA_OK;
+  if (pool_q8 == nullptr || block_table == nullptr || seq_ids == nullptr || positions == nullptr ||
+      c_kv == nullptr || k_pe == nullptr)
+    return XMLA_ERR_INVALID_ARG;
+  if ((((uintptr_t)pool_q8) | ((uintptr_t)c_kv) | ((uintptr_t)k_pe)) & 15u)
+    return XMLA_ERR_INVALID_ARG;
+  RopeTable tab = {};
+  if (rope_cfg != nullptr) {
+    if (!yarn_cfg_ok(rope_cfg)) return XMLA_ERR_INVALID_ARG;
+    if (rope_cfg->rotary_dim != kDRope) return XMLA_ERR_SHAPE;
+    tab = make_rope_table(rope_cfg);
+  }
+  const cudaError_t e = launch_cache_append_q8(
+      (uint8_t*)pool_q8, num_blocks, block_table, max_blocks, batch, seq_ids, positions,
+      (const __nv_bfloat16*)c_kv, (const __nv_bfloat16*)k_pe, status_dev,
+      rope_cfg != nullptr ? 1 : 0, tab, T, (cudaStream_t)stream);
+  return e == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+}
+
+extern "C" xmla_status xmla_decode_q8_profiled(
+    const xmla_yarn_cfg* cfg, const void* q, const void* W_UK, const void* W_UV,
+    const void* pool_q8, int64_t num_blocks, const int32_t* block_table, int32_t max_blocks,
+    const int32_t* seqlens, int32_t batch, int32_t q_len, int64_t max_seqlen, float softmax_scale,
+    int32_t num_splits, void* workspace, size_t workspace_bytes, int32_t* status_dev, void* out,
+    void* stream, void* attn_start, void* attn_stop) {
+  return run_decode(cfg, q, W_UK, W_UV, pool_q8, num_blocks, block_table, max_blocks, seqlens,
+                    batch, q_len, max_seqlen, softmax_scale, num_splits, workspace,
+                    workspace_bytes, status_dev, out, stream, attn_start, attn_stop, nullptr,
+                    nullptr, 0, INT64_MAX, nullptr, true);
+}
+
+extern "C" xmla_status xmla_decode_q8(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,
+                                      const void* W_UV, const void* pool_q8, int64_t num_blocks,
+                                      const int32_t* block_table, int32_t max_blocks,
+                                      const int32_t* seqlens, int32_t batch, int32_t q_len,
+                                      int64_t max_seqlen, float softmax_scale, int32_t num_splits,
+                                      void* workspace, size_t workspace_bytes,
+                                      int32_t* status_dev, void* out, void* stream) {
+  return xmla_decode_q8_profiled(cfg, q, W_UK, W_UV, pool_q8, num_blocks, block_table,
+                                 max_blocks, seqlens, batch, q_len, max_seqlen, softmax_scale,
+                                 num_splits, workspace, workspace_bytes, status_dev, out, stream,
+                                 nullptr, nullptr);
+}
 
 extern "C" size_t xmla_shard_partial_floats(int32_t batch, int32_t q_len) {
   if (batch < 1 || q_len < 1 || q_len > kMaxQLen) return 0;

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <utility>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/xmla.h"
@@ -20,6 +21,14 @@ constexpr int kDV = 128;
 constexpr int kDQ = kDNope + kDRope;      // 192
 constexpr int kDRow = kDLatent + kDRope;  // 576 bf16 per cache row
 constexpr int kPage = 64;                 // tokens per cache block
+// 8-bit cache row: 576 int8 codes, then 18 int8 block exponents (blocks of 32
+// values, value = code * 2^e), then 14 zero bytes: 608 B, a multiple of 16
+constexpr int kQ8Block = 32;
+constexpr int kQ8Blocks = kDRow / kQ8Block;  // 18
+constexpr int kQ8Row = 608;
+constexpr int kQ8EMin = -14;
+constexpr int kQ8EMax = 8;
+constexpr int kQ8MaxQLen = 8;  // queries per sequence and call on the 8-bit cache
 constexpr int kMaxQLen = 65536;  // new tokens per sequence and call (decode steps to prefill chunks)
 
 // Default limit of one bounded wait inside a kernel (nanoseconds).
@@ -333,6 +342,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | ((b_mn_major ? 1u : 0u) << 16)    // B major
          | ((uint32_t)(N >> 3) << 17)        // N / 8
          | ((uint32_t)(M >> 4) << 24);       // M / 16
+}
+
+// The same for f16 A/B (format code 0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major,
+                                                     bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // Launch with programmatic stream serialization allowed (PDL): the kernel may

@@ -29,6 +29,8 @@ EXPORTS = [
     "xmla_decode_profiled", "xmla_decode_step", "xmla_decode_noalloc",
     "xmla_shard_partial_floats", "xmla_decode_shard_workspace_size", "xmla_decode_shard",
     "xmla_combine_shards",
+    "xmla_cache_append_q8", "xmla_decode_q8_workspace_size", "xmla_decode_q8_num_splits",
+    "xmla_decode_q8", "xmla_decode_q8_profiled",
     "xmla_selftest_wait_timeout",
     "xmla_status_string",
 ]
@@ -106,6 +108,16 @@ def lib() -> ctypes.CDLL:
         L.xmla_decode_shard.restype = ctypes.c_int
         L.xmla_combine_shards.argtypes = [vp, i32, vp, i32, i32, vp, vp]
         L.xmla_combine_shards.restype = ctypes.c_int
+        L.xmla_cache_append_q8.argtypes = L.xmla_cache_append.argtypes
+        L.xmla_cache_append_q8.restype = ctypes.c_int
+        L.xmla_decode_q8_workspace_size.argtypes = [i32, i32, i64, i32, i32]
+        L.xmla_decode_q8_workspace_size.restype = sz
+        L.xmla_decode_q8_num_splits.argtypes = [i32, i32, i64, i32, i32]
+        L.xmla_decode_q8_num_splits.restype = i32
+        L.xmla_decode_q8.argtypes = L.xmla_decode.argtypes
+        L.xmla_decode_q8.restype = ctypes.c_int
+        L.xmla_decode_q8_profiled.argtypes = L.xmla_decode_profiled.argtypes
+        L.xmla_decode_q8_profiled.restype = ctypes.c_int
         L.xmla_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
         L.xmla_selftest_wait_timeout.restype = ctypes.c_int
         L.xmla_status_string.argtypes = [ctypes.c_int]
@@ -295,6 +307,57 @@ def xmla_combine_shards(partials, num_shards, W_UV, batch, q_len, out, stream=No
     _check(lib().xmla_combine_shards(_ptr(partials), int(num_shards), _ptr(W_UV), int(batch),
                                      int(q_len), _ptr(out), _stream(stream)),
            "xmla_combine_shards")
+
+
+def xmla_cache_append_q8(pool_q8: torch.Tensor, num_blocks: int, block_table: torch.Tensor,
+                         max_blocks: int, batch: int, seq_ids: torch.Tensor,
+                         positions: torch.Tensor, c_kv: torch.Tensor, k_pe: torch.Tensor,
+                         rope_cfg: xmla_yarn_cfg | None, T: int,
+                         status: torch.Tensor | None = None, stream=None) -> None:
+    _check(lib().xmla_cache_append_q8(_ptr(pool_q8), int(num_blocks), _ptr(block_table),
+                                      int(max_blocks), int(batch), _ptr(seq_ids), _ptr(positions),
+                                      _ptr(c_kv), _ptr(k_pe),
+                                      None if rope_cfg is None else ctypes.byref(rope_cfg), int(T),
+                                      _ptr(status), _stream(stream)),
+           "xmla_cache_append_q8")
+
+
+def xmla_decode_q8_workspace_size(batch: int, q_len: int, max_seqlen: int, num_sms: int,
+                                  num_splits: int = 0) -> int:
+    return int(lib().xmla_decode_q8_workspace_size(int(batch), int(q_len), int(max_seqlen),
+                                                   int(num_sms), int(num_splits)))
+
+
+def xmla_decode_q8_num_splits(batch: int, q_len: int, max_seqlen: int, num_sms: int,
+                              num_splits: int = 0) -> int:
+    return int(lib().xmla_decode_q8_num_splits(int(batch), int(q_len), int(max_seqlen),
+                                               int(num_sms), int(num_splits)))
+
+
+def xmla_decode_q8(cfg, q, W_UK, W_UV, pool_q8, num_blocks, block_table, max_blocks, seqlens,
+                   batch, q_len, max_seqlen, softmax_scale, num_splits, workspace,
+                   workspace_bytes, status, out, stream=None) -> None:
+    _check(lib().xmla_decode_q8(ctypes.byref(cfg), _ptr(q), _ptr(W_UK), _ptr(W_UV), _ptr(pool_q8),
+                                int(num_blocks), _ptr(block_table), int(max_blocks),
+                                _ptr(seqlens), int(batch), int(q_len), int(max_seqlen),
+                                float(softmax_scale), int(num_splits), _ptr(workspace),
+                                int(workspace_bytes), _ptr(status), _ptr(out), _stream(stream)),
+           "xmla_decode_q8")
+
+
+def xmla_decode_q8_profiled(cfg, q, W_UK, W_UV, pool_q8, num_blocks, block_table, max_blocks,
+                            seqlens, batch, q_len, max_seqlen, softmax_scale, num_splits,
+                            workspace, workspace_bytes, status, out, stream=None,
+                            attn_start=None, attn_stop=None) -> None:
+    ev = [None if e is None else (e.cuda_event if hasattr(e, "cuda_event") else int(e))
+          for e in (attn_start, attn_stop)]
+    _check(lib().xmla_decode_q8_profiled(ctypes.byref(cfg), _ptr(q), _ptr(W_UK), _ptr(W_UV),
+                                         _ptr(pool_q8), int(num_blocks), _ptr(block_table),
+                                         int(max_blocks), _ptr(seqlens), int(batch), int(q_len),
+                                         int(max_seqlen), float(softmax_scale), int(num_splits),
+                                         _ptr(workspace), int(workspace_bytes), _ptr(status),
+                                         _ptr(out), _stream(stream), ev[0], ev[1]),
+           "xmla_decode_q8_profiled")
 
 
 def xmla_selftest_wait_timeout(status: torch.Tensor, timeout_ns: int, stream=None) -> None:

@@ -31,13 +31,15 @@ def f64(t: torch.Tensor) -> np.ndarray:
 
 
 def gpu_step(wl: workloads.Workload, inp: workloads.LayerInputs, cfg, *, num_splits: int = 0,
-             pool_fill=0.0, decoder: session.Decoder | None = None, fused: bool = True):
+             pool_fill=0.0, decoder: session.Decoder | None = None, fused: bool = True,
+             cache: str = "bf16"):
     """Fill the cache with every token but each sequence's q_len newest, then run
     one decode step (RoPE q, RoPE + append the new tokens, decode)."""
     dev = torch.device("cuda")
     prefix, new = session.split_prefix(wl, inp)
-    st = session.build_layer(cfg, wl, prefix, dev, pool_fill=pool_fill)
-    dec = decoder or session.Decoder(wl.batch, wl.q_len, wl.max_seqlen, dev, num_splits)
+    st = session.build_layer(cfg, wl, prefix, dev, pool_fill=pool_fill, cache=cache)
+    dec = decoder or session.Decoder(wl.batch, wl.q_len, wl.max_seqlen, dev, num_splits,
+                                     cache=cache)
     q = inp.q.to(dev).clone()
     out = dec.step(cfg, st, q, new.c_kv.to(dev), new.k_pe.to(dev).clone(), new.positions.to(dev),
                    new.seq_ids.to(dev), xmla.xmla_softmax_scale(cfg, 192), fused=fused)

@@ -69,6 +69,12 @@ def test_workspace_plan(x):
     assert x.xmla_decode_workspace_size(1, 4096, 4096, 148) > 0     # a prefill chunk
     assert x.xmla_decode_workspace_size(0, 1, 4096, 148) == 0
     assert x.xmla_decode_workspace_size(1, 4, 3, 148) == 0         # max_seqlen < q_len
+    # the 8-bit cache: 32 rows per CTA at any q_len <= 8, one f16 query row each
+    assert x.xmla_decode_q8_num_splits(1, 1, 262144, 148) == 148
+    assert x.xmla_decode_q8_num_splits(8, 4, 131072, 148) == 4     # 32 (seq, query) units
+    assert x.xmla_decode_q8_workspace_size(1, 1, 262144, 148) == ws
+    assert x.xmla_decode_q8_workspace_size(1, 8, 4096, 148) > 0
+    assert x.xmla_decode_q8_workspace_size(1, 9, 4096, 148) == 0   # q_len > 8
 
 
 def test_argument_validation_without_gpu(x):
@@ -88,6 +94,13 @@ def test_argument_validation_without_gpu(x):
     assert L.xmla_rope_yarn(ctypes.byref(bad), None, 1, 1, 64, 64, 0, None, None) == 2
     assert L.xmla_cache_append(None, 4, None, 1, 1, None, None, None, None, None, 0, None, None) == 0
     assert L.xmla_cache_append(None, 4, None, 1, 1, None, None, None, None, None, 3, None, None) == 1
+    assert L.xmla_cache_append_q8(None, 4, None, 1, 1, None, None, None, None, None, 0, None,
+                                  None) == 0
+    assert L.xmla_cache_append_q8(None, 4, None, 1, 1, None, None, None, None, None, 3, None,
+                                  None) == 1
+    st = L.xmla_decode_q8(ctypes.byref(cfg), None, None, None, None, 1, None, 1, None, 1, 1, 64,
+                          0.1, 0, None, 0, None, None, None)
+    assert st == 1
     assert L.xmla_selftest_wait_timeout(None, 1000, None) == 1
     for code in range(8):
         assert x.xmla_status_string(code)
