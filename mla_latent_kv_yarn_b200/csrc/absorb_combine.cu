@@ -150,6 +150,51 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
   }
 }
 
+// Rope columns of q_ext for the rows [r_lo, r_hi) (at most kRopeRows) of all 32
+// heads, for a prompt chunk whose latent columns come from the tensor-core
+// absorb.  The rotation angle depends only on the position and the pair, so the
+// block forms cos and sin once per (row, pair) -- float64, the same arithmetic as
+// rope_pair -- and applies them to every head.
+__device__ __forceinline__ void q_rope_rows_block(int r_lo, int r_hi, const __nv_bfloat16* q,
+                                                  const int32_t* seqlens,
+                                                  __nv_bfloat16* __restrict__ q_ext, int q_len,
+                                                  int split, float qscale, const RopeTable& tab,
+                                                  AbsorbSmem& sm) {
+  constexpr int kPairs = kDRope / 2;
+  static_assert(sizeof(sm.sq) >= 2 * sizeof(double) * 4 * kPairs, "cos/sin table");
+  double* cs = reinterpret_cast<double*>(&sm.sq[0][0]);  // [row][pair] (cos, sin)
+  const int t = threadIdx.x;
+  const int nr = r_hi - r_lo;
+  pdl_wait();
+  if (t < nr * kPairs) {
+    const int r = r_lo + t / kPairs, i = t % kPairs;
+    const int64_t pos = (int64_t)seqlens[r / q_len] - q_len + (r % q_len);
+    double sn, c;
+    sincos((double)pos * tab.inv_freq[i], &sn, &c);
+    cs[2 * t] = c * tab.magnitude;
+    cs[2 * t + 1] = sn * tab.magnitude;
+  }
+  __syncthreads();
+  for (int e = t; e < nr * kHeads * kPairs; e += kAbsorbThreads) {
+    const int rr = e / (kHeads * kPairs), h = (e / kPairs) % kHeads, i = e % kPairs;
+    const int r = r_lo + rr;
+    const double c = cs[2 * (rr * kPairs + i)], sn = cs[2 * (rr * kPairs + i) + 1];
+    const __nv_bfloat16* x = q + ((int64_t)r * kHeads + h) * kDQ + kDNope;
+    const double x1 = (double)__bfloat162float(x[i]), x2 = (double)__bfloat162float(x[i + kPairs]);
+    const double v1 = (x1 * c - x2 * sn) * (double)qscale;
+    const double v2 = (x2 * c + x1 * sn) * (double)qscale;
+    const __nv_bfloat16 h1 = __double2bfloat16(v1), h2 = __double2bfloat16(v2);
+    __nv_bfloat16* o = q_ext + q_ext_row(r, h, 0, split) * kDRow + kDLatent;
+    o[i] = h1;
+    o[i + kPairs] = h2;
+    if (split) {
+      __nv_bfloat16* ol = q_ext + q_ext_row(r, h, 1, split) * kDRow + kDLatent;
+      ol[i] = __double2bfloat16(v1 - (double)__bfloat162float(h1));
+      ol[i + kPairs] = __double2bfloat16(v2 - (double)__bfloat162float(h2));
+    }
+  }
+}
+
 // ---------------------------------------------------------------- length-aware split plan
 
 // Sum (kMax false) or maximum over the 128 threads of a block, returned to all.
@@ -255,12 +300,17 @@ static bool plan_ok(const WorkPlanArgs& plan) {
 // griddepcontrol.wait (a preceding kernel may have written them).
 // kPlan: one more block computes the length-aware plan (batch > 1).
 // kRows: 0 = every absorb block takes all rows; 1 = kAbsorbRows query rows each
-// (kAbsorbBlocks blocks per kAbsorbRows rows); 2 = the same for the rope blocks
-// only (a prompt chunk, whose latent part the tensor-core absorb computes).
+// (kAbsorbBlocks blocks per kAbsorbRows rows); 2 = the rope columns only, kRopeRows
+// rows of all heads per block (a prompt chunk, whose latent part the tensor-core
+// absorb computes).
+// Mode 2 blocks take kRopeRows rows of all 32 heads each (q_rope_rows_block).
+constexpr int kRopeRows = 4;
+
 template <int kRows>
 struct AbsorbGrid {
   static constexpr int kPerRows = kRows == 2 ? kHeads : kAbsorbBlocks;
-  __device__ __forceinline__ static int blocks(int rows) {
+  __host__ __device__ __forceinline__ static int blocks(int rows) {
+    if constexpr (kRows == 2) return (rows + kRopeRows - 1) / kRopeRows;
     return kRows ? kPerRows * ((rows + kAbsorbRows - 1) / kAbsorbRows) : kAbsorbBlocks;
   }
   // block -> (head, column block, first row, end row)
@@ -292,6 +342,12 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
       return;
     }
   }
+  if constexpr (kRows == 2) {
+    const int r_lo = blockIdx.x * kRopeRows;
+    q_rope_rows_block(r_lo, min(rows, r_lo + kRopeRows), q, seqlens, q_ext, q_len, split, qscale,
+                      tab, sm.absorb);
+    return;
+  }
   int h, cb, r_lo, r_hi;
   G::map(blockIdx.x, rows, h, cb, r_lo, r_hi);
   q_absorb_block<kRows != 0, kF16>(h, cb, q, W_UK, seqlens, q_ext, rows, q_len, split, qscale,
@@ -321,6 +377,12 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
   using G = AbsorbGrid<kRows>;
   const int absorb_blocks = G::blocks(rows);
   if (blockIdx.x < absorb_blocks) {
+    if constexpr (kRows == 2) {
+      const int r_lo = blockIdx.x * kRopeRows;
+      q_rope_rows_block(r_lo, min(rows, r_lo + kRopeRows), q, seqlens, q_ext, q_len, split,
+                        qscale, q_tab, sm.absorb);
+      return;
+    }
     int h, cb, r_lo, r_hi;
     G::map(blockIdx.x, rows, h, cb, r_lo, r_hi);
     q_absorb_block<kRows != 0>(h, cb, q, W_UK, seqlens, q_ext, rows, q_len, split, qscale, q_tab,
@@ -359,7 +421,8 @@ cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
   const int mode = rope_only ? 2 : rows > kAbsorbRows ? 1 : 0;
   const int64_t nrb = (rows + kAbsorbRows - 1) / kAbsorbRows;
   const unsigned absorb_blocks =
-      (unsigned)(mode == 2 ? kHeads * nrb : mode == 1 ? kAbsorbBlocks * nrb : kAbsorbBlocks);
+      (unsigned)(mode == 2 ? AbsorbGrid<2>::blocks(rows)
+                           : mode == 1 ? kAbsorbBlocks * nrb : kAbsorbBlocks);
   if (f16) {
     if (mode == 2) return cudaErrorInvalidValue;
     if (plan != nullptr) {
@@ -401,8 +464,9 @@ cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_
   const int64_t prod_blocks = p.T > 0 ? kProdBlocks : 0;
   const int mode = rope_only ? 2 : rows > kAbsorbRows ? 1 : 0;
   const int64_t nrb = (rows + kAbsorbRows - 1) / kAbsorbRows;
-  const int64_t absorb_blocks =
-      mode == 2 ? kHeads * nrb : mode == 1 ? (int64_t)kAbsorbBlocks * nrb : kAbsorbBlocks;
+  const int64_t absorb_blocks = mode == 2   ? (int64_t)AbsorbGrid<2>::blocks(rows)
+                               : mode == 1 ? (int64_t)kAbsorbBlocks * nrb
+                                           : kAbsorbBlocks;
   auto kern = [&](bool with_plan) {
     if (with_plan)
       return mode == 2 ? step_prologue_kernel<true, 2>
