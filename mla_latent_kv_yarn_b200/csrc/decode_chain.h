@@ -130,10 +130,12 @@ cudaError_t launch_cache_append_q8(uint8_t* pool, int64_t num_blocks, const int3
                                    const __nv_bfloat16* k_pe, int32_t* status, int rotate,
                                    const RopeTable& tab, int64_t T, cudaStream_t st);
 
-// Split-K attention over the 8-bit pool (dp.pool_q8), 32 rows per CTA, f16
-// q_ext (q_map as for launch_split_kv with 32-row boxes); writes the same
-// partials as launch_split_kv.
-cudaError_t launch_split_kv_q8(const CUtensorMap& q_map, const DecodeParams& dp, int64_t items,
-                               cudaStream_t st);
+// Split-K attention over the 8-bit pool ([num_blocks, 64, 608] bytes), 32 rows
+// per CTA, f16 q_ext (q_map as for launch_split_kv with 32-row boxes); writes
+// the same partials as launch_split_kv.  (The pool pointer is an argument of
+// its own: DecodeParams is the bf16 kernel's parameter block, whose code
+// generation has proven sensitive to its layout.)
+cudaError_t launch_split_kv_q8(const CUtensorMap& q_map, const DecodeParams& dp,
+                               const uint8_t* pool_q8, int64_t items, cudaStream_t st);
 
 }  // namespace xmla

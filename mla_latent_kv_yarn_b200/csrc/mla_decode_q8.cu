@@ -138,7 +138,8 @@ __device__ __forceinline__ void q8_to_f16x4(uint32_t w, __half2 scale, uint32_t&
 
 template <int kMode>
 __global__ void __launch_bounds__(kQ8Threads, 1)
-    mla_decode_q8_kernel(const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p) {
+    mla_decode_q8_kernel(const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p,
+                         const uint8_t* __restrict__ pool_q8) {
   using L = Q8Layout;
   constexpr int NR = L::NR;
   extern __shared__ uint8_t smem_raw[];
@@ -244,7 +245,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     auto page_ptr = [&](int i, bool& valid) -> const uint8_t* {
       const int32_t blk = bt[i];
       valid = blk >= 0 && (int64_t)blk < p.num_blocks;
-      return p.pool_q8 + (int64_t)(valid ? blk : 0) * kQ8PageBytes;
+      return pool_q8 + (int64_t)(valid ? blk : 0) * kQ8PageBytes;
     };
     if (cw == 0 && lane == 0) {
       // the cache pages are final once the kernels before this one are done;
@@ -542,8 +543,8 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
 }
 
 template <int kMode>
-static cudaError_t launch_q8(const CUtensorMap& tq, const DecodeParams& dp, int64_t items,
-                             cudaStream_t st) {
+static cudaError_t launch_q8(const CUtensorMap& tq, const DecodeParams& dp, const uint8_t* pool_q8,
+                             int64_t items, cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -555,14 +556,14 @@ static cudaError_t launch_q8(const CUtensorMap& tq, const DecodeParams& dp, int6
     attr_set[dev] = true;
   }
   return launch_pdl(mla_decode_q8_kernel<kMode>, dim3((unsigned)items), dim3(kQ8Threads),
-                    Q8Layout::kSmem, st, tq, dp);
+                    Q8Layout::kSmem, st, tq, dp, pool_q8);
 }
 
-cudaError_t launch_split_kv_q8(const CUtensorMap& q_map, const DecodeParams& dp, int64_t items,
-                               cudaStream_t st) {
-  if (dp.pool_q8 == nullptr) return cudaErrorInvalidValue;
-  return dp.work_tab != nullptr ? launch_q8<1>(q_map, dp, items, st)
-                                : launch_q8<0>(q_map, dp, items, st);
+cudaError_t launch_split_kv_q8(const CUtensorMap& q_map, const DecodeParams& dp,
+                               const uint8_t* pool_q8, int64_t items, cudaStream_t st) {
+  if (pool_q8 == nullptr) return cudaErrorInvalidValue;
+  return dp.work_tab != nullptr ? launch_q8<1>(q_map, dp, pool_q8, items, st)
+                                : launch_q8<0>(q_map, dp, pool_q8, items, st);
 }
 
 }  // namespace xmla

@@ -46,8 +46,6 @@ struct DecodeParams {
   // instead of part_o / part_ml
   __nv_bfloat16* o_hi;
   __nv_bfloat16* o_lo;
-  // the 8-bit pool [num_blocks, 64, 608] bytes (launch_split_kv_q8 only)
-  const uint8_t* pool_q8;
 };
 
 // Split-K attention over `items` work items; nr = rows per CTA (32 or 64);

@@ -319,9 +319,8 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   const bool direct = P.gemm && P.split && P.nsplit == 1 && !P.table && shard_partial == nullptr;
   dp.o_hi = direct ? o_hi : nullptr;
   dp.o_lo = direct ? o_lo : nullptr;
-  dp.pool_q8 = q8 ? (const uint8_t*)pool : nullptr;
   if (record_event(attn_start, st) != cudaSuccess) return XMLA_ERR_CUDA;
-  const cudaError_t ea = q8 ? launch_split_kv_q8(tmap_q, dp, P.items, st)
+  const cudaError_t ea = q8 ? launch_split_kv_q8(tmap_q, dp, (const uint8_t*)pool, P.items, st)
                             : launch_split_kv(P.nr, P.split, tmap_pool, tmap_q, dp, P.items, st);
   if (ea != cudaSuccess) return XMLA_ERR_CUDA;
   if (record_event(attn_stop, st) != cudaSuccess) return XMLA_ERR_CUDA;
