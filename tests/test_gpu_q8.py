@@ -179,3 +179,29 @@ def test_q8_workload_step_40l_b32_layer0_sampled():
     seqs = [int(np.argmax(wl.seqlens)), int(np.argmin(wl.seqlens)), 5]
     gc.assert_close(out, _oracle_q8(wl, inp, ocfg, seqs), "q8 step_40l_b32 layer 0",
                     plain_max_abs=True)
+
+
+def test_q8_bad_block_id_is_reported_not_faulted():
+    wl = workloads.custom(1, 1, [200], seed=824)
+    cfg, _ = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    _, dec, st = gc.gpu_step(wl, inp, cfg, cache="q8")
+    st.block_table[0, 1] = st.num_blocks + 7          # points outside the pool
+    dec.status.zero_()
+    out = dec.decode(cfg, st, inp.q.cuda().clone(), 0.1)
+    torch.cuda.synchronize()
+    assert dec.check_status() == 5
+    assert torch.isfinite(out.float()).all()
+
+
+def test_q8_sequence_longer_than_max_seqlen_is_reported():
+    wl = workloads.custom(1, 1, [200], seed=825)
+    cfg, _ = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    _, dec, st = gc.gpu_step(wl, inp, cfg, cache="q8")
+    st.seqlens[0] = 10_000                            # > max_seqlen given to the plan (200)
+    dec.status.zero_()
+    out = dec.decode(cfg, st, inp.q.cuda().clone(), 0.1)
+    torch.cuda.synchronize()
+    assert dec.check_status() == 5
+    assert torch.isfinite(out.float()).all()
