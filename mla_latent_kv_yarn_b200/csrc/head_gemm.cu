@@ -173,49 +173,71 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Each thread converts its row's 32 columns of a column block; the warp
+    // passes them through a private staging tile in the (now idle) operand
+    // stages, so that every global store writes 64 contiguous bytes of a row
+    // (8 rows x 4 lanes per instruction) instead of 16 bytes in 32 rows.
     const int quarter = warp & 3;
-    const int row = r0 + 32 * quarter + lane;
     const bool ok = mbar_wait(bar(2 * L::kStages), 0, abort_flag, p.status, p.wait_limit_ns);
     tc_fence_after();
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quarter) << 16);
+    constexpr uint32_t kStgRow = 80;                   // 64 B of a row + 16 B of padding
+    constexpr uint32_t kStgPart = 32 * kStgRow;
+    uint8_t* stg = smem + quarter * 2 * kStgPart;      // [part][32 rows][80 B]
+    const int srow = lane >> 2, piece = lane & 3;  // staging row (+ 8 j) and 16-byte piece
 #pragma unroll 1
     for (int cc = 0; cc < L::kN / 32; ++cc) {
       float v[32];
       tmem_ld32(t_lane + 32 * cc, v);
       tc_wait_ld();
-      if (!ok || *abort_flag || row >= p.rows) continue;
-      if constexpr (kAbsorb) {
-        uint32_t hi[16], lo[16];
+      if (!__all_sync(0xffffffffu, ok && *abort_flag == 0)) continue;
+      uint32_t w0[16], w1[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
+      for (int k = 0; k < 16; ++k) {
+        if constexpr (kAbsorb) {
           const float a = v[2 * k] * p.scale, b = v[2 * k + 1] * p.scale;
           const __nv_bfloat162 hv = __floats2bfloat162_rn(a, b);
           const __nv_bfloat162 lv =
               __floats2bfloat162_rn(a - __low2float(hv), b - __high2float(hv));
-          hi[k] = *reinterpret_cast<const uint32_t*>(&hv);
-          lo[k] = *reinterpret_cast<const uint32_t*>(&lv);
-        }
-        // q_ext rows: the 32 heads' hi parts of query row r, then their lo parts
-        uint4* dh = reinterpret_cast<uint4*>(
-            p.q_ext + ((int64_t)(2 * row) * kHeads + h) * kDRow + n0 + 32 * cc);
-        uint4* dl = reinterpret_cast<uint4*>(
-            p.q_ext + ((int64_t)(2 * row + 1) * kHeads + h) * kDRow + n0 + 32 * cc);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          dh[u] = make_uint4(hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3]);
-          dl[u] = make_uint4(lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3]);
-        }
-      } else {
-        uint32_t o[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
+          w0[k] = *reinterpret_cast<const uint32_t*>(&hv);
+          w1[k] = *reinterpret_cast<const uint32_t*>(&lv);
+        } else {
           const __nv_bfloat162 ov = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-          o[k] = *reinterpret_cast<const uint32_t*>(&ov);
+          w0[k] = *reinterpret_cast<const uint32_t*>(&ov);
+          w1[k] = 0u;
         }
-        uint4* d = reinterpret_cast<uint4*>(p.out + ((int64_t)row * kHeads + h) * kDV + 32 * cc);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) d[u] = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
       }
+      constexpr int kParts = kAbsorb ? 2 : 1;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        *reinterpret_cast<uint4*>(stg + lane * kStgRow + 16 * u) =
+            make_uint4(w0[4 * u], w0[4 * u + 1], w0[4 * u + 2], w0[4 * u + 3]);
+        if constexpr (kParts == 2)
+          *reinterpret_cast<uint4*>(stg + kStgPart + lane * kStgRow + 16 * u) =
+              make_uint4(w1[4 * u], w1[4 * u + 1], w1[4 * u + 2], w1[4 * u + 3]);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int part = 0; part < kParts; ++part) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int rr = srow + 8 * j;
+          const int grow = r0 + 32 * quarter + rr;
+          if (grow < p.rows) {
+            const uint4 val =
+                *reinterpret_cast<const uint4*>(stg + part * kStgPart + rr * kStgRow + 16 * piece);
+            if constexpr (kAbsorb) {
+              // q_ext rows: the 32 heads' hi parts of query row r, then their lo parts
+              *reinterpret_cast<uint4*>(p.q_ext + ((int64_t)(2 * grow + part) * kHeads + h) * kDRow +
+                                        n0 + 32 * cc + 8 * piece) = val;
+            } else {
+              *reinterpret_cast<uint4*>(p.out + ((int64_t)grow * kHeads + h) * kDV + 32 * cc +
+                                        8 * piece) = val;
+            }
+          }
+        }
+      }
+      __syncwarp();
     }
   }
 
