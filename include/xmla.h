@@ -179,7 +179,10 @@ int32_t xmla_decode_num_splits(int32_t batch, int32_t q_len, int64_t max_seqlen,
  * is row t % 64 of block block_table[b*max_blocks + t/64]).
  *   cfg: YaRN parameters used to rotate q_pe (host pointer);
  *   q: device bf16 [batch, q_len, 32, 192] = [q_nope 128 | q_pe 64], q_pe NOT
- *      rotated (the call rotates it);
+ *      rotated (the call rotates it).  q and out may also be pinned host memory
+ *      mapped into the device (unified addressing) when q_len <= 8: they are
+ *      read and written with ordinary loads and stores; a prompt chunk
+ *      (q_len > 8) reads q by TMA and needs it in device memory;
  *   W_UK: device bf16 [32, 128, 512]; W_UV: device bf16 [32, 512, 128];
  *   pool: device bf16 [num_blocks, 64, 576], 16-byte aligned;
  *   block_table: device int32 [batch, max_blocks];
