@@ -174,7 +174,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- work item
-  const int item = blockIdx.x;
+  // with the split query (prompt chunks, short contexts) later queries see more
+  // pages: the grid runs them first, so the short work items fill the tail
+  const int item = kSplitQ ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
   int b = 0, g = 0;
   int64_t seqlen = 0, npages = 0, p_begin = 0, p_end = 0;
   if constexpr (kMode != kWorkTable) {
