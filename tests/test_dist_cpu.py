@@ -79,3 +79,24 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["steps"] == 2 and d["higher_is_better"] is True
+
+
+def test_zero_copy_needs_a_mapped_buffer():
+    # without a device (or for memory that is not pinned and mapped) the end-to-end
+    # loop keeps the explicit copies
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.host_mapped(torch.zeros(16, dtype=torch.uint8)) is False
+
+
+def test_stage_tensors_packs_views_at_256_byte_boundaries():
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+    ts = [torch.arange(5, dtype=torch.int64), torch.ones((3, 7), dtype=torch.bfloat16),
+          torch.arange(3, dtype=torch.int32)]
+    buf, views = bench.stage_tensors(ts, "cpu")
+    assert [v.data_ptr() - buf.data_ptr() for v in views] == [0, 256, 512]
+    for t, v in zip(ts, views):
+        assert torch.equal(t, v)
