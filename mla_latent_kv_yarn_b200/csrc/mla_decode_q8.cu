@@ -299,12 +299,31 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         const uint32_t ew = c < 2 ? ex0.x : c < 4 ? ex0.y : c < 6 ? ex0.z : c < 8 ? ex0.w : ex1.x;
         int e = (int)(int8_t)((ew >> (16 * (c & 1) + ex_shift)) & 0xffu);
         e = min(max(e, kQ8EMin), kQ8EMax);
-        const __half2 scale = __half2half2(__ushort_as_half((unsigned short)((e + 15) << 10)));
         uint32_t o[8];
-        q8_to_f16x4(v[c].x, scale, o[0], o[1]);
-        q8_to_f16x4(v[c].y, scale, o[2], o[3]);
-        q8_to_f16x4(v[c].z, scale, o[4], o[5]);
-        q8_to_f16x4(v[c].w, scale, o[6], o[7]);
+        if (e <= 5) {
+          // (code + 128) under the f16 exponent 25 + e reads 2^(e+10) + (code+128) 2^e;
+          // subtracting 1152 * 2^e (exact: both lie in [2^(e+10), 2^(e+11))) leaves
+          // code * 2^e, one operation fewer per pair than the general path
+          const uint32_t magic = (uint32_t)((25 + e) << 2) * 0x01010101u;
+          const __half2 sub =
+              __half2half2(__ushort_as_half((unsigned short)(((25 + e) << 10) | 0x80)));
+          const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t x = wv[q] ^ 0x80808080u;
+            const uint32_t a = __byte_perm(x, magic, 0x4140), bb = __byte_perm(x, magic, 0x4342);
+            const __half2 ra = __hsub2(*reinterpret_cast<const __half2*>(&a), sub);
+            const __half2 rb = __hsub2(*reinterpret_cast<const __half2*>(&bb), sub);
+            o[2 * q] = *reinterpret_cast<const uint32_t*>(&ra);
+            o[2 * q + 1] = *reinterpret_cast<const uint32_t*>(&rb);
+          }
+        } else {
+          const __half2 scale = __half2half2(__ushort_as_half((unsigned short)((e + 15) << 10)));
+          q8_to_f16x4(v[c].x, scale, o[0], o[1]);
+          q8_to_f16x4(v[c].y, scale, o[2], o[3]);
+          q8_to_f16x4(v[c].z, scale, o[4], o[5]);
+          q8_to_f16x4(v[c].w, scale, o[6], o[7]);
+        }
         uint8_t* dst = buf + c * L::kChunk;
         *reinterpret_cast<uint4*>(dst + (((2 * jq) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         *reinterpret_cast<uint4*>(dst + (((2 * jq + 1) ^ sw) << 4)) =

@@ -124,6 +124,20 @@ def test_q8_decode_matches_the_oracle(batch, q_len, seqlens):
     gc.assert_close(out, _oracle_q8(wl, inp, ocfg), f"q8 {batch} {q_len} {seqlens}")
 
 
+@pytest.mark.parametrize("magnitude", [2.0 ** -12, 4096.0])
+def test_q8_decode_with_small_and_large_cache_values(magnitude):
+    # block exponents at the bottom of the range and above 5 (the converters'
+    # general path): the latent and rope values scaled by a power of two
+    wl = workloads.custom(2, 2, [700, 130], seed=826)
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    inp.c_kv.mul_(magnitude)
+    inp.k_pe.mul_(magnitude)
+    out, dec, _ = gc.gpu_step(wl, inp, cfg, cache="q8")
+    assert dec.check_status() == 0
+    gc.assert_close(out, _oracle_q8(wl, inp, ocfg), f"q8 values x {magnitude}")
+
+
 def test_q8_split_count_only_changes_rounding():
     wl = workloads.custom(1, 1, [9000], seed=823)
     cfg, ocfg = gc.cfgs()
