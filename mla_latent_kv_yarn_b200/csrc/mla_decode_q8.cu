@@ -81,7 +81,9 @@ struct Q8Layout {
 };
 
 // Over the 16 threads of one row parity (lane bits 0, 2, 3, 4): on return v[0]
-// holds the reduction of value j = b0 + 2 b2 + 4 b3 + 8 b4.
+// holds the reduction of value j = b0 + 2 b2 + 4 b3 + 8 b4.  (The bf16 kernel's
+// copy stays in its own translation unit: that kernel's code generation has
+// proven sensitive to changes around it.)
 template <bool kMax>
 __device__ __forceinline__ void q8_xpose_reduce16(float (&v)[16], int lane) {
   constexpr int kMask[4] = {16, 8, 4, 1};
@@ -336,6 +338,8 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
   } else if (warp == 1 || warp == 2) {
     // ================================================================ tensor-core issuers
     if (lane == 0 && n_pages > 0) {
+      // tc_mma_bf16 issues tcgen05.mma kind::f16; the operand type (f16 here) is
+      // the instruction descriptor's
       constexpr uint32_t idesc_qk = idesc_f16_f32(64, NR, false, false);
       constexpr uint32_t idesc_pv = idesc_f16_f32(128, NR, true, true);
       const uint64_t d_page_k = smem_desc_sw128(base + L::kOffPage, 16, 1024);     // K-major
