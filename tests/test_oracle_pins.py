@@ -552,3 +552,45 @@ def test_q8_row_halves_the_cache_as_the_page_says():
     # [P1] section 三, 方案 A: the q8_0 cache halves the bf16 one (12.5 GB -> ~6.3 GB).
     # 576 one-byte codes + 18 exponent bytes against 576 bf16 values:
     assert (576 + om.Q8_BLOCKS) / (576 * 2) == pytest.approx(6.3 / 12.5, rel=0.05)
+
+
+def test_chunk_of_queries_equals_one_query_at_a_time():
+    # a prompt chunk: query j at position N - q_len + j sees tokens 0..that position,
+    # which is the one-query call over the first position + 1 tokens (both forms)
+    rng = np.random.default_rng(21)
+    cfg = om.YarnConfig()
+    N, q_len, H = 40, 24, 2
+    q = rng.standard_normal((q_len, H, om.D_NOPE + om.D_ROPE))
+    c = rng.standard_normal((N, om.D_LATENT))
+    kp = rng.standard_normal((N, om.D_ROPE))
+    wk = rng.standard_normal((H, om.D_NOPE, om.D_LATENT)) / 512 ** 0.5
+    wv = rng.standard_normal((H, om.D_LATENT, om.D_V)) / 512 ** 0.5
+    kr = om.rope(kp, np.arange(N), cfg)
+    full = om.mla_attention_absorbed(q, c, kr, wk, wv, cfg)
+    full_x = om.mla_attention_expanded(q, c, kp, wk, wv, cfg)
+    for j in range(q_len):
+        t = N - q_len + j + 1
+        one = om.mla_attention_absorbed(q[j:j + 1], c[:t], kr[:t], wk, wv, cfg)[0]
+        np.testing.assert_allclose(full[j], one, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(full_x[j], one, rtol=1e-9, atol=1e-11)
+
+
+def test_attention_over_dequantised_rows_is_the_attention_of_those_values():
+    # the 8-bit path's reference is the plain attention over code * 2^e; rows that
+    # are exactly representable quantise to themselves, so both give the same output
+    rng = np.random.default_rng(22)
+    cfg = om.YarnConfig()
+    N, H = 70, 2
+    codes = rng.integers(-127, 128, (N, 576))
+    codes[:, ::32] = 127
+    e = rng.integers(-8, -4, (N, 18))
+    rows = (codes.reshape(N, 18, 32) * np.exp2(e)[..., None]).reshape(N, 576)
+    c8, e8 = om.q8_quantize(rows)
+    deq = om.q8_dequantize(c8, e8)
+    assert np.array_equal(deq, rows)
+    q = rng.standard_normal((1, H, 192))
+    wk = rng.standard_normal((H, 128, 512)) / 512 ** 0.5
+    wv = rng.standard_normal((H, 512, 128)) / 512 ** 0.5
+    a = om.mla_attention_absorbed(q, deq[:, :512], deq[:, 512:], wk, wv, cfg)
+    b = om.mla_attention_absorbed(q, rows[:, :512], rows[:, 512:], wk, wv, cfg)
+    assert np.array_equal(a, b)
