@@ -501,10 +501,12 @@ def run_xmla(args, wl):
     # address space): the bytes still cross the bus every step, without the two
     # copy operations and their fixed latency.  Only for small steps (at most 64 KiB
     # of inputs: a decode step of a few sequences; larger inputs move faster as
-    # one copy) and decode steps (a prompt chunk's tensor-core absorb reads the
-    # query by TMA, which stays on device memory).
-    zero_copy = (wl.q_len <= 8 and h2d <= 64 * 1024 and host_mapped(h_in) and
-                 host_mapped(h_out))
+    # one copy), decode steps (a prompt chunk's tensor-core absorb reads the
+    # query by TMA, which stays on device memory), and inputs read once: the
+    # producer's 144 blocks each read every hidden state, which over the bus cost
+    # more than one copy (2.73 vs 3.47 TB/s measured).
+    zero_copy = (wl.q_len <= 8 and h2d <= 64 * 1024 and not args.with_producer and
+                 host_mapped(h_in) and host_mapped(h_out))
     if world > 1:
         f = torch.tensor([1 if zero_copy else 0], dtype=torch.int32, device=dev)
         dist.all_reduce(f, op=dist.ReduceOp.MIN)
