@@ -344,6 +344,34 @@ def test_length_aware_plan_is_deterministic():
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+def _host_mapped(t: torch.Tensor) -> bool:
+    try:
+        from cuda.bindings import runtime as rt
+        err, dptr = rt.cudaHostGetDevicePointer(t.data_ptr(), 0)
+        return int(err) == 0 and int(dptr) == t.data_ptr()
+    except Exception:
+        return False
+
+
+def test_decode_step_buffers_in_mapped_host_memory():
+    # a decode call (q_len <= 8) may take q and out in pinned host memory mapped into
+    # the device: the same output as with device buffers
+    wl = workloads.custom(2, 2, [300, 129], seed=27)
+    cfg, _ = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    _, dec, st = gc.gpu_step(wl, inp, cfg)
+    q_h = inp.q.clone().pin_memory()
+    out_h = torch.zeros((wl.batch, wl.q_len, 32, 128), dtype=torch.bfloat16).pin_memory()
+    if not (_host_mapped(q_h) and _host_mapped(out_h)):
+        pytest.skip("pinned host memory is not mapped into the device")
+    scale = xmla.xmla_softmax_scale(cfg)
+    want = dec.decode(cfg, st, inp.q.cuda(), scale).clone()
+    dec.decode(cfg, st, q_h, scale, out=out_h)
+    torch.cuda.synchronize()
+    assert dec.check_status() == 0
+    assert torch.equal(out_h.view(torch.int16), want.cpu().view(torch.int16))
+
+
 def test_decode_is_deterministic_and_split_count_only_changes_rounding():
     wl = workloads.custom(1, 1, [9000], seed=23)
     cfg, ocfg = gc.cfgs()
