@@ -186,9 +186,10 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle sample
 
-def oracle_sample(wl, seconds: float):
-    """Time the fp64 expanded oracle on the first S tokens of sequence 0 (one
-    query at position S-1, 32 heads), S chosen for about `seconds` of work."""
+def oracle_sample(wl, seconds: float, form: str = "expanded"):
+    """Time the fp64 oracle (expanded, or absorbed over pre-rotated rope keys) on
+    the first S tokens of sequence 0 (one query at position S-1, 32 heads), S
+    chosen for about `seconds` of work."""
     import numpy as np
     import torch
 
@@ -210,9 +211,14 @@ def oracle_sample(wl, seconds: float):
     q = inp.q[0].double().numpy()
     cfg = om.YarnConfig()
 
+    kr = om.rope(kp, np.arange(n_max), cfg) if form == "absorbed" else None
+
     def run(n):
         t0 = time.perf_counter()
-        om.mla_attention_expanded(q, c[:n], kp[:n], wk, wv, cfg)
+        if form == "absorbed":
+            om.mla_attention_absorbed(q, c[:n], kr[:n], wk, wv, cfg)
+        else:
+            om.mla_attention_expanded(q, c[:n], kp[:n], wk, wv, cfg)
         return time.perf_counter() - t0
 
     probe_n = min(n_max, 4096)
@@ -614,6 +620,14 @@ def run_xmla(args, wl):
                 "kind": "oracle",
                 "sample": f"fp64 expanded oracle (numpy), sequence 0 of {wl.name}, first {n} "
                           f"tokens, 32 heads, q_len 1, one layer ({t:.1f} s)"}
+            n2, run2, cores2 = oracle_sample(wl, args.cpu_seconds / 2, form="absorbed")
+            t2 = run2(n2)
+            line["cpu_baseline_absorbed"] = {
+                "value": round(n2 * ROW_BYTES / t2 / 1e9, 6), "unit": "GB/s", "cores": cores2,
+                "kind": "oracle",
+                "sample": f"fp64 absorbed oracle (numpy, rope keys rotated beforehand), sequence 0 "
+                          f"of {wl.name}, first {n2} tokens, 32 heads, q_len 1, one layer "
+                          f"({t2:.1f} s)"}
         print(json.dumps(line), flush=True)
     del graph, graph_k
     if world > 1:
