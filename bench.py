@@ -58,6 +58,11 @@ def parse_args():
                          "(torchrun) each rank holds one shard and the partials are all-gathered "
                          "over NCCL; on one GPU, rank 0's share is timed (its shard, the gathered "
                          "partials' combine; the all-gather becomes a local copy)")
+    ap.add_argument("--workloads", default="decode_4k,step_40l_b32,verify_q4_b8,decode_512k_b4",
+                    help="other workloads measured in the same run (one GPU; step and split-K "
+                         "kernel times and roofline fractions under the line's 'workloads' key); "
+                         "empty to skip")
+    ap.add_argument("--extra-steps", type=int, default=20)
     ap.add_argument("--with-producer", action="store_true",
                     help="the step starts from the new tokens' hidden states: "
                          "kv_a_proj_with_mqa + RoPE + append (xmla_kv_produce), then decode")
@@ -455,10 +460,11 @@ def run_xmla(args, wl):
             dist.barrier()
         return ms, attn
 
+    # the clock sampler runs over every timed phase of this workload (the steps,
+    # the kernel-timed steps and the end-to-end steps), so it takes many samples
     clocks = ClockSampler(local)
     clocks.start()
     step_ms, _ = timed(graph, False)
-    clk = clocks.stop()
     _, attn_ms = timed(graph_k, True)
     total_ms = max_over_ranks(sum(step_ms), dev)
     status = dec.check_status()
@@ -555,6 +561,7 @@ def run_xmla(args, wl):
             zc_ms.append(ee0[i].elapsed_time(ee1[i]))
         e2e_total = max_over_ranks(sum(zc_ms), dev)
         del graph_zc
+    clk = clocks.stop()
 
     q8 = args.cache == "q8"
     cache_bytes_layer = sum(wl.seqlens) * (Q8_ROW_BYTES if q8 else ROW_BYTES)
@@ -611,6 +618,10 @@ def run_xmla(args, wl):
             "device_status": status,
         }
         if clk is not None:
+            # the step time scaled to the maximum SM clock, for runs whose clocks differ
+            clk["ms_per_step_x_mhz_over_max"] = round(
+                total_ms / args.steps * clk["sm_mhz"] / clk["sm_max_mhz"], 5) \
+                if clk.get("sm_max_mhz") else None
             line["clocks"] = clk
         if world == 1 and not args.no_cpu_baseline and not q8:
             n, run, cores = oracle_sample(wl, args.cpu_seconds)
@@ -628,12 +639,131 @@ def run_xmla(args, wl):
                 "sample": f"fp64 absorbed oracle (numpy, rope keys rotated beforehand), sequence 0 "
                           f"of {wl.name}, first {n2} tokens, 32 heads, q_len 1, one layer "
                           f"({t2:.1f} s)"}
-        print(json.dumps(line), flush=True)
     del graph, graph_k
+    if rank == 0:
+        extra = [w for w in args.workloads.split(",") if w and w != wl.name]
+        if extra and world == 1 and not q8 and not args.with_producer:
+            layers.clear()
+            del d_in, d_out, dec, flush_w, flush_r
+            torch.cuda.empty_cache()
+            line["workloads"] = {w: measure_other(workloads.workload(w), args, dev, cfg, scale)
+                                 for w in extra}
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def measure_other(wl, args, dev, cfg, scale):
+    """Another workload in the same run, timed like the headline one (the step
+    captured in a CUDA graph, L2 flushed before every step, CUDA events on the
+    stream; the split-K kernel timed in a second graph with events around it),
+    without the end-to-end and CPU legs.  Returns step and kernel times and the
+    kernel's fractions of the HBM and tensor rooflines."""
+    import torch
+
+    from mla_latent_kv_yarn_b200 import session, workloads
+
+    steps = max(3, args.extra_steps)
+    layers = []
+    for layer in range(wl.layers):
+        inp = workloads.layer_inputs(wl, layer, dev)
+        prefix, new = session.split_prefix(wl, inp)
+        st = session.build_layer(cfg, wl, prefix, dev)
+        layers.append({"st": st, "q": inp.q.clone(), "c": new.c_kv.clone(), "k": new.k_pe.clone(),
+                       "pos": new.positions.clone(), "sid": new.seq_ids.clone(),
+                       "out": torch.empty((wl.batch, wl.q_len, 32, 128), dtype=torch.bfloat16,
+                                          device=dev)})
+        del inp, prefix, new
+    torch.cuda.synchronize()
+    dec = session.Decoder(wl.batch, wl.q_len, wl.max_seqlen, dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in layers]
+    for a, b in ev:
+        a.record()
+        b.record()
+
+    def step(events):
+        for L, e in zip(layers, ev):
+            dec.step(cfg, L["st"], L["q"], L["c"], L["k"], L["pos"], L["sid"], scale,
+                     out=L["out"], events=e if events else None)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(False)
+        step(False)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph, graph_k = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(False)
+    with torch.cuda.graph(graph_k):
+        step(True)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def flush(i):
+        flush_w.fill_(i & 0xFF)
+        flush_r.sum()
+
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        flush(i)
+        graph.replay()
+        flush(i)
+        graph_k.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ms, attn_ms = [], []
+    for i in range(steps):
+        flush(i + 1)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        e1.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+    for i in range(steps):
+        flush(i + 1)
+        graph_k.replay()
+        torch.cuda.synchronize()
+        attn_ms.extend(a.elapsed_time(b) for a, b in ev)
+    clk = clocks.stop()
+    status = dec.check_status()
+    del graph, graph_k
+    cache_bytes_layer = sum(wl.seqlens) * ROW_BYTES
+    pairs = sum(wl.q_len * (n - wl.q_len) + wl.q_len * (wl.q_len + 1) // 2 for n in wl.seqlens)
+    flops_layer = 2176 * 32 * pairs
+    peak, peak_kind = measured_peaks()
+    tpeak, tpeak_kind = measured_tensor_peak()
+    step_mean = statistics.mean(step_ms)
+    kern = statistics.mean(attn_ms)
+    res = {
+        "config": {k: v for k, v in workload_config(wl, 1).items() if k not in ("l2", "parallelism")},
+        "steps": steps,
+        "ms_per_step": round(step_mean, 5),
+        "value": round(cache_bytes_layer * wl.layers / (step_mean * 1e-3) / 1e9, 3), "unit": "GB/s",
+        "pct_of_hbm_peak": round(100.0 * cache_bytes_layer * wl.layers / (step_mean * 1e-3) / 1e9
+                                 / peak, 2),
+        "attended_tokens_per_s": round(sum(wl.seqlens) * wl.layers / (step_mean * 1e-3), 1),
+        "kernel_ms": round(kern, 5),
+        "kernel_hbm_frac": round(cache_bytes_layer / (kern * 1e-3) / 1e9 / peak, 4),
+        "kernel_tensor_frac": round(flops_layer / (kern * 1e-3) / 1e12 / tpeak, 4),
+        "peak_source": {"hbm": peak_kind, "tensor": tpeak_kind},
+        "gpu_launches": 3 * wl.layers * steps,
+        "device_status": status,
+    }
+    if wl.q_len > 1:
+        res["attended_pairs_per_s"] = round(pairs * wl.layers / (step_mean * 1e-3), 1)
+    if clk is not None:
+        res["clocks"] = clk
+    layers.clear()
+    del dec, flush_w, flush_r
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_shards(args, wl):

@@ -179,10 +179,13 @@ int32_t xmla_decode_num_splits(int32_t batch, int32_t q_len, int64_t max_seqlen,
  * is row t % 64 of block block_table[b*max_blocks + t/64]).
  *   cfg: YaRN parameters used to rotate q_pe (host pointer);
  *   q: device bf16 [batch, q_len, 32, 192] = [q_nope 128 | q_pe 64], q_pe NOT
- *      rotated (the call rotates it).  q and out may also be pinned host memory
- *      mapped into the device (unified addressing) when q_len <= 8: they are
- *      read and written with ordinary loads and stores; a prompt chunk
- *      (q_len > 8) reads q by TMA and needs it in device memory;
+ *      rotated (the call rotates it).  This deliberately differs from
+ *      rotating q_pe with xmla_rope_yarn before the call: a q_pe already
+ *      rotated would be rotated a second time, so pass the raw query.  q and
+ *      out may also be pinned host memory mapped into the device (unified
+ *      addressing) when q_len <= 8: they are read and written with ordinary
+ *      loads and stores; a prompt chunk (q_len > 8) reads q by TMA and needs
+ *      it in device memory;
  *   W_UK: device bf16 [32, 128, 512]; W_UV: device bf16 [32, 512, 128];
  *   pool: device bf16 [num_blocks, 64, 576], 16-byte aligned;
  *   block_table: device int32 [batch, max_blocks];
@@ -398,9 +401,11 @@ xmla_status xmla_combine_shards(const float* partials, int32_t num_shards, const
  *   - Sizes whose workspace (xmla_decode_workspace_size) exceeds
  *     XMLA_NOALLOC_SCRATCH_BYTES are rejected with XMLA_ERR_WORKSPACE before
  *     anything is launched.
- *   - The first call on a device looks up the scratch array's device address
- *     (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture on that device.
+ *   - The first call in a CUDA context looks up the scratch array's device
+ *     address in that context (cudaGetSymbolAddress) and caches it for that
+ *     context only (a context created anew, e.g. after cudaDeviceReset, gets
+ *     a fresh lookup); make that first call before any stream capture on
+ *     the device.
  *   - All calls share the one array and it keeps the previous call's
  *     contents.  Nothing in it has to start at zero: every value a call reads
  *     was written earlier by the same call.  Calls whose work may overlap on

@@ -238,10 +238,13 @@ __device__ __forceinline__ void work_plan_block(const WorkPlanArgs& a, PlanSmem&
   const int units = a.batch * a.groups;  // < a.ctas <= kMaxPlanCtas = 2 * kAbsorbThreads
   pdl_wait();                            // the lengths may come from the kernel launched before
   long long tot = 0, wmax = 0;
+  // w_s[u]: the unit's cost in pages (short units of the mixed kernel take one
+  // pass per query of the row group)
   for (int u = t; u < units; u += kAbsorbThreads) {
     int64_t n = a.seqlens[u / a.groups];
     if (n < 0 || n > a.max_seqlen) n = 0;  // the split-K kernel reports the bad length
-    const int w = (int)((n + kPage - 1) / kPage);
+    int w = (int)((n + kPage - 1) / kPage);
+    if (w <= a.short_pages) w *= a.short_weight;
     w_s[u] = w;
     tot += w;
     wmax = max(wmax, (long long)w);
@@ -281,7 +284,9 @@ __device__ __forceinline__ void work_plan_block(const WorkPlanArgs& a, PlanSmem&
   }
   const int first0 = before + incl - v;
   auto emit = [&](int u, int first, int ns) {
-    const int w = w_s[u];
+    int64_t n = a.seqlens[u / a.groups];  // the unit's pages, unweighted
+    if (n < 0 || n > a.max_seqlen) n = 0;
+    const int w = (int)((n + kPage - 1) / kPage);
     const int pps = (w + ns - 1) / ns;
     a.unit_tab[u] = make_int2(first, ns);
     for (int s = 0; s < ns; ++s)

@@ -39,6 +39,10 @@ struct WorkPlanArgs {
   int32_t ctas;  // split-K grid size, units < ctas <= kMaxPlanCtas
   int4* work_tab;
   int2* unit_tab;
+  // a unit of at most short_pages pages costs short_weight times its pages
+  // (the mixed kernel runs one pass per query over a short sequence)
+  int32_t short_pages;
+  int32_t short_weight;
 };
 
 // q_ext[r, h] for rows r = b*q_len + j; qscale = softmax scale * log2 e.

@@ -152,109 +152,74 @@ enum WorkMode : int {
   kWorkTable = 2,   // entry blockIdx of p.work_tab (written by the preceding kernel)
 };
 
-template <int NR, int kMode, bool kSplitQ>
-__global__ void __launch_bounds__(kDecodeThreads, 1)
-    mla_decode_kernel(const __grid_constant__ CUtensorMap tmap_pool,
-                      const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p) {
-  using L = DecodeLayout<NR, kSplitQ>;
-  extern __shared__ uint8_t smem_raw[];
-  uint32_t base = smem_u32(smem_raw);
-  const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
-  uint8_t* smem = smem_raw + pad;
-  base += pad;
+// What one pass of the split-K attention covers: queries [j0, j0 + jn) of
+// sequence b (32 rows each) over its logical pages [p_begin, p_begin +
+// n_pages); the split's partials go to rows [row0, row0 + 32 jn).
+struct DecodePass {
+  int b;
+  int j0;
+  int jn;
+  int n_pages;
+  int64_t seqlen;
+  int64_t npages;   // pages of the whole sequence
+  int64_t p_begin;
+  int64_t row0;     // first partial row
+  int32_t qrow0;    // first q_ext row loaded for the QK product
+};
 
-  auto bar = [&](int i) -> uint32_t { return base + L::kOffBars + 8u * (uint32_t)i; };
+// Barrier initialisation of one pass (one thread); clears the abort flag.
+// `bars`: shared address of the pass's barrier set (L::kNumBars words).
+template <int NR, bool kSplitQ>
+__device__ __forceinline__ void decode_init_barriers(uint32_t bars, volatile int* abort_flag) {
+  using L = DecodeLayout<NR, kSplitQ>;
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
+  mbar_init(bar(L::kBarQ), 1);
+  for (int i = 0; i < L::kLatSlots; ++i) {
+    mbar_init(bar(L::kBarLatFull + i), 1);
+    mbar_init(bar(L::kBarLatEmpty + i), 1);
+  }
+  for (int i = 0; i < L::kRopeSlots; ++i) {
+    mbar_init(bar(L::kBarRopeFull + i), 1);
+    mbar_init(bar(L::kBarRopeEmpty + i), 1);
+  }
+  for (int i = 0; i < 2; ++i) {
+    mbar_init(bar(L::kBarSFull + i), 1);
+    mbar_init(bar(L::kBarSFree + i), kSoftmaxThreads);
+    mbar_init(bar(L::kBarPFull + i), kSoftmaxThreads);
+    mbar_init(bar(L::kBarPvDone + i), 1);
+  }
+  mbar_init(bar(L::kBarDrain + 0), 1);
+  mbar_init(bar(L::kBarDrain + 1), 1);
+  *abort_flag = 0;
+  fence_barrier_init();
+}
+
+// The roles of a CTA over one pass (DecodePass): warp 0 streams the pages by
+// TMA, warp 1 issues QK, warp 2 issues PV, warps 3-6 run the softmax and write
+// the split's (m, l, O).  The caller initialises the barrier set at `bars`
+// (decode_init_barriers) and allocates tensor memory.
+// kQHiRows (single query only): q_ext is in the split layout and the pass
+// uses the hi rows alone, query k of the pass at row qrow0 + 64 k (32-row
+// boxes; a 32-row box lands with the same 128-byte swizzle phase as the
+// corresponding half of a 64-row one, the halves being 4 KB apart).
+template <int NR, bool kSplitQ, bool kQHiRows = false>
+__device__ __forceinline__ void decode_pass(uint8_t* smem, uint32_t base, uint32_t bars,
+                                            uint32_t tmem_base, const CUtensorMap& tmap_pool,
+                                            const CUtensorMap& tmap_q, const DecodeParams& p,
+                                            const DecodePass& w) {
+  using L = DecodeLayout<NR, kSplitQ>;
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
   float* m_used = reinterpret_cast<float*>(smem + L::kOffMUsed);
   float* m_next = reinterpret_cast<float*>(smem + L::kOffMNext);
   float* alpha_s = reinterpret_cast<float*>(smem + L::kOffAlpha);
   float* red = reinterpret_cast<float*>(smem + L::kOffRed);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
-
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- work item
-  // with the split query (prompt chunks, short contexts) later queries see more
-  // pages: the grid runs them first, so the short work items fill the tail
-  const int item = kSplitQ ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
-  int b = 0, g = 0;
-  int64_t seqlen = 0, npages = 0, p_begin = 0, p_end = 0;
-  if constexpr (kMode != kWorkTable) {
-    const int split = item % p.nsplit;
-    const int bg = item / p.nsplit;
-    g = bg % p.groups;
-    b = bg / p.groups;
-    seqlen = p.seqlens[b];
-    if (seqlen < p.q_len || seqlen > p.max_seqlen) {
-      if (threadIdx.x == 0) record_status(p.status, XMLA_ERR_DEVICE_OOB);
-      seqlen = 0;
-    }
-    npages = (seqlen + kPage - 1) / kPage;
-    const int64_t p_lo = kMode == kWorkRanged ? min(p.page_lo, npages) : 0;
-    const int64_t p_hi = kMode == kWorkRanged ? min(p.page_hi, npages) : npages;
-    const int64_t pps = (p_hi - p_lo + p.nsplit - 1) / p.nsplit;
-    p_begin = p_lo + (int64_t)split * pps;
-    p_end = min(p_hi, p_begin + pps);
-  }
-
-  // ---- setup (independent of the previous kernel's results)
-  if (threadIdx.x == 0) {
-    mbar_init(bar(L::kBarQ), 1);
-    for (int i = 0; i < L::kLatSlots; ++i) {
-      mbar_init(bar(L::kBarLatFull + i), 1);
-      mbar_init(bar(L::kBarLatEmpty + i), 1);
-    }
-    for (int i = 0; i < L::kRopeSlots; ++i) {
-      mbar_init(bar(L::kBarRopeFull + i), 1);
-      mbar_init(bar(L::kBarRopeEmpty + i), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(L::kBarSFull + i), 1);
-      mbar_init(bar(L::kBarSFree + i), kSoftmaxThreads);
-      mbar_init(bar(L::kBarPFull + i), kSoftmaxThreads);
-      mbar_init(bar(L::kBarPvDone + i), 1);
-    }
-    mbar_init(bar(L::kBarDrain + 0), 1);
-    mbar_init(bar(L::kBarDrain + 1), 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(base + L::kOffTmem, L::kTmemCols);
-    tmem_relinquish();
-  }
-  if (threadIdx.x >= 32 * kSoftmaxWarp0 && threadIdx.x < 32 * kSoftmaxWarp0 + NR)
-    m_used[threadIdx.x - 32 * kSoftmaxWarp0] = -INFINITY;
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + L::kOffTmem);
-  if constexpr (kMode == kWorkTable) {
-    // the table comes from the kernel launched before this one
-    pdl_wait();
-    const int4 e = p.work_tab[item];
-    if (e.x >= 0 && e.x < p.batch * p.groups) {
-      g = e.x % p.groups;
-      b = e.x / p.groups;
-      seqlen = p.seqlens[b];
-      if (seqlen < p.q_len || seqlen > p.max_seqlen) {
-        if (threadIdx.x == 0) record_status(p.status, XMLA_ERR_DEVICE_OOB);
-        seqlen = 0;
-      }
-      npages = (seqlen + kPage - 1) / kPage;
-      p_begin = min((int64_t)e.y, npages);
-      p_end = min((int64_t)e.z, npages);
-    }
-  }
-  const int j0 = g * (NR / 32);
-  const int jn = min(p.q_len - j0, NR / 32);
-  const int nrows = jn * 32;
-  // causal: pages past this CTA's last query position hold nothing it may see
-  // (a prefill chunk's early queries; at decode sizes this is the last page)
-  p_end = min(p_end, (seqlen - p.q_len + j0 + jn - 1) / kPage + 1);
-  const int n_pages = (int)max((int64_t)0, p_end - p_begin);
-  const int32_t qrow0 = (int32_t)(((int64_t)b * p.q_len + j0) * (L::kSplitQ ? 64 : 32));
-  pdl_launch_dependents();
+  const int b = w.b;
+  const int64_t seqlen = w.seqlen, npages = w.npages, p_begin = w.p_begin;
+  const int j0 = w.j0, jn = w.jn, nrows = jn * 32, n_pages = w.n_pages;
+  const int32_t qrow0 = w.qrow0;
 
   if (warp == 0) {
     // ================================================================ TMA producer
@@ -283,7 +248,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       pdl_wait();
       mbar_arrive_expect_tx(bar(L::kBarQ), 9u * L::kQChunk);
       for (int c = 0; c < 9; ++c)
-        tma_load_2d(base + L::kOffQ + c * L::kQChunk, &tmap_q, c * 64, qrow0, bar(L::kBarQ));
+        if constexpr (kQHiRows) {
+#pragma unroll
+          for (int k = 0; k < NR / 32; ++k)
+            tma_load_2d(base + L::kOffQ + c * L::kQChunk + k * 4096u, &tmap_q, c * 64,
+                        qrow0 + 64 * k, bar(L::kBarQ));
+        } else {
+          tma_load_2d(base + L::kOffQ + c * L::kQChunk, &tmap_q, c * 64, qrow0, bar(L::kBarQ));
+        }
       for (int i = 0; i < n_pages && ok; ++i) {
         int32_t blk = nb0;
         nb0 = nb1;
@@ -620,7 +592,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
 
     // ---- epilogue: unnormalised O, running max m and sum l of this split
-    const int64_t row0 = (int64_t)item * NR;
+    const int64_t row0 = w.row0;
     bool have = ok && n_pages > 0;
     if (have) {
       const int pi = n_pages - 1;
@@ -714,12 +686,243 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
   }
 
+}
+
+// The sequence, row group and page range of work item `item` (modes
+// kWorkSplit and kWorkRanged: split item % nsplit of unit item / nsplit).
+template <int kMode>
+__device__ __forceinline__ void split_work_item(const DecodeParams& p, int item, int& b, int& g,
+                                                int64_t& seqlen, int64_t& npages,
+                                                int64_t& p_begin, int64_t& p_end) {
+  const int split = item % p.nsplit;
+  const int bg = item / p.nsplit;
+  g = bg % p.groups;
+  b = bg / p.groups;
+  seqlen = p.seqlens[b];
+  if (seqlen < p.q_len || seqlen > p.max_seqlen) {
+    if (threadIdx.x == 0) record_status(p.status, XMLA_ERR_DEVICE_OOB);
+    seqlen = 0;
+  }
+  npages = (seqlen + kPage - 1) / kPage;
+  const int64_t p_lo = kMode == kWorkRanged ? min(p.page_lo, npages) : 0;
+  const int64_t p_hi = kMode == kWorkRanged ? min(p.page_hi, npages) : npages;
+  const int64_t pps = (p_hi - p_lo + p.nsplit - 1) / p.nsplit;
+  p_begin = p_lo + (int64_t)split * pps;
+  p_end = min(p_hi, p_begin + pps);
+}
+
+// The same from entry `item` of the work table (mode kWorkTable); read after
+// the preceding kernel, which wrote the table, has completed.
+__device__ __forceinline__ void table_work_item(const DecodeParams& p, int item, int& b, int& g,
+                                                int64_t& seqlen, int64_t& npages,
+                                                int64_t& p_begin, int64_t& p_end) {
+  const int4 e = p.work_tab[item];
+  if (e.x >= 0 && e.x < p.batch * p.groups) {
+    g = e.x % p.groups;
+    b = e.x / p.groups;
+    seqlen = p.seqlens[b];
+    if (seqlen < p.q_len || seqlen > p.max_seqlen) {
+      if (threadIdx.x == 0) record_status(p.status, XMLA_ERR_DEVICE_OOB);
+      seqlen = 0;
+    }
+    npages = (seqlen + kPage - 1) / kPage;
+    p_begin = min((int64_t)e.y, npages);
+    p_end = min((int64_t)e.z, npages);
+  }
+}
+
+template <int NR, int kMode, bool kSplitQ>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    mla_decode_kernel(const __grid_constant__ CUtensorMap tmap_pool,
+                      const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p) {
+  using L = DecodeLayout<NR, kSplitQ>;
+  extern __shared__ uint8_t smem_raw[];
+  uint32_t base = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  base += pad;
+  float* m_used = reinterpret_cast<float*>(smem + L::kOffMUsed);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
+  const int warp = threadIdx.x >> 5;
+
+  // ---- work item
+  // with the split query (prompt chunks, short contexts) later queries see more
+  // pages: the grid runs them first, so the short work items fill the tail
+  const int item = kSplitQ ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  int b = 0, g = 0;
+  int64_t seqlen = 0, npages = 0, p_begin = 0, p_end = 0;
+  if constexpr (kMode != kWorkTable)
+    split_work_item<kMode>(p, item, b, g, seqlen, npages, p_begin, p_end);
+
+  // ---- setup (independent of the previous kernel's results)
+  if (threadIdx.x == 0) decode_init_barriers<NR, kSplitQ>(base + L::kOffBars, abort_flag);
+  if (warp == 1) {
+    tmem_alloc(base + L::kOffTmem, L::kTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x >= 32 * kSoftmaxWarp0 && threadIdx.x < 32 * kSoftmaxWarp0 + NR)
+    m_used[threadIdx.x - 32 * kSoftmaxWarp0] = -INFINITY;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + L::kOffTmem);
+  if constexpr (kMode == kWorkTable) {
+    // the table comes from the kernel launched before this one
+    pdl_wait();
+    table_work_item(p, item, b, g, seqlen, npages, p_begin, p_end);
+  }
+  const int j0 = g * (NR / 32);
+  const int jn = min(p.q_len - j0, NR / 32);
+  // causal: pages past this CTA's last query position hold nothing it may see
+  // (a prefill chunk's early queries; at decode sizes this is the last page)
+  p_end = min(p_end, (seqlen - p.q_len + j0 + jn - 1) / kPage + 1);
+  const int n_pages = (int)max((int64_t)0, p_end - p_begin);
+  const int32_t qrow0 = (int32_t)(((int64_t)b * p.q_len + j0) * (L::kSplitQ ? 64 : 32));
+  pdl_launch_dependents();
+
+  const DecodePass w{b, j0, jn, n_pages, seqlen, npages, p_begin, (int64_t)item * NR, qrow0};
+  decode_pass<NR, kSplitQ>(smem, base, base + L::kOffBars, tmem_base, tmap_pool, tmap_q, p, w);
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+
+// Split-K attention that chooses the query's precision per sequence, for a
+// batch holding short and long sequences at once.  q_ext is in the split
+// layout (hi and lo rows).  A sequence of at most kSplitQMaxSeqlen tokens is
+// dominated by a few tokens and its output is large, so the ~2^-9 relative
+// error of a single bf16 query reaches the output bound there: it is attended
+// with the query as hi + lo parts (tmap_q2, 64-row boxes), one pass of 32 rows
+// per query of the CTA's row group.  A longer sequence is attended with the hi
+// rows alone (tmap_q, 32-row boxes), NR rows in one pass, with the deeper page
+// ring.  The partials are laid out as
+// mla_decode_kernel<NR, kMode, false> writes them, so the combine is the same.
+// Each pass has a barrier set of its own (a finished pass may still have
+// tensor-core arrivals in flight on its barriers).
+template <int NR>
+struct MixedLayout {
+  using LL = DecodeLayout<NR, false>;
+  using LS = DecodeLayout<32, true>;
+  static constexpr int kShortPasses = NR / 32;
+  // the short passes' barrier sets: LS's own, then one more per extra pass
+  static constexpr uint32_t kOffBars2 = (LS::kBytes + 7u) & ~7u;
+  static constexpr uint32_t kShortBytes = kOffBars2 + (kShortPasses - 1) * LS::kNumBars * 8;
+  static constexpr uint32_t kTmemCols = LL::kTmemCols > LS::kTmemCols ? LL::kTmemCols
+                                                                       : LS::kTmemCols;
+  static constexpr uint32_t kBytes = LL::kBytes > kShortBytes ? LL::kBytes : kShortBytes;
+  static constexpr uint32_t kSmem = kBytes + 1024;
+  static_assert(kSmem <= 232448, "shared memory per CTA");
+};
+
+// The passes of a short sequence in the mixed kernel: one per query of the
+// CTA's row group, 32 rows each, with the hi/lo query and a barrier set of its
+// own.  (Kept inline: compiled out of line, as a call, it put the kernel's long
+// pass into a markedly slower code generation -- verify_q4_b8 430 -> 547 us.)
+template <int NR>
+__device__ __forceinline__ void mixed_short_passes(uint8_t* smem, uint32_t base, uint32_t tmem_base,
+                                                const CUtensorMap* tmap_pool,
+                                                const CUtensorMap* tmap_q2,
+                                                const DecodeParams* pp, int item, int b, int jg,
+                                                int64_t seqlen, int64_t npages, int64_t p_begin,
+                                                int64_t p_end) {
+  using M = MixedLayout<NR>;
+  using LS = typename M::LS;
+  const DecodeParams& p = *pp;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LS::kOffAbort);
+  float* m_used = reinterpret_cast<float*>(smem + LS::kOffMUsed);
+#pragma unroll 1
+  for (int jj = 0; jj < M::kShortPasses; ++jj) {
+    const int j0 = jg + jj;
+    if (j0 >= p.q_len) break;
+    const uint32_t bars =
+        base + (jj == 0 ? LS::kOffBars : M::kOffBars2 + (uint32_t)(jj - 1) * LS::kNumBars * 8u);
+    if (threadIdx.x == 0) decode_init_barriers<32, true>(bars, abort_flag);
+    if (threadIdx.x >= 32 * kSoftmaxWarp0 && threadIdx.x < 32 * kSoftmaxWarp0 + 32)
+      m_used[threadIdx.x - 32 * kSoftmaxWarp0] = -INFINITY;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const int64_t pe = min(p_end, (seqlen - p.q_len + j0) / kPage + 1);
+    const int n_pages = (int)max((int64_t)0, pe - p_begin);
+    const DecodePass w{b, j0, 1, n_pages, seqlen, npages, p_begin, (int64_t)item * NR + 32 * jj,
+                       (int32_t)(((int64_t)b * p.q_len + j0) * 64)};
+    decode_pass<32, true>(smem, base, bars, tmem_base, *tmap_pool, *tmap_q2, p, w);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+}
+
+template <int NR, int kMode>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    mla_decode_mixed_kernel(const __grid_constant__ CUtensorMap tmap_pool,
+                            const __grid_constant__ CUtensorMap tmap_q,
+                            const __grid_constant__ CUtensorMap tmap_q2, const DecodeParams p) {
+  using M = MixedLayout<NR>;
+  using LL = typename M::LL;
+  extern __shared__ uint8_t smem_raw[];
+  uint32_t base = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  base += pad;
+  float* m_used = reinterpret_cast<float*>(smem + LL::kOffMUsed);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + LL::kOffAbort);
+  const int warp = threadIdx.x >> 5;
+  const int item = (int)blockIdx.x;
+  int b = 0, g = 0;
+  int64_t seqlen = 0, npages = 0, p_begin = 0, p_end = 0;
+  if constexpr (kMode != kWorkTable)
+    split_work_item<kMode>(p, item, b, g, seqlen, npages, p_begin, p_end);
+
+  // ---- setup for a long sequence, as in mla_decode_kernel (a short one
+  // discards the barriers and sets up its passes in their own layout)
+  if (threadIdx.x == 0) decode_init_barriers<NR, false>(base + LL::kOffBars, abort_flag);
+  if (warp == 1) {
+    tmem_alloc(base + LL::kOffTmem, M::kTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x >= 32 * kSoftmaxWarp0 && threadIdx.x < 32 * kSoftmaxWarp0 + NR)
+    m_used[threadIdx.x - 32 * kSoftmaxWarp0] = -INFINITY;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + LL::kOffTmem);
+  if constexpr (kMode == kWorkTable) {
+    pdl_wait();  // the table comes from the kernel launched before this one
+    table_work_item(p, item, b, g, seqlen, npages, p_begin, p_end);
+  }
+  const int jg = g * (NR / 32);
+  pdl_launch_dependents();
+  if (seqlen > kSplitQMaxSeqlen) {
+    const int jn = min(p.q_len - jg, NR / 32);
+    p_end = min(p_end, (seqlen - p.q_len + jg + jn - 1) / kPage + 1);
+    const int n_pages = (int)max((int64_t)0, p_end - p_begin);
+    const DecodePass w{b, jg, jn, n_pages, seqlen, npages, p_begin, (int64_t)item * NR,
+                       (int32_t)(((int64_t)b * p.q_len + jg) * 64)};
+    decode_pass<NR, false, true>(smem, base, base + LL::kOffBars, tmem_base, tmap_pool, tmap_q, p,
+                                 w);
+  } else {
+    __syncthreads();  // every thread holds the tensor-memory base: its slot lies in the short ring
+    if (threadIdx.x == 0) {
+      for (int i = 0; i < LL::kNumBars; ++i)
+        asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(base + LL::kOffBars + 8u * i)
+                     : "memory");
+    }
+    mixed_short_passes<NR>(smem, base, tmem_base, &tmap_pool, &tmap_q2, &p, item, b, jg, seqlen,
+                           npages, p_begin, p_end);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, M::kTmemCols);
   }
 }
 
@@ -763,6 +966,43 @@ cudaError_t launch_split_kv(int nr, bool split_q, const CUtensorMap& pool_map,
                    : launch_mode<32, false>(mode, pool_map, q_map, dp, items, st);
   if (nr == 64 && !split_q) return launch_mode<64, false>(mode, pool_map, q_map, dp, items, st);
   return cudaErrorInvalidValue;
+}
+
+
+template <int NR, int kMode>
+static cudaError_t launch_mixed(const CUtensorMap& tp, const CUtensorMap& tq,
+                                const CUtensorMap& tq2, const DecodeParams& dp, int64_t items,
+                                cudaStream_t st) {
+  using M = MixedLayout<NR>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(mla_decode_mixed_kernel<NR, kMode>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, M::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  return launch_pdl(mla_decode_mixed_kernel<NR, kMode>, dim3((unsigned)items),
+                    dim3(kDecodeThreads), M::kSmem, st, tp, tq, tq2, dp);
+}
+
+cudaError_t launch_split_kv_mixed(int nr, const CUtensorMap& pool_map, const CUtensorMap& q_map,
+                                  const CUtensorMap& q2_map, const DecodeParams& dp,
+                                  int64_t items, cudaStream_t st) {
+  const int mode = dp.work_tab != nullptr                          ? kWorkTable
+                   : (dp.page_lo != 0 || dp.page_hi != INT64_MAX) ? kWorkRanged
+                                                                  : kWorkSplit;
+  if (nr != 32 && nr != 64) return cudaErrorInvalidValue;
+  if (mode == kWorkTable)
+    return nr == 32 ? launch_mixed<32, kWorkTable>(pool_map, q_map, q2_map, dp, items, st)
+                    : launch_mixed<64, kWorkTable>(pool_map, q_map, q2_map, dp, items, st);
+  if (mode == kWorkRanged)
+    return nr == 32 ? launch_mixed<32, kWorkRanged>(pool_map, q_map, q2_map, dp, items, st)
+                    : launch_mixed<64, kWorkRanged>(pool_map, q_map, q2_map, dp, items, st);
+  return nr == 32 ? launch_mixed<32, kWorkSplit>(pool_map, q_map, q2_map, dp, items, st)
+                  : launch_mixed<64, kWorkSplit>(pool_map, q_map, q2_map, dp, items, st);
 }
 
 }  // namespace xmla

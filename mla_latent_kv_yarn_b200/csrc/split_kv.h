@@ -13,6 +13,10 @@ namespace xmla {
 
 constexpr int kMaxSplits = 1024;
 
+// Sequences of at most this many tokens are attended with the query as a hi
+// and a lo bf16 part (see launch_split_kv and launch_split_kv_mixed).
+constexpr int64_t kSplitQMaxSeqlen = 4096;
+
 // Arguments of the split-K attention kernel.  Partial results are laid out
 // per work item: (sequence b, row group g, split s) in that order, or, with a
 // work table, in the order of the table's entries.
@@ -55,5 +59,15 @@ struct DecodeParams {
 cudaError_t launch_split_kv(int nr, bool split_q, const CUtensorMap& pool_map,
                             const CUtensorMap& q_map, const DecodeParams& dp, int64_t items,
                             cudaStream_t st);
+
+// Split-K attention of a batch that may hold short and long sequences, q_ext
+// in the split layout (as for split_q): each CTA attends its sequence with the
+// hi/lo query (q2_map: box 64 x 64) when it has at most kSplitQMaxSeqlen
+// tokens, one pass per query of its nr-row group, else with the hi rows alone
+// (q_map: the same rows, box 64 x 32).  Writes the partials
+// launch_split_kv(nr, false, ...) writes.
+cudaError_t launch_split_kv_mixed(int nr, const CUtensorMap& pool_map, const CUtensorMap& q_map,
+                                  const CUtensorMap& q2_map, const DecodeParams& dp,
+                                  int64_t items, cudaStream_t st);
 
 }  // namespace xmla

@@ -30,19 +30,23 @@ __global__ void wait_timeout_selftest_kernel(int32_t* status, uint64_t limit_ns)
 
 // ---------------------------------------------------------------- host plan
 
-// Up to this many tokens per sequence, and for every call with more than
-// kSplitQMinChunk new tokens (a prefill chunk, whose first queries see only a
-// few tokens), the query goes to the QK product as a hi and a lo bf16 part
-// (the split-K kernel's split_q layout, one query of 32 heads per CTA).  A
-// short context is dominated by a few tokens and its output is large (|out|
+// Up to kSplitQMaxSeqlen tokens per sequence, and for every call with more
+// than kSplitQMinChunk new tokens (a prefill chunk, whose first queries see
+// only a few tokens), the query goes to the QK product as a hi and a lo bf16
+// part (the split-K kernel's split_q layout, one query of 32 heads per CTA).
+// A short context is dominated by a few tokens and its output is large (|out|
 // up to ~4), so the ~2^-9 relative score error of a single bf16 query reaches
 // the 1e-2 output bound there; the split costs a shallower page ring, which
-// only long decode contexts, dominated by streaming, would notice.
-constexpr int64_t kSplitQMaxSeqlen = 4096;
+// only long decode contexts, dominated by streaming, would notice.  A decode
+// call of several sequences whose longest exceeds kSplitQMaxSeqlen may also
+// hold short ones: it runs the mixed kernel, which makes that choice per
+// sequence on the device (q_ext in the split layout; long sequences use the hi
+// rows alone).
 constexpr int32_t kSplitQMinChunk = 8;
 
 struct Plan {
-  bool split;   // hi/lo query (split_q)
+  bool split;   // hi/lo query (split_q) for every sequence
+  bool mixed;   // hi/lo query for the sequences of <= kSplitQMaxSeqlen tokens only
   bool gemm;    // a prompt chunk: absorb and W_UV on the tensor cores (head_gemm.cu)
   int nr;       // rows per CTA (32 or 64)
   int groups;   // row groups per sequence
@@ -66,8 +70,11 @@ static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_
   if (B < 1 || q_len < 1 || q_len > (q8 ? kQ8MaxQLen : kMaxQLen) || max_seqlen < q_len ||
       max_seqlen > (int64_t)0x7fffffff - kPage || num_sms < 1 || num_splits < 0 || span_pages < 0)
     return false;
+  // query rows, and (row, head) pairs, are counted in 32-bit integers by the kernels
+  if ((int64_t)B * q_len * kHeads > (int64_t)0x7fffffff) return false;
   Plan P;
   P.split = !q8 && (max_seqlen <= kSplitQMaxSeqlen || q_len > kSplitQMinChunk);
+  P.mixed = !q8 && !P.split && B > 1;
   P.nr = q8 || P.split || q_len == 1 ? 32 : 64;
   P.groups = (q_len * 32 + P.nr - 1) / P.nr;
   int64_t max_pages = (max_seqlen + kPage - 1) / kPage;
@@ -89,8 +96,8 @@ static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_
             num_sms <= kMaxPlanCtas;
   P.items = P.table ? num_sms : units * P.nsplit;
   if (P.items > 0x7fffffff) return false;
-  // q_ext: bf16 rows of 576; split, each row also has its low half
-  const size_t qext = (size_t)B * q_len * kHeads * kDRow * 2 * (P.split ? 2 : 1);
+  // q_ext: bf16 rows of 576; split or mixed, each row also has its low half
+  const size_t qext = (size_t)B * q_len * kHeads * kDRow * 2 * (P.split || P.mixed ? 2 : 1);
   P.off_qext = 0;
   P.off_o = align_up(qext, 1024);
   P.off_ml = align_up(P.off_o + (size_t)P.items * P.nr * kDLatent * 4, 1024);
@@ -244,9 +251,15 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
     return XMLA_ERR_CUDA;
   // the QK product's B tile: 64 rows (32 heads hi then lo when split, 32 heads of one query
   // at 32 rows per CTA, else 2 queries x 32 heads)
-  if (!encode_rows576(&tmap_q, q_ext, (uint64_t)rows * kHeads * (P.split ? 2 : 1),
-                      P.split || P.nr == 64 ? 64 : 32))
+  // mixed: q_ext in the split layout, read as 32-row boxes of hi rows (long
+  // sequences, tmap_q) and as 64-row boxes of hi and lo rows (short ones, tmap_q2)
+  if (!encode_rows576(&tmap_q, q_ext, (uint64_t)rows * kHeads * (P.split || P.mixed ? 2 : 1),
+                      P.mixed ? 32 : P.split || P.nr == 64 ? 64 : 32))
     return XMLA_ERR_CUDA;
+  CUtensorMap tmap_q2;
+  if (P.mixed && !encode_rows576(&tmap_q2, q_ext, (uint64_t)rows * kHeads * 2, 64))
+    return XMLA_ERR_CUDA;
+  const int split_arg = P.split || P.mixed ? 1 : 0;
 
   const float qscale = softmax_scale * kLog2e;
   const RopeTable tab = make_rope_table(cfg);
@@ -259,6 +272,9 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
     plan.ctas = (int32_t)P.items;
     plan.work_tab = (int4*)(ws + P.off_wtab);
     plan.unit_tab = (int2*)(ws + P.off_utab);
+    // a short sequence's CTA runs one pass per query of its row group
+    plan.short_pages = P.mixed ? (int32_t)(kSplitQMaxSeqlen / kPage) : 0;
+    plan.short_weight = P.nr / 32;
   }
   // Every kernel of the chain waits (griddepcontrol.wait) for its predecessor
   // before reading anything a kernel of this step may have written, so once
@@ -289,10 +305,10 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   const cudaError_t e0 =
       ap != nullptr
           ? launch_step_prologue((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
-                                 rows, q_len, P.split ? 1 : 0, qscale, tab, *ap, tab, pa,
+                                 rows, q_len, split_arg, qscale, tab, *ap, tab, pa,
                                  P.table ? &plan : nullptr, P.gemm, st)
           : launch_q_absorb((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
-                            rows, q_len, P.split ? 1 : 0, qscale, tab,
+                            rows, q_len, split_arg, qscale, tab,
                             P.table ? &plan : nullptr, P.gemm, st, q8);
   if (e0 != cudaSuccess) return XMLA_ERR_CUDA;
   if (P.gemm && launch_absorb_gemm(tmap_qin, tmap_wuk, gp, st) != cudaSuccess) return XMLA_ERR_CUDA;
@@ -320,8 +336,10 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   dp.o_hi = direct ? o_hi : nullptr;
   dp.o_lo = direct ? o_lo : nullptr;
   if (record_event(attn_start, st) != cudaSuccess) return XMLA_ERR_CUDA;
-  const cudaError_t ea = q8 ? launch_split_kv_q8(tmap_q, dp, (const uint8_t*)pool, P.items, st)
-                            : launch_split_kv(P.nr, P.split, tmap_pool, tmap_q, dp, P.items, st);
+  const cudaError_t ea =
+      q8      ? launch_split_kv_q8(tmap_q, dp, (const uint8_t*)pool, P.items, st)
+      : P.mixed ? launch_split_kv_mixed(P.nr, tmap_pool, tmap_q, tmap_q2, dp, P.items, st)
+                : launch_split_kv(P.nr, P.split, tmap_pool, tmap_q, dp, P.items, st);
   if (ea != cudaSuccess) return XMLA_ERR_CUDA;
   if (record_event(attn_stop, st) != cudaSuccess) return XMLA_ERR_CUDA;
   if (shard_partial != nullptr) {
@@ -534,7 +552,8 @@ extern "C" xmla_status xmla_combine_shards(const float* partials, int32_t num_sh
                                            const void* W_UV, int32_t batch, int32_t q_len,
                                            void* out, void* stream) {
   if (partials == nullptr || W_UV == nullptr || out == nullptr) return XMLA_ERR_INVALID_ARG;
-  if (batch < 1 || q_len < 1 || q_len > kMaxQLen || num_shards < 1 || num_shards > kMaxSplits)
+  if (batch < 1 || q_len < 1 || q_len > kMaxQLen || num_shards < 1 || num_shards > kMaxSplits ||
+      (int64_t)batch * q_len * kHeads > (int64_t)0x7fffffff)
     return XMLA_ERR_SHAPE;
   if ((((uintptr_t)partials) | ((uintptr_t)W_UV) | ((uintptr_t)out)) & 15u)
     return XMLA_ERR_INVALID_ARG;
@@ -562,23 +581,66 @@ constexpr size_t kNoAllocScratchBytes = (size_t)XMLA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 static std::mutex g_noalloc_mutex;
-static void* g_noalloc_addr[64] = {};
 
-// Device address of the scratch array on the current device.  In host code
-// the array's name is only a host-side stand-in, so the real address is asked
-// from the runtime once per device (with that device current) and cached.
-static xmla_status noalloc_scratch(void** addr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return XMLA_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return XMLA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return XMLA_ERR_CUDA;
-    g_noalloc_addr[dev] = p;
+// The array's device address belongs to the CUDA context that loaded the
+// library's module: a context destroyed and created again (cudaDeviceReset,
+// or the primary context released and retained anew) loads the module again,
+// possibly elsewhere.  Addresses are therefore cached per context, keyed on
+// the context's unique id (cuCtxGetId), never reused across contexts.
+struct NoAllocSlot {
+  unsigned long long ctx_id;
+  void* addr;
+};
+static NoAllocSlot g_noalloc_slots[64] = {};
+static int g_noalloc_next = 0;
+
+static bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  if (get_current == nullptr || get_id == nullptr) {
+    void* p1 = nullptr;
+    void* p2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &p2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess)
+      return false;
+    get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p1);
+    get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p2);
   }
-  *addr = g_noalloc_addr[dev];
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current context.  In host code
+// the array's name is only a host-side stand-in, so the real address is asked
+// from the runtime (with the context's device current) the first time a
+// context is seen, and cached for that context.
+static xmla_status noalloc_scratch(void** addr) {
+  unsigned long long id = 0;
+  if (!current_context_id(&id)) {
+    // no context current yet: let the runtime make the device's primary
+    // context current (and initialise it), then ask again
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess ||
+        !current_context_id(&id))
+      return XMLA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  for (const NoAllocSlot& s : g_noalloc_slots) {
+    if (s.addr != nullptr && s.ctx_id == id) {
+      *addr = s.addr;
+      return XMLA_OK;
+    }
+  }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return XMLA_ERR_CUDA;
+  g_noalloc_slots[g_noalloc_next] = NoAllocSlot{id, p};
+  g_noalloc_next = (g_noalloc_next + 1) % 64;
+  *addr = p;
   return XMLA_OK;
 }
 

@@ -91,9 +91,9 @@ def workload(index_or_name) -> Workload:
 
 
 def custom(batch: int, q_len: int, seqlens, *, contiguous: bool = False, seed: int = 7,
-           heads: int = N_HEADS, name: str = "custom") -> Workload:
-    return Workload(name, batch, q_len, list(int(n) for n in seqlens), contiguous=contiguous,
-                    seed=seed, heads=heads)
+           heads: int = N_HEADS, name: str = "custom", layers: int = 1) -> Workload:
+    return Workload(name, batch, q_len, list(int(n) for n in seqlens), layers=layers,
+                    contiguous=contiguous, seed=seed, heads=heads)
 
 
 _TENSOR_IDS = {"q": 1, "c_kv": 2, "k_pe": 3, "W_UK": 4, "W_UV": 5, "blocks": 6, "hidden": 7,

@@ -77,10 +77,35 @@ def compare(out: torch.Tensor, ref: dict[int, np.ndarray]):
     return (max(e[0] for e in errs), max(e[1] for e in errs), max(e[2] for e in errs))
 
 
-def assert_close(out, ref, what="", plain_max_abs: bool = False):
+# Below this |ref| the bf16 output's own rounding is at most 2^-8 (half an ulp
+# of a value under 2), so the plain max-abs bound is attainable there; above it
+# the rounding alone reaches 0.0078 (|ref| in [2, 4)) or 0.0156 ([4, 8)).
+PLAIN_BELOW = 2.0
+
+
+def plain_max_abs_below(out, ref: dict[int, np.ndarray], limit: float = PLAIN_BELOW) -> float:
+    """Max-abs error over the elements whose reference is below `limit` in magnitude."""
+    got = f64(out)
+    worst = 0.0
+    for b, r in ref.items():
+        d = np.abs(got[b] - r)[np.abs(r) < limit]
+        if d.size:
+            worst = max(worst, float(d.max()))
+    return worst
+
+
+def assert_close(out, ref, what="", plain_max_abs: bool = False, plain_below: bool = False):
+    """rel L2 <= 5e-3 and the widened bound on every element; plain_max_abs: also
+    |err| <= 1e-2 on every element; plain_below: also |err| <= 1e-2 on every
+    element with |ref| < PLAIN_BELOW.  The message reports the plain max-abs error,
+    the one below PLAIN_BELOW and the widened excess side by side."""
     max_abs, rel, widened = compare(out, ref)
+    below = plain_max_abs_below(out, ref)
     ok = np.isfinite(max_abs) and rel <= REL_L2 and widened <= MAX_ABS
     if plain_max_abs:
         ok = ok and max_abs <= MAX_ABS
-    assert ok, f"{what}: max_abs={max_abs:.3e} rel_l2={rel:.3e} widened={widened:.3e}"
+    if plain_below:
+        ok = ok and below <= MAX_ABS
+    assert ok, (f"{what}: max_abs={max_abs:.3e} max_abs(|ref|<{PLAIN_BELOW:g})={below:.3e} "
+                f"rel_l2={rel:.3e} widened={widened:.3e}")
     return max_abs, rel

@@ -104,3 +104,14 @@ def test_argument_validation_without_gpu(x):
     assert L.xmla_selftest_wait_timeout(None, 1000, None) == 1
     for code in range(8):
         assert x.xmla_status_string(code)
+
+
+def test_row_counts_beyond_int32_are_rejected(x):
+    L = x.lib()
+    # batch * q_len * 32 (query rows times heads) must stay below 2^31
+    assert x.xmla_decode_workspace_size(1 << 16, 1024, 65536, 148) == 0   # 2^31 exactly
+    assert x.xmla_decode_workspace_size((1 << 16) - 1, 1024, 65536, 148) > 0
+    assert x.xmla_decode_q8_workspace_size(1 << 28, 8, 4096, 148) == 0
+    # the shard combine checks the same bound before touching any pointer
+    fake = ctypes.c_void_p(256)
+    assert L.xmla_combine_shards(fake, 2, fake, 1 << 16, 1024, fake, None) == 2

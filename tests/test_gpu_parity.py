@@ -27,11 +27,17 @@ def _half_ulp_bf16(v: np.ndarray) -> np.ndarray:
     return np.exp2(np.floor(np.log2(a)) - 8.0)
 
 
-@pytest.mark.parametrize("theta,factor", [(1e4, 64.0), (1e7, 64.0), (1e4, 1.0)])
-def test_rope_within_half_ulp_of_oracle(theta, factor):
+@pytest.mark.parametrize("theta,factor,mscale,mscale_all", [
+    (1e4, 64.0, 1.0, 1.0), (1e7, 64.0, 1.0, 1.0), (1e4, 1.0, 1.0, 1.0),
+    (1e4, 64.0, 0.707, 1.0),   # cos/sin carry mscale(s, 0.707) / mscale(s, 1) = 0.9139...
+    (1e4, 64.0, 1.0, 0.5),     # ... and mscale(s, 1) / mscale(s, 0.5) = 1.0941...
+])
+def test_rope_within_half_ulp_of_oracle(theta, factor, mscale, mscale_all):
     cfg, ocfg = gc.cfgs(theta)
     cfg.factor = factor
-    ocfg = om.YarnConfig(rope_theta=theta, factor=factor)
+    cfg.mscale = mscale
+    cfg.mscale_all_dim = mscale_all
+    ocfg = om.YarnConfig(rope_theta=theta, factor=factor, mscale=mscale, mscale_all_dim=mscale_all)
     g = torch.Generator().manual_seed(5)
     R, H = 37, 32
     q = torch.randn((R, H, 192), generator=g).to(torch.bfloat16)
@@ -231,10 +237,11 @@ def _plan_tables(dec: session.Decoder):
     def up(x, a):
         return (x + a - 1) // a * a
     split = dec.max_seqlen <= 4096                  # hi/lo query up to 4096 tokens
+    hilo_rows = split or dec.batch > 1              # a batch past 4096 tokens keeps both parts too
     nr = 32 if dec.q_len == 1 or split else 64
     groups = (dec.q_len * 32 + nr - 1) // nr
     items = dec.sms
-    off_o = up(dec.batch * dec.q_len * 32 * 576 * 2 * (2 if split else 1), 1024)
+    off_o = up(dec.batch * dec.q_len * 32 * 576 * 2 * (2 if hilo_rows else 1), 1024)
     off_ml = up(off_o + items * nr * 512 * 4, 1024)
     off_w = up(off_ml + items * nr * 2 * 4, 1024)
     off_u = up(off_w + items * 16, 256)

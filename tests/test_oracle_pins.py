@@ -90,6 +90,54 @@ def test_yarn_band_edges_at_theta_1e4():
     assert base[22] / 64 < f[22] < base[22]
 
 
+def test_yarn_ramp_interior_values_by_hand():
+    """Inside the band the blend is linear in the pair index: at theta = 1e4 the
+    band edges are 10 and 23 (above), so pair i takes the fraction
+    r = (i - 10) / 13 of the divided frequency and 1 - r of the kept one:
+        f_i = base_i * (1 - r * (1 - 1/64)).
+    Worked out by hand as exact fractions (base_i = 10^(-i/8)):
+      pair 12: r = 2/13,  1 - (2/13)(63/64)  = 706/832 = 353/416
+      pair 16: r = 6/13,  1 - (6/13)(63/64)  = 454/832 = 227/416, base 1/100
+      pair 20: r = 10/13, 1 - (10/13)(63/64) = 202/832 = 101/416
+      pair 22: r = 12/13, 1 - (12/13)(63/64) = 76/832  = 19/208"""
+    f = om.yarn_inv_freq(om.YarnConfig())
+    assert f[16] == pytest.approx(227.0 / 41600.0, rel=1e-14)          # 0.00545673076923...
+    assert f[12] == pytest.approx(10.0 ** -1.5 * 353.0 / 416.0, rel=1e-14)
+    assert f[20] == pytest.approx(10.0 ** -2.5 * 101.0 / 416.0, rel=1e-14)
+    assert f[22] == pytest.approx(10.0 ** -2.75 * 19.0 / 208.0, rel=1e-14)
+    # an off-by-one band (edges 11 and 24) or a ramp that is not linear in i would
+    # move pair 16 away from 227/41600
+    assert abs(f[16] - 0.01 * (1 - 5 / 13 * 63 / 64)) > 1e-4
+
+
+def test_cos_sin_factor_with_unequal_mscales():
+    """cos/sin carry mscale(s, mscale) / mscale(s, mscale_all_dim); with
+    mscale = 0.707 and mscale_all_dim = 1 at s = 64 that is
+    (0.1 * 0.707 * ln 64 + 1) / (0.1 * ln 64 + 1) = 1.29403303399... / 1.41588830833...
+    = 0.91393723..., and the logit scale keeps mscale_all_dim only."""
+    ln64 = 6.0 * math.log(2.0)
+    cfg = om.YarnConfig(mscale=0.707, mscale_all_dim=1.0)
+    want = (0.1 * 0.707 * ln64 + 1.0) / (0.1 * ln64 + 1.0)
+    assert want == pytest.approx(0.9139372, abs=1e-7)
+    assert om.cos_sin_factor(cfg) == pytest.approx(want, rel=1e-15)
+    # swapped numerator and denominator would give 1/want = 1.0941...
+    assert abs(om.cos_sin_factor(cfg) - 1.0 / want) > 0.1
+    # the factor scales the rotated vector's length, at every position
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((4, 64))
+    y = om.rope(x, np.array([0, 7, 4096, 300000]), cfg)
+    assert np.allclose(np.linalg.norm(y, axis=1), want * np.linalg.norm(x, axis=1), rtol=1e-13)
+    # position 0: a pure scaling by the factor
+    assert np.allclose(y[0], want * x[0], rtol=1e-14, atol=0)
+    # the logit scale uses mscale_all_dim alone: unchanged from the default config
+    assert om.softmax_scale(cfg) == pytest.approx(0.14467962580268923172, rel=1e-14)
+    half = om.YarnConfig(mscale=1.0, mscale_all_dim=0.5)
+    assert om.softmax_scale(half) == pytest.approx((0.05 * ln64 + 1.0) ** 2 / math.sqrt(192.0),
+                                                   rel=1e-14)
+    assert om.cos_sin_factor(half) == pytest.approx((0.1 * ln64 + 1.0) / (0.05 * ln64 + 1.0),
+                                                    rel=1e-15)
+
+
 # ---------------------------------------------------------------- RoPE
 
 def test_rope_matches_complex_rotation():

@@ -25,13 +25,18 @@ def _built():
 
 def test_noalloc_decode_matches_workspace_decode_on_two_calls():
     wl = workloads.custom(2, 2, [3000, 700], seed=41)
-    cfg, _ = gc.cfgs()
+    cfg, ocfg = gc.cfgs()
     inp = workloads.layer_inputs(wl, 0, "cpu")
-    # reference: the existing entry point with a caller-allocated workspace
-    ref, dec, st = gc.gpu_step(wl, inp, cfg)
-    ref_np = {b: gc.f64(ref[b]) for b in range(wl.batch)}
+    # the cache with every token appended (one decode step through the workspace path)
+    _, dec, st = gc.gpu_step(wl, inp, cfg)
     q = inp.q.cuda()
     scale = xmla.xmla_softmax_scale(cfg, 192)
+    # reference: xmla_decode on the same cache with a caller-allocated workspace
+    ref = dec.decode(cfg, st, q, scale).clone()
+    torch.cuda.synchronize()
+    assert dec.check_status() == 0
+    gc.assert_close(ref, gc.oracle_out(wl, inp, ocfg), "workspace decode vs oracle",
+                    plain_max_abs=True)
     for _ in range(2):  # the scratch keeps the previous call's contents
         out = torch.full_like(ref, float("nan"))
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -40,7 +45,8 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls():
                                  scale, 0, status, out)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
-        gc.assert_close(out, ref_np, "noalloc vs workspace decode", plain_max_abs=True)
+        # the same plan and kernels as xmla_decode: bit for bit the same output
+        assert torch.equal(out, ref)
 
 
 def test_noalloc_decode_rejects_sizes_beyond_its_scratch():
