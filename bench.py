@@ -38,6 +38,9 @@ METRIC = "MLA decode: latent-KV HBM GB/s (% of B200 peak) and attended tokens/s"
 ROW_BYTES = 1152  # one cache row: [c_kv 512 | k_pe 64] bf16
 Q8_ROW_BYTES = 608  # one 8-bit cache row: 576 codes, 18 exponents, 14 pad bytes
 FALLBACK_HBM_GBS = 6650.0
+# a device-side wait queued before a directly launched step, long enough for the
+# host to queue the whole step behind it (~50 us at the B200's clock)
+HOST_AHEAD_CYCLES = 100_000
 FALLBACK_BF16_TFLOPS = 1590.0
 
 
@@ -401,9 +404,7 @@ def run_xmla(args, wl):
                 dec.step(cfg, L["st"], L["q"], L["c_new"], L["k_new"], L["pos"], L["sid"], scale,
                          out=L["out"], events=ev if events else None)
 
-    # eager warm-up (loads modules), then capture the step twice: `graph` is what
-    # is timed; `graph_k` also records CUDA events around the split-K kernel
-    # (event nodes split the programmatic launch chain, so it is timed apart)
+    # eager warm-up (loads modules), then capture the step: `graph` is what is timed
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
@@ -414,9 +415,6 @@ def run_xmla(args, wl):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         step(events=False)
-    graph_k = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_k):
-        step(events=True)
     torch.cuda.synchronize()
     if dec.check_status() != 0:
         raise RuntimeError(f"device status {dec.check_status()} after warm-up")
@@ -435,17 +433,18 @@ def run_xmla(args, wl):
         flush_l2(i)
         graph.replay()
         flush_l2(i)
-        graph_k.replay()
+        torch.cuda._sleep(HOST_AHEAD_CYCLES)
+        step(events=True)
     torch.cuda.synchronize()
 
-    def timed(g, collect_attn: bool):
+    def timed(g):
         """K steps, each bracketed by events on the stream; L2 flushed between."""
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        ms, attn = [], []
+        ms = []
         for i in range(args.steps):
             flush_l2(i + 1)
             e0[i].record(stream)
@@ -453,19 +452,39 @@ def run_xmla(args, wl):
             e1[i].record(stream)
             e1[i].synchronize()
             ms.append(e0[i].elapsed_time(e1[i]))
-            if collect_attn:
-                attn.extend(a.elapsed_time(b) for a, b in ev_attn)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        return ms, attn
+        return ms
+
+    def timed_kernel():
+        """Every layer's split-K kernel timed alone: CUDA events recorded on the
+        stream immediately before and after it (xmla_decode_step's profiling
+        events).  The step is launched directly for this, not replayed from the
+        graph (an event-record node inside a graph breaks the programmatic launch
+        chain and delays the next kernel by several microseconds), queued behind
+        the L2 flush and a short device-side wait, so the device never waits for
+        the host."""
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        attn = []
+        for i in range(args.steps):
+            flush_l2(i + 1)
+            torch.cuda._sleep(HOST_AHEAD_CYCLES)
+            step(events=True)
+            torch.cuda.synchronize()
+            attn.extend(a.elapsed_time(b) for a, b in ev_attn)
+        if world > 1:
+            dist.barrier()
+        return attn
 
     # the clock sampler runs over every timed phase of this workload (the steps,
     # the kernel-timed steps and the end-to-end steps), so it takes many samples
     clocks = ClockSampler(local)
     clocks.start()
-    step_ms, _ = timed(graph, False)
-    _, attn_ms = timed(graph_k, True)
+    step_ms = timed(graph)
+    attn_ms = timed_kernel()
     total_ms = max_over_ranks(sum(step_ms), dev)
     status = dec.check_status()
     # a cache that fits in L2 is also timed warm: the same steps back to back with
@@ -639,7 +658,7 @@ def run_xmla(args, wl):
                 "sample": f"fp64 absorbed oracle (numpy, rope keys rotated beforehand), sequence 0 "
                           f"of {wl.name}, first {n2} tokens, 32 heads, q_len 1, one layer "
                           f"({t2:.1f} s)"}
-    del graph, graph_k
+    del graph
     if rank == 0:
         extra = [w for w in args.workloads.split(",") if w and w != wl.name]
         if extra and world == 1 and not q8 and not args.with_producer:
@@ -696,11 +715,9 @@ def measure_other(wl, args, dev, cfg, scale):
         step(False)
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
-    graph, graph_k = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         step(False)
-    with torch.cuda.graph(graph_k):
-        step(True)
     flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
 
@@ -713,7 +730,8 @@ def measure_other(wl, args, dev, cfg, scale):
         flush(i)
         graph.replay()
         flush(i)
-        graph_k.replay()
+        torch.cuda._sleep(HOST_AHEAD_CYCLES)
+        step(True)
     torch.cuda.synchronize()
     clocks = ClockSampler(dev.index or 0)
     clocks.start()
@@ -726,14 +744,15 @@ def measure_other(wl, args, dev, cfg, scale):
         e1.record(stream)
         e1.synchronize()
         step_ms.append(e0.elapsed_time(e1))
-    for i in range(steps):
+    for i in range(steps):  # the split-K kernels alone, as in run_xmla's timed_kernel
         flush(i + 1)
-        graph_k.replay()
+        torch.cuda._sleep(HOST_AHEAD_CYCLES)
+        step(True)
         torch.cuda.synchronize()
         attn_ms.extend(a.elapsed_time(b) for a, b in ev)
     clk = clocks.stop()
     status = dec.check_status()
-    del graph, graph_k
+    del graph
     cache_bytes_layer = sum(wl.seqlens) * ROW_BYTES
     pairs = sum(wl.q_len * (n - wl.q_len) + wl.q_len * (wl.q_len + 1) // 2 for n in wl.seqlens)
     flops_layer = 2176 * 32 * pairs

@@ -68,6 +68,7 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
   const int t = threadIdx.x;
   if (cb == kDLatent / 64) {
     pdl_wait();
+    pdl_launch_dependents();
     constexpr int kPairs = kDRope / 2;
     for (int e = row_lo * kPairs + t; e < row_hi * kPairs; e += kAbsorbThreads) {
       const int r = e / kPairs, i = e % kPairs;
@@ -110,6 +111,7 @@ __device__ __forceinline__ void q_absorb_block(int h, int cb, const __nv_bfloat1
     }
   }
   pdl_wait();
+  pdl_launch_dependents();
   for (int r0 = row_lo; r0 < row_hi; r0 += kAbsorbRows) {
     const int nr = min(kAbsorbRows, row_hi - r0);
     __syncthreads();
@@ -166,6 +168,7 @@ __device__ __forceinline__ void q_rope_rows_block(int r_lo, int r_hi, const __nv
   const int t = threadIdx.x;
   const int nr = r_hi - r_lo;
   pdl_wait();
+  pdl_launch_dependents();
   if (t < nr * kPairs) {
     const int r = r_lo + t / kPairs, i = t % kPairs;
     const int64_t pos = (int64_t)seqlens[r / q_len] - q_len + (r % q_len);
@@ -237,6 +240,7 @@ __device__ __forceinline__ void work_plan_block(const WorkPlanArgs& a, PlanSmem&
   const int t = threadIdx.x;
   const int units = a.batch * a.groups;  // < a.ctas <= kMaxPlanCtas = 2 * kAbsorbThreads
   pdl_wait();                            // the lengths may come from the kernel launched before
+  pdl_launch_dependents();
   long long tot = 0, wmax = 0;
   // w_s[u]: the unit's cost in pages (short units of the mixed kernel take one
   // pass per query of the row group)
@@ -311,6 +315,16 @@ static bool plan_ok(const WorkPlanArgs& plan) {
 // Mode 2 blocks take kRopeRows rows of all 32 heads each (q_rope_rows_block).
 constexpr int kRopeRows = 4;
 
+// The block-table lines of WorkPlanArgs, shared out over every thread of the
+// grid.  The table is not written by this kernel or the preceding one in a
+// decode call, and a prefetch only moves a line into L2, so it is issued at
+// once, before any wait.
+__device__ __forceinline__ void prefetch_block_table(const WorkPlanArgs& a) {
+  const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t l = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; l < a.bt_lines; l += nthr)
+    prefetch_l2(a.bt_prefetch + l * 32);
+}
+
 template <int kRows>
 struct AbsorbGrid {
   static constexpr int kPerRows = kRows == 2 ? kHeads : kAbsorbBlocks;
@@ -338,7 +352,11 @@ __global__ void __launch_bounds__(kAbsorbThreads) q_absorb_kernel(
     AbsorbSmem absorb;
     PlanSmem plan;
   } sm;
-  pdl_launch_dependents();
+  // every role signals dependent launches right after its own wait for the
+  // preceding kernel: a dependent grid starts only once every kernel older than
+  // this one has completed (the split-K kernel reads sequence lengths and block
+  // ids before its own wait, relying on that)
+  prefetch_block_table(plan);
   using G = AbsorbGrid<kRows>;
   const int absorb_blocks = G::blocks(rows);
   if constexpr (kPlan) {
@@ -378,7 +396,9 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
     ProduceSmem<kAbsorbThreads / 32> produce;
     PlanSmem plan;
   } sm;
-  pdl_launch_dependents();
+  // every role signals dependent launches right after its own wait (as in
+  // q_absorb_kernel)
+  prefetch_block_table(plan);
   using G = AbsorbGrid<kRows>;
   const int absorb_blocks = G::blocks(rows);
   if (blockIdx.x < absorb_blocks) {
@@ -404,11 +424,14 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
   const int prod_blocks = pa.T > 0 ? kProdBlocks : 0;
   if (blockIdx.x < absorb_blocks + kPlanBlocks + prod_blocks) {
     produce_block<kAbsorbThreads / 32>(blockIdx.x - absorb_blocks - kPlanBlocks, threadIdx.x, pa,
-                                       k_tab, sm.produce, [] { __syncthreads(); },
-                                       [] { pdl_wait(); });
+                                       k_tab, sm.produce, [] { __syncthreads(); }, [] {
+                                         pdl_wait();
+                                         pdl_launch_dependents();
+                                       });
     return;
   }
   pdl_wait();
+  pdl_launch_dependents();
   const int64_t total = ap.T * kRowPieces;
   const int64_t idx =
       (int64_t)(blockIdx.x - absorb_blocks - kPlanBlocks - prod_blocks) * kAbsorbThreads +
@@ -421,46 +444,41 @@ __global__ void __launch_bounds__(kAbsorbThreads) step_prologue_kernel(
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
                             int split, float qscale, const RopeTable& tab,
-                            const WorkPlanArgs* plan, bool rope_only, cudaStream_t st,
-                            bool f16) {
+                            const WorkPlanArgs& plan, bool with_plan, bool rope_only,
+                            cudaStream_t st, bool f16) {
   const int mode = rope_only ? 2 : rows > kAbsorbRows ? 1 : 0;
   const int64_t nrb = (rows + kAbsorbRows - 1) / kAbsorbRows;
   const unsigned absorb_blocks =
       (unsigned)(mode == 2 ? AbsorbGrid<2>::blocks(rows)
                            : mode == 1 ? kAbsorbBlocks * nrb : kAbsorbBlocks);
+  if (with_plan && !plan_ok(plan)) return cudaErrorInvalidValue;
+  const unsigned blocks = absorb_blocks + (with_plan ? 1u : 0u);
   if (f16) {
     if (mode == 2) return cudaErrorInvalidValue;
-    if (plan != nullptr) {
-      if (!plan_ok(*plan)) return cudaErrorInvalidValue;
-      return launch_pdl(mode == 1 ? q_absorb_kernel<true, 1, true> : q_absorb_kernel<true, 0, true>,
-                        dim3(absorb_blocks + 1), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens,
-                        q_ext, rows, q_len, 0, qscale, tab, *plan);
-    }
-    return launch_pdl(mode == 1 ? q_absorb_kernel<false, 1, true> : q_absorb_kernel<false, 0, true>,
-                      dim3(absorb_blocks), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext,
-                      rows, q_len, 0, qscale, tab, WorkPlanArgs{});
-  }
-  auto kern = [&](bool with_plan) {
     if (with_plan)
+      return launch_pdl(mode == 1 ? q_absorb_kernel<true, 1, true> : q_absorb_kernel<true, 0, true>,
+                        dim3(blocks), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows,
+                        q_len, 0, qscale, tab, plan);
+    return launch_pdl(mode == 1 ? q_absorb_kernel<false, 1, true> : q_absorb_kernel<false, 0, true>,
+                      dim3(blocks), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows,
+                      q_len, 0, qscale, tab, plan);
+  }
+  auto kern = [&](bool p) {
+    if (p)
       return mode == 2 ? q_absorb_kernel<true, 2> : mode == 1 ? q_absorb_kernel<true, 1>
                                                               : q_absorb_kernel<true, 0>;
     return mode == 2 ? q_absorb_kernel<false, 2> : mode == 1 ? q_absorb_kernel<false, 1>
                                                              : q_absorb_kernel<false, 0>;
   };
-  if (plan != nullptr) {
-    if (!plan_ok(*plan)) return cudaErrorInvalidValue;
-    return launch_pdl(kern(true), dim3(absorb_blocks + 1), dim3(kAbsorbThreads), 0, st, q, W_UK,
-                      seqlens, q_ext, rows, q_len, split, qscale, tab, *plan);
-  }
-  return launch_pdl(kern(false), dim3(absorb_blocks), dim3(kAbsorbThreads), 0, st, q, W_UK,
-                    seqlens, q_ext, rows, q_len, split, qscale, tab, WorkPlanArgs{});
+  return launch_pdl(kern(with_plan), dim3(blocks), dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens,
+                    q_ext, rows, q_len, split, qscale, tab, plan);
 }
 
 cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                                  const int32_t* seqlens, __nv_bfloat16* q_ext, int rows,
                                  int q_len, int split, float qscale, const RopeTable& q_tab,
                                  const AppendArgs& ap, const RopeTable& k_tab,
-                                 const ProduceArgs* pa, const WorkPlanArgs* plan,
+                                 const ProduceArgs* pa, const WorkPlanArgs& plan, bool with_plan,
                                  bool rope_only, cudaStream_t st) {
   const int64_t append_blocks = (ap.T * kRowPieces + kAbsorbThreads - 1) / kAbsorbThreads;
   if (append_blocks > (1 << 20)) return cudaErrorInvalidValue;
@@ -472,22 +490,17 @@ cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_
   const int64_t absorb_blocks = mode == 2   ? (int64_t)AbsorbGrid<2>::blocks(rows)
                                : mode == 1 ? (int64_t)kAbsorbBlocks * nrb
                                            : kAbsorbBlocks;
-  auto kern = [&](bool with_plan) {
-    if (with_plan)
+  auto kern = [&](bool with) {
+    if (with)
       return mode == 2 ? step_prologue_kernel<true, 2>
                        : mode == 1 ? step_prologue_kernel<true, 1> : step_prologue_kernel<true, 0>;
     return mode == 2 ? step_prologue_kernel<false, 2>
                      : mode == 1 ? step_prologue_kernel<false, 1> : step_prologue_kernel<false, 0>;
   };
-  if (plan != nullptr) {
-    if (!plan_ok(*plan)) return cudaErrorInvalidValue;
-    return launch_pdl(kern(true), dim3((unsigned)(absorb_blocks + 1 + prod_blocks + append_blocks)),
-                      dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, split,
-                      qscale, q_tab, ap, k_tab, p, *plan);
-  }
-  return launch_pdl(kern(false), dim3((unsigned)(absorb_blocks + prod_blocks + append_blocks)),
-                    dim3(kAbsorbThreads), 0, st, q, W_UK, seqlens, q_ext, rows, q_len, split,
-                    qscale, q_tab, ap, k_tab, p, WorkPlanArgs{});
+  if (with_plan && !plan_ok(plan)) return cudaErrorInvalidValue;
+  const int64_t blocks = absorb_blocks + (with_plan ? 1 : 0) + prod_blocks + append_blocks;
+  return launch_pdl(kern(with_plan), dim3((unsigned)blocks), dim3(kAbsorbThreads), 0, st, q, W_UK,
+                    seqlens, q_ext, rows, q_len, split, qscale, q_tab, ap, k_tab, p, plan);
 }
 
 // ---------------------------------------------------------------- combine + W_UV

@@ -43,19 +43,26 @@ struct WorkPlanArgs {
   // (the mixed kernel runs one pass per query over a short sequence)
   int32_t short_pages;
   int32_t short_weight;
+  // block-table lines (32 entries of 128 B each) every block of the first
+  // kernel helps bring into L2, so that the split-K kernel's first block-id
+  // reads hit it; 0 = none.  Read by every launch of the first kernel, with
+  // or without a plan.
+  const int32_t* bt_prefetch;
+  int64_t bt_lines;
 };
 
 // q_ext[r, h] for rows r = b*q_len + j; qscale = softmax scale * log2 e.
 // split: each query row as a hi and a lo bf16 row (the split-K kernel's
-// split_q layout).  plan (nullable): also compute the length-aware plan.
+// split_q layout).  with_plan: also compute the length-aware plan of `plan`
+// (whose block-table prefetch fields are used either way).
 // rope_only: only the rope columns (the latent part comes from
 // launch_absorb_gemm).
 // f16: q_ext holds f16 values (single rows) for the 8-bit cache's kernel.
 cudaError_t launch_q_absorb(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                             const int32_t* seqlens, __nv_bfloat16* q_ext, int rows, int q_len,
                             int split, float qscale, const RopeTable& tab,
-                            const WorkPlanArgs* plan, bool rope_only, cudaStream_t st,
-                            bool f16 = false);
+                            const WorkPlanArgs& plan, bool with_plan, bool rope_only,
+                            cudaStream_t st, bool f16 = false);
 
 // The new tokens of a decode step, appended by step_prologue_kernel.
 struct AppendArgs {
@@ -74,13 +81,13 @@ struct AppendArgs {
 };
 
 // q_absorb and the cache rows of the same step in one launch: ready rows are
-// appended (ap), rows from hidden states are produced (pa, nullable); plan
-// (nullable) as for launch_q_absorb.
+// appended (ap), rows from hidden states are produced (pa, nullable); plan and
+// with_plan as for launch_q_absorb.
 cudaError_t launch_step_prologue(const __nv_bfloat16* q, const __nv_bfloat16* W_UK,
                                  const int32_t* seqlens, __nv_bfloat16* q_ext, int rows,
                                  int q_len, int split, float qscale, const RopeTable& q_tab,
                                  const AppendArgs& ap, const RopeTable& k_tab,
-                                 const ProduceArgs* pa, const WorkPlanArgs* plan,
+                                 const ProduceArgs* pa, const WorkPlanArgs& plan, bool with_plan,
                                  bool rope_only, cudaStream_t st);
 
 // Merge of the splits and the W_UV product, written to out[rows, 32, 128].

@@ -276,6 +276,10 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
     plan.short_pages = P.mixed ? (int32_t)(kSplitQMaxSeqlen / kPage) : 0;
     plan.short_weight = P.nr / 32;
   }
+  // the first kernel brings the block table into L2 for the split-K kernel's
+  // first block-id reads (after an L2 flush or eviction they would miss)
+  plan.bt_prefetch = block_table;
+  plan.bt_lines = ((int64_t)batch * max_blocks + 31) / 32;
   // Every kernel of the chain waits (griddepcontrol.wait) for its predecessor
   // before reading anything a kernel of this step may have written, so once
   // the first kernel completes all earlier work on the stream has landed.
@@ -305,11 +309,10 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
   const cudaError_t e0 =
       ap != nullptr
           ? launch_step_prologue((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
-                                 rows, q_len, split_arg, qscale, tab, *ap, tab, pa,
-                                 P.table ? &plan : nullptr, P.gemm, st)
+                                 rows, q_len, split_arg, qscale, tab, *ap, tab, pa, plan, P.table,
+                                 P.gemm, st)
           : launch_q_absorb((const __nv_bfloat16*)q, (const __nv_bfloat16*)W_UK, seqlens, q_ext,
-                            rows, q_len, split_arg, qscale, tab,
-                            P.table ? &plan : nullptr, P.gemm, st, q8);
+                            rows, q_len, split_arg, qscale, tab, plan, P.table, P.gemm, st, q8);
   if (e0 != cudaSuccess) return XMLA_ERR_CUDA;
   if (P.gemm && launch_absorb_gemm(tmap_qin, tmap_wuk, gp, st) != cudaSuccess) return XMLA_ERR_CUDA;
 
