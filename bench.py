@@ -309,12 +309,26 @@ def roofline_line(wl, achieved, peak, peak_kind, traffic, cache_bytes, kernel_ms
               "flops_per_launch": flops, "peak_source": tpeak_kind}
     rows = 32 if wl.q_len == 1 or wl.q_len > 8 or wl.max_seqlen <= 4096 else 64
     lead, other = (tensor, hbm) if wl.q_len > 8 else (hbm, tensor)
-    name = "mla_decode_q8_kernel" if q8 else f"mla_decode_kernel<{rows}>"
+    name = ("mla_decode_q8_kernel" if q8 else "prefill_attn_kernel" if wl.q_len >= PREFILL_MIN_CHUNK
+            else f"mla_decode_kernel<{rows}>")
     line = dict(lead, kernel=name, kernel_ms=round(kernel_ms, 5))
     line[other["bound"]] = {k: v for k, v in other.items() if k != "bound"}
     if lead is tensor:
         line["traffic"] = traffic
     return line
+
+
+# a chunk of at least this many new tokens per sequence runs the non-absorbed
+# prompt path (the library's kPrefillMinChunk)
+PREFILL_MIN_CHUNK = 64
+
+
+def pair_flops(wl) -> int:
+    """Algorithmic flop per attended (query, cache token) pair and head of the
+    attention kernel that runs: absorbed (decode, short chunks) QK over 576 and
+    PV over 512 dims, 2 x (576 + 512); non-absorbed (prompt chunks) QK over
+    192 and PV over 128, 2 x (192 + 128)."""
+    return 2 * (192 + 128) if wl.q_len >= PREFILL_MIN_CHUNK else 2 * (576 + 512)
 
 
 def host_mapped(t) -> bool:
@@ -589,16 +603,16 @@ def run_xmla(args, wl):
     gbs = job_throughput(cache_bytes_layer * wl.layers, args.steps, total_ms, world)
     peak, peak_kind = measured_peaks()
     tpeak, tpeak_kind = measured_tensor_peak()
-    # 2176 flop per attended (query row, cache token) pair: QK over 576, PV over 512;
     # query j of a sequence of n tokens attends n - q_len + j + 1 tokens (causal)
     pairs = sum(wl.q_len * (n - wl.q_len) + wl.q_len * (wl.q_len + 1) // 2 for n in wl.seqlens)
-    flops_layer = 2176 * 32 * pairs
+    flops_layer = pair_flops(wl) * 32 * pairs
     attn_mean_ms = statistics.mean(attn_ms)
     achieved = cache_bytes_layer / (attn_mean_ms * 1e-3) / 1e9
     ksha = kernel_sources_sha()
     traffic = None if q8 else traffic_record(ksha, wl.name)
     # per layer and step: prologue (append or producer + q absorb), split-K
-    # attention, combine; on the 8-bit cache the append is a kernel of its own
+    # attention, combine; on the 8-bit cache the append is a kernel of its own; a
+    # prompt chunk: query prep (+ append), K/V expansion, attention
     launches = (4 if q8 else 3) * wl.layers * args.steps
 
     if rank == 0:
@@ -755,7 +769,7 @@ def measure_other(wl, args, dev, cfg, scale):
     del graph
     cache_bytes_layer = sum(wl.seqlens) * ROW_BYTES
     pairs = sum(wl.q_len * (n - wl.q_len) + wl.q_len * (wl.q_len + 1) // 2 for n in wl.seqlens)
-    flops_layer = 2176 * 32 * pairs
+    flops_layer = pair_flops(wl) * 32 * pairs
     peak, peak_kind = measured_peaks()
     tpeak, tpeak_kind = measured_tensor_peak()
     step_mean = statistics.mean(step_ms)

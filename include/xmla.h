@@ -201,9 +201,15 @@ int32_t xmla_decode_num_splits(int32_t batch, int32_t q_len, int64_t max_seqlen,
  * Supported: 1 <= batch, 1 <= q_len <= 65536, q_len <= max_seqlen <= 2^31 - 64,
  * num_blocks*64 < 2^31.  A q_len of a few tokens is a decode step (speculative
  * verification above 1); a long q_len is a chunk of a prompt (chunked
- * prefill), attended causally in the same absorbed form: each query sees the
- * cache up to its own position, and the pages past a CTA's last query are
- * skipped.  Errors: XMLA_ERR_INVALID_ARG, XMLA_ERR_SHAPE,
+ * prefill), attended causally: each query sees the cache up to its own
+ * position.  Up to 63 new tokens per sequence the chunk runs in the same
+ * absorbed form as a decode step; from 64 on, in the non-absorbed form of the
+ * MLA module ([P5] MLA section: kv_b_proj expands K_nope and V per head from
+ * the cached latent): K_nope and V of every cached token are expanded per
+ * head into the workspace, then attention runs per head over [K_nope |
+ * rotated k_pe] and V with fp16 tensor-core operands.  The workspace then
+ * holds, per sequence, max_seqlen (rounded up to 128) tokens x 32 heads x 256
+ * fp16 values.  Errors: XMLA_ERR_INVALID_ARG, XMLA_ERR_SHAPE,
  * XMLA_ERR_WORKSPACE, XMLA_ERR_CUDA, XMLA_ERR_UNSUPPORTED (not an sm_100
  * device); device errors via status_dev. */
 xmla_status xmla_decode(const xmla_yarn_cfg* cfg, const void* q, const void* W_UK,

@@ -16,8 +16,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libxmla.so")
 SOURCES = ["rope_append.cu", "mla_decode.cu", "absorb_combine.cu", "xmla_api.cu", "kv_produce.cu",
-           "head_gemm.cu", "mla_decode_q8.cu", "q8_append.cu"]
+           "head_gemm.cu", "mla_decode_q8.cu", "q8_append.cu", "prefill.cu"]
 HEADERS = ["xmla_device.cuh", "yarn.cuh", "append.cuh", "decode_chain.h", "split_kv.h", "produce.cuh",
+           "prefill.h",
            os.path.join("..", "..", "include", "xmla.h")]
 
 NVCC_FLAGS = [

@@ -1,0 +1,691 @@
+// Prompt chunks in the non-absorbed form, on the tensor cores.
+//
+// [P5] "mHC+MLA+MTP 是什么？拆开给 Agent 用的百亿 MoE", section "MLA：256K 上下文的
+//      '内存革命'": kv_b_proj expands K_nope and V per head (32 x (128 + 128)) from
+//      the cached 512-dim latent; attention then runs per head over
+//      [K_nope | rotated k_pe] (192 dims) and V (128 dims).
+// [P1] "256K 长上下文真能本地用：Xing4.0 原生长上下文的工程代价拆解", section 三 (方案 D):
+//      prompt processing is what grows with the context.
+//
+// A decode step has one query per sequence and is bound by reading the cache
+// once, which the absorbed form does.  A prompt chunk has hundreds or
+// thousands of queries per sequence, and every cached token is attended by all
+// of them: the work is the products, and the non-absorbed form needs 2 x (192
+// + 128) flop per (query, token, head) against 2 x (576 + 512) absorbed.  A
+// chunk runs three kernels, chained with programmatic dependent launch:
+//   prep    the queries as fp16 rows [q_nope | rope(q_pe)] (and, for a decode
+//           step, the append of the chunk's cache rows);
+//   expand  K_nope[t, h] = W_UK[h] c_kv[t] and V[t, h] = W_UV[h]^T c_kv[t] for
+//           every cached token of each sequence, a tcgen05 GEMM (bf16 inputs,
+//           fp32 accumulators) written as fp16, and the rotated rope key
+//           copied out as fp16;
+//   attend  per (sequence, head, tile of 128 queries): flash-style attention
+//           over tiles of 128 tokens, S = Q K^T and O += P V on tcgen05 with
+//           fp16 operands and fp32 accumulators in tensor memory, one softmax
+//           thread per query row, the output written directly (V already
+//           carries W_UV).
+// fp16 operands carry 11 significant bits: emulating these roundings on the
+// CPU keeps every element of a fresh prompt within 1e-2 + 2^-8 |ref| of the
+// fp64 definition, where bf16 operands (8 bits) do not.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "append.cuh"
+#include "decode_chain.h"
+#include "prefill.h"
+
+namespace xmla {
+
+namespace {
+
+constexpr uint32_t kTile = 16384;  // one 128-row x 64-element box of 2-byte values (128-byte rows)
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int32_t x, int32_t y,
+                                            int32_t z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// kind::f16 products take fp16 or bf16 operands; the instruction descriptor
+// carries which (idesc_f16_f32 / idesc_bf16_f32)
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  tc_mma_bf16(d_tmem, a_desc, b_desc, idesc, accumulate);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// ---------------------------------------------------------------- prep
+
+constexpr int kPrepThreads = 256;
+constexpr int kPrepRows = 4;  // query rows (all 32 heads) per block
+
+// Blocks [0, ceil(rows / kPrepRows)): qh[r, h] = [q_nope | rope(q_pe, pos_r)]
+// as fp16, pos_r = seqlens[b] - q_len + j for r = b * q_len + j (the angle in
+// float64 once per (row, pair), as rope_pair).  The blocks after them append
+// the chunk's ready cache rows (one thread per 16-byte piece, the rope key
+// rotated on the way), as the decode step's first kernel does.
+__global__ void __launch_bounds__(kPrepThreads)
+    prefill_prep_kernel(const __nv_bfloat16* q, const int32_t* seqlens, __half* __restrict__ qh,
+                        int rows, int q_len, const RopeTable q_tab, const AppendArgs ap,
+                        const RopeTable k_tab) {
+  __shared__ double cs[kPrepRows][kDRope / 2][2];
+  pdl_wait();  // q, the lengths and the cache may come from the kernel launched before
+  pdl_launch_dependents();
+  const int t = threadIdx.x;
+  const int q_blocks = (rows + kPrepRows - 1) / kPrepRows;
+  if ((int)blockIdx.x < q_blocks) {
+    const int r_lo = blockIdx.x * kPrepRows;
+    const int nr = min(kPrepRows, rows - r_lo);
+    constexpr int kPairs = kDRope / 2;
+    if (t < nr * kPairs) {
+      const int rr = t / kPairs, i = t % kPairs;
+      const int r = r_lo + rr;
+      const int64_t pos = (int64_t)seqlens[r / q_len] - q_len + (r % q_len);
+      double s, c;
+      sincos((double)pos * q_tab.inv_freq[i], &s, &c);
+      cs[rr][i][0] = c * q_tab.magnitude;
+      cs[rr][i][1] = s * q_tab.magnitude;
+    }
+    __syncthreads();
+    // q_nope: 16 pieces of 8 values per (row, head)
+    for (int e = t; e < nr * kHeads * 16; e += kPrepThreads) {
+      const int64_t rh = (int64_t)r_lo * kHeads + e / 16;
+      const int u = e % 16;
+      const uint4 v = *reinterpret_cast<const uint4*>(q + rh * kDQ + 8 * u);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+      uint4 o;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ow[k] = pack_half2(__low2float(b2[k]), __high2float(b2[k]));
+      *reinterpret_cast<uint4*>(qh + rh * kDQ + 8 * u) = o;
+    }
+    // rotated q_pe: pair (i, i + 32) of every (row, head)
+    for (int e = t; e < nr * kHeads * kPairs; e += kPrepThreads) {
+      const int rr = e / (kHeads * kPairs), i = e % kPairs;
+      const int64_t rh = (int64_t)(r_lo + rr) * kHeads + (e / kPairs) % kHeads;
+      const __nv_bfloat16* x = q + rh * kDQ + kDNope;
+      const double x1 = (double)__bfloat162float(x[i]), x2 = (double)__bfloat162float(x[i + kPairs]);
+      const double c = cs[rr][i][0], s = cs[rr][i][1];
+      __half* o = qh + rh * kDQ + kDNope;
+      o[i] = __double2half(x1 * c - x2 * s);
+      o[i + kPairs] = __double2half(x2 * c + x1 * s);
+    }
+    return;
+  }
+  const int64_t idx = (int64_t)(blockIdx.x - q_blocks) * kPrepThreads + t;
+  if (idx < ap.T * kRowPieces)
+    append_piece(idx, ap.pool, ap.num_blocks, ap.block_table, ap.max_blocks, ap.batch, ap.seq_ids,
+                 ap.positions, ap.c_kv, ap.k_pe, ap.status, ap.rotate, k_tab);
+}
+
+// ---------------------------------------------------------------- expand
+
+// One CTA: 128 tokens (two cache pages) x one head.  D_K[t, d] = sum_c c_kv[t, c]
+// W_UK[h][d][c] and D_V[t, v] = sum_c c_kv[t, c] W_UV[h][c][v], K = 512 latent
+// dims in 4 stages of 128 through a 2-stage ring.  The A operand (the pages'
+// latent columns) is K-major; W_UK[h] is K-major as stored ([d][c]) and
+// W_UV[h] MN-major ([c][v]); all by TMA with the 128-byte swizzle.
+constexpr int kExpThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kExpStages = 2;
+constexpr uint32_t kExpStageBytes = 6 * kTile;  // A: 2 K-chunks; B_K: 2; B_V: 2 N-halves
+constexpr uint32_t kExpOffBars = kExpStages * kExpStageBytes;
+constexpr int kExpNumBars = 2 * kExpStages + 1;  // full, empty, done
+constexpr uint32_t kExpOffTmem = kExpOffBars + 8 * kExpNumBars;
+constexpr uint32_t kExpOffAbort = kExpOffTmem + 4;
+constexpr uint32_t kExpSmem = kExpOffAbort + 4 + 1024;
+static_assert(kExpSmem <= 232448, "shared memory per CTA");
+
+__global__ void __launch_bounds__(kExpThreads, 1)
+    kv_expand_kernel(const __grid_constant__ CUtensorMap tmap_pool,
+                     const __grid_constant__ CUtensorMap tmap_wuk,
+                     const __grid_constant__ CUtensorMap tmap_wuv, const PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint32_t base = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  base += pad;
+  auto bar = [&](int i) -> uint32_t { return base + kExpOffBars + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kExpOffAbort);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int64_t t0 = (int64_t)blockIdx.x * 128;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kExpStages; ++s) {
+      mbar_init(bar(s), 1);
+      mbar_init(bar(kExpStages + s), 1);
+    }
+    mbar_init(bar(2 * kExpStages), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(base + kExpOffTmem, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + kExpOffTmem);
+  pdl_wait();  // the chunk's rows were appended by the kernel launched before
+  pdl_launch_dependents();
+  int64_t seqlen = p.seqlens[b];
+  if (seqlen < p.q_len || seqlen > p.max_seqlen) {
+    if (threadIdx.x == 0) record_status(p.status, XMLA_ERR_DEVICE_OOB);
+    seqlen = 0;
+  }
+  const bool active = t0 < seqlen;
+
+  if (warp == 0) {
+    if (lane == 0 && active) {
+      tma_prefetch_desc(&tmap_pool);
+      tma_prefetch_desc(&tmap_wuk);
+      tma_prefetch_desc(&tmap_wuv);
+      // the tile's two pages; a page past the sequence's end is replaced by the
+      // first (its rows are never written out)
+      const int64_t pg0 = t0 / kPage;
+      const int64_t npages = (seqlen + kPage - 1) / kPage;
+      int32_t blk[2];
+      for (int k = 0; k < 2; ++k) {
+        const int64_t pg = pg0 + k < npages ? pg0 + k : pg0;
+        int32_t bk = p.block_table[(int64_t)b * p.max_blocks + pg];
+        if (bk < 0 || (int64_t)bk >= p.num_blocks) {
+          record_status(p.status, XMLA_ERR_DEVICE_OOB);
+          bk = (int32_t)p.num_blocks;  // past the end: the tensor copy reads zeros
+        }
+        blk[k] = bk;
+      }
+      int issued = 0;
+      for (int c = 0; c < 4; ++c) {
+        const int s = c % kExpStages;
+        if (c >= kExpStages &&
+            !mbar_wait(bar(kExpStages + s), (uint32_t)(((c - kExpStages) / kExpStages) & 1),
+                       abort_flag, p.status, p.wait_limit_ns))
+          break;
+        const uint32_t st = base + s * kExpStageBytes;
+        mbar_arrive_expect_tx(bar(s), kExpStageBytes);
+        for (int k = 0; k < 2; ++k)      // A: latent columns 128c + 64k of both pages
+          for (int pg = 0; pg < 2; ++pg)
+            tma_load_2d(st + k * kTile + pg * (kTile / 2), &tmap_pool, 128 * c + 64 * k,
+                        blk[pg] * kPage, bar(s));
+        for (int k = 0; k < 2; ++k)      // B_K: W_UK[h] rows d, columns 128c + 64k
+          tma_load_2d(st + (2 + k) * kTile, &tmap_wuk, 128 * c + 64 * k, h * kDNope, bar(s));
+        for (int j = 0; j < 2; ++j)      // B_V: W_UV[h] rows 128c.., v columns 64j..
+          tma_load_2d(st + (4 + j) * kTile, &tmap_wuv, 64 * j, h * kDLatent + 128 * c, bar(s));
+        ++issued;
+      }
+      for (int c = issued > kExpStages ? issued - kExpStages : 0; c < issued; ++c)
+        mbar_wait(bar(c % kExpStages), (uint32_t)((c / kExpStages) & 1), nullptr, p.status,
+                  p.wait_limit_ns);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && active) {
+      constexpr uint32_t idesc_k = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_v = idesc_bf16_f32(128, 128, false, true);
+      bool ok = true;
+      for (int c = 0; c < 4 && ok; ++c) {
+        const int s = c % kExpStages;
+        if (!(ok = mbar_wait(bar(s), (uint32_t)((c / kExpStages) & 1), abort_flag, p.status,
+                             p.wait_limit_ns)))
+          break;
+        tc_fence_after();
+        const uint32_t st = base + s * kExpStageBytes;
+        const uint64_t a_desc = smem_desc_sw128(st, 16, 1024);
+        const uint64_t bk_desc = smem_desc_sw128(st + 2 * kTile, 16, 1024);
+        const uint64_t bv_desc = smem_desc_sw128(st + 4 * kTile, kTile, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {  // K = 128 in steps of 16
+          const uint32_t kmaj = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
+          const uint32_t acc = (c | k) != 0 ? 1u : 0u;
+          tc_mma_bf16(tmem_base, a_desc + kmaj, bk_desc + kmaj, idesc_k, acc);
+          tc_mma_bf16(tmem_base + 128, a_desc + kmaj, bv_desc + ((k * 2048) >> 4), idesc_v, acc);
+        }
+        tc_commit(bar(kExpStages + s));
+      }
+      tc_commit(bar(2 * kExpStages));
+    }
+  } else if (active) {
+    // epilogue: thread = token row; fp32 -> fp16, 256 contiguous bytes per output row;
+    // rows past the sequence's end are written as zeros (the attention reads the
+    // whole 128-token tile that holds the last token, and a zero probability
+    // times a value read from an unwritten row could be NaN)
+    const int quarter = warp & 3;
+    const int64_t t = t0 + 32 * quarter + lane;
+    const bool valid = active && t < seqlen;
+    const int64_t row = (int64_t)b * p.s_pad + t;
+    const bool ok = mbar_wait(bar(2 * kExpStages), 0, abort_flag, p.status, p.wait_limit_ns);
+    tc_fence_after();
+    const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quarter) << 16);
+#pragma unroll 1
+    for (int part = 0; part < 2; ++part) {  // K_nope, then V
+      __half* dst = (part == 0 ? p.kx : p.vx) + (row * kHeads + h) * 128;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float v[32];
+        tmem_ld32(t_lane + part * 128 + 32 * cc, v);
+        tc_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          w[k] = valid && ok ? pack_half2(v[2 * k], v[2 * k + 1]) : 0u;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          reinterpret_cast<uint4*>(dst + 32 * cc)[u] =
+              make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      }
+    }
+    // the rotated rope key, shared by all heads: written by the head-0 CTA of the tile
+    if (h == 0) {
+      uint4 o[8];
+      if (valid) {
+        const int32_t bk = p.block_table[(int64_t)b * p.max_blocks + t / kPage];
+        const bool in = bk >= 0 && (int64_t)bk < p.num_blocks;
+        const uint4* src =
+            reinterpret_cast<const uint4*>(p.pool + ((int64_t)bk * kPage + t % kPage) * kDRow + kDLatent);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 x = in ? src[u] : make_uint4(0u, 0u, 0u, 0u);
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+          o[u] = make_uint4(pack_half2(__low2float(b2[0]), __high2float(b2[0])),
+                            pack_half2(__low2float(b2[1]), __high2float(b2[1])),
+                            pack_half2(__low2float(b2[2]), __high2float(b2[2])),
+                            pack_half2(__low2float(b2[3]), __high2float(b2[3])));
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) o[u] = make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) reinterpret_cast<uint4*>(p.kp + row * kDRope)[u] = o[u];
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, 256);
+  }
+}
+
+// ---------------------------------------------------------------- attend
+
+// One CTA: 128 queries of one sequence x one head.  Tensor memory: two S
+// buffers [128 queries x 128 tokens] (columns 0 and 128) and O [128 x 128 v]
+// (columns 256..383), fp32.  Shared memory: Q (3 boxes of 64 dims), two K
+// stages (K_nope: 2 boxes, rope key: 1 box), one V stage (2 boxes of 64 v),
+// one P tile (2 boxes of 64 tokens).
+constexpr int kAttThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 softmax (a row each)
+constexpr uint32_t kAttOffQ = 0;
+constexpr uint32_t kAttOffK = kAttOffQ + 3 * kTile;
+constexpr uint32_t kAttKStage = 3 * kTile;
+constexpr uint32_t kAttOffV = kAttOffK + 2 * kAttKStage;
+constexpr uint32_t kAttOffP = kAttOffV + 2 * kTile;
+constexpr uint32_t kAttOffBars = kAttOffP + 2 * kTile;
+// barriers
+constexpr int kBQ = 0;
+constexpr int kBKFull = 1;    // 2
+constexpr int kBKEmpty = 3;   // 2
+constexpr int kBVFull = 5;
+constexpr int kBSFull = 6;    // 2
+constexpr int kBSFree = 8;    // 2
+constexpr int kBPFull = 10;
+constexpr int kBPvDone = 11;
+constexpr int kBDrain = 12;
+constexpr int kAttNumBars = 13;
+constexpr uint32_t kAttOffTmem = kAttOffBars + 8 * kAttNumBars;
+constexpr uint32_t kAttOffAbort = kAttOffTmem + 4;
+constexpr uint32_t kAttSmem = kAttOffAbort + 4 + 1024;
+static_assert(kAttSmem <= 232448, "shared memory per CTA");
+constexpr uint32_t kColS = 0, kColO = 256;
+// a row's running maximum is raised only when a score passes it by this much
+// (log2 units), so an O rescale is rare
+constexpr float kAttLazyMax = 8.0f;
+
+__global__ void __launch_bounds__(kAttThreads, 1)
+    prefill_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                        const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_kp,
+                        const __grid_constant__ CUtensorMap tmap_v, const PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint32_t base = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  base += pad;
+  auto bar = [&](int i) -> uint32_t { return base + kAttOffBars + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kAttOffAbort);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // the last query tiles see the most tokens: they run first
+  const int qt = (int)(gridDim.x - 1 - blockIdx.x);
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int j0 = qt * 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBQ), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBKFull + i), 1);
+      mbar_init(bar(kBKEmpty + i), 1);
+      mbar_init(bar(kBSFull + i), 1);
+      mbar_init(bar(kBSFree + i), 128);
+    }
+    mbar_init(bar(kBVFull), 1);
+    mbar_init(bar(kBPFull), 128);
+    mbar_init(bar(kBPvDone), 1);
+    mbar_init(bar(kBDrain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(base + kAttOffTmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + kAttOffTmem);
+  pdl_wait();  // Q, K, V and the rope key come from the kernels launched before
+  pdl_launch_dependents();
+  int64_t seqlen = p.seqlens[b];
+  if (seqlen < p.q_len || seqlen > p.max_seqlen) {
+    if (threadIdx.x == 0) record_status(p.status, XMLA_ERR_DEVICE_OOB);
+    seqlen = 0;
+  }
+  const int jn = seqlen > 0 ? min(p.q_len - j0, 128) : 0;  // queries of this tile
+  // key tiles: every token up to the tile's last query position
+  const int nt = jn > 0 ? (int)((seqlen - p.q_len + j0 + jn - 1) / 128 + 1) : 0;
+  const int64_t krow0 = (int64_t)b * p.s_pad;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && nt > 0) {
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_kp);
+      tma_prefetch_desc(&tmap_v);
+      const int32_t qrow0 = b * p.q_len + j0;
+      mbar_arrive_expect_tx(bar(kBQ), 3 * kTile);
+      for (int k = 0; k < 3; ++k)
+        tma_load_3d(base + kAttOffQ + k * kTile, &tmap_q, 64 * k, h, qrow0, bar(kBQ));
+      auto load_k = [&](int i) {
+        const int s = i & 1;
+        if (i >= 2 && !mbar_wait(bar(kBKEmpty + s), (uint32_t)(((i - 2) >> 1) & 1), abort_flag,
+                                 p.status, p.wait_limit_ns))
+          return false;
+        const uint32_t st = base + kAttOffK + s * kAttKStage;
+        const int32_t r = (int32_t)(krow0 + 128 * (int64_t)i);
+        mbar_arrive_expect_tx(bar(kBKFull + s), kAttKStage);
+        tma_load_3d(st, &tmap_k, 0, h, r, bar(kBKFull + s));
+        tma_load_3d(st + kTile, &tmap_k, 64, h, r, bar(kBKFull + s));
+        tma_load_2d(st + 2 * kTile, &tmap_kp, 0, r, bar(kBKFull + s));
+        return true;
+      };
+      auto load_v = [&](int i) {
+        if (i >= 1 && !mbar_wait(bar(kBPvDone), (uint32_t)((i - 1) & 1), abort_flag, p.status,
+                                 p.wait_limit_ns))
+          return false;
+        const int32_t r = (int32_t)(krow0 + 128 * (int64_t)i);
+        mbar_arrive_expect_tx(bar(kBVFull), 2 * kTile);
+        tma_load_3d(base + kAttOffV, &tmap_v, 0, h, r, bar(kBVFull));
+        tma_load_3d(base + kAttOffV + kTile, &tmap_v, 64, h, r, bar(kBVFull));
+        return true;
+      };
+      // order: K0, K1, V0, then K(i + 1), V(i): V(i) waits for PV(i - 1), K(i + 1)
+      // only for QK(i - 1)
+      bool ok = load_k(0);
+      int k_issued = ok ? 1 : 0, v_issued = 0;
+      if (ok && nt > 1) ok = load_k(1), k_issued += ok;
+      if (ok) ok = load_v(0), v_issued += ok;
+      for (int i = 1; i < nt && ok; ++i) {
+        if (i + 1 < nt) {
+          if (!(ok = load_k(i + 1))) break;
+          ++k_issued;
+        }
+        if (!(ok = load_v(i))) break;
+        ++v_issued;
+      }
+      // every copy issued must land before the CTA may exit
+      mbar_wait(bar(kBQ), 0, nullptr, p.status, p.wait_limit_ns);
+      for (int i = k_issued > 2 ? k_issued - 2 : 0; i < k_issued; ++i)
+        mbar_wait(bar(kBKFull + (i & 1)), (uint32_t)((i >> 1) & 1), nullptr, p.status,
+                  p.wait_limit_ns);
+      if (v_issued > 0)
+        mbar_wait(bar(kBVFull), (uint32_t)((v_issued - 1) & 1), nullptr, p.status, p.wait_limit_ns);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nt > 0) {
+      constexpr uint32_t idesc_qk = idesc_f16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_f16_f32(128, 128, false, true);
+      const uint64_t d_q = smem_desc_sw128(base + kAttOffQ, 16, 1024);
+      const uint64_t d_k = smem_desc_sw128(base + kAttOffK, 16, 1024);
+      const uint64_t d_p = smem_desc_sw128(base + kAttOffP, 16, 1024);
+      const uint64_t d_v = smem_desc_sw128(base + kAttOffV, kTile, 1024);
+      auto wait = [&](int idx, uint32_t parity) {
+        return mbar_wait(bar(idx), parity, abort_flag, p.status, p.wait_limit_ns);
+      };
+      auto qk = [&](int i) {
+        const int s = i & 1;
+        if (!wait(kBKFull + s, (uint32_t)((i >> 1) & 1))) return false;
+        if (i >= 2 && !wait(kBSFree + s, (uint32_t)(((i - 2) >> 1) & 1))) return false;
+        tc_fence_after();
+        const uint64_t bk = d_k + ((s * kAttKStage) >> 4);
+#pragma unroll
+        for (int k = 0; k < 12; ++k) {  // K = 192 in steps of 16
+          const uint32_t off = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
+          tc_mma_f16(tmem_base + kColS + 128 * s, d_q + off, bk + off, idesc_qk, k != 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kBKEmpty + s));
+        tc_commit(bar(kBSFull + s));
+        return true;
+      };
+      bool ok = wait(kBQ, 0);
+      tc_fence_after();
+      if (ok) ok = qk(0);
+      for (int i = 0; i < nt && ok; ++i) {
+        if (i + 1 < nt && !(ok = qk(i + 1))) break;
+        if (!(ok = wait(kBPFull, (uint32_t)(i & 1)))) break;
+        if (!(ok = wait(kBVFull, (uint32_t)(i & 1)))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {  // K = 128 tokens in steps of 16
+          const uint32_t aoff = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
+          tc_mma_f16(tmem_base + kColO, d_p + aoff, d_v + ((k * 2048) >> 4), idesc_pv,
+                     (i | k) != 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kBPvDone));
+      }
+      tc_commit(bar(kBDrain));
+      mbar_wait(bar(kBDrain), 0, nullptr, p.status, p.wait_limit_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax, one query row per thread
+    const int quarter = warp & 3;
+    const int row = 32 * quarter + lane;  // tensor-memory lane = query row of the tile
+    const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quarter) << 16);
+    const int j = j0 + row;
+    // the row's last visible token (the query's own position); -1 for a padding row
+    const int64_t qpos = j < j0 + jn ? seqlen - p.q_len + j : -1;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < nt; ++i) {
+      const int s = i & 1;
+      ok = mbar_wait(bar(kBSFull + s), (uint32_t)((i >> 1) & 1), abort_flag, p.status,
+                     p.wait_limit_ns);
+      tc_fence_after();
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float tmp[32];
+        tmem_ld32(t_lane + kColS + 128 * s + 32 * c, tmp);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) x[32 * c + k] = tmp[k];
+      }
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(kBSFree + s));
+      const int64_t tbase = 128 * (int64_t)i;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 128; ++k) {
+        x[k] = tbase + k <= qpos ? x[k] * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[k]);
+      }
+      // P and O of the previous tile are in use until its PV product completes
+      bool okp = true;
+      if (i >= 1)
+        okp = mbar_wait(bar(kBPvDone), (uint32_t)((i - 1) & 1), abort_flag, p.status,
+                        p.wait_limit_ns);
+      if (__any_sync(0xffffffffu, !ok || !okp)) {
+        ok = false;
+        break;
+      }
+      const bool raise = mx > m_used + kAttLazyMax;
+      if (__any_sync(0xffffffffu, raise)) {
+        // the warp rescales its rows of O together (tensor-memory access is per warp)
+        const float m_new = raise ? mx : m_used;
+        const float alpha = m_used == -INFINITY ? 0.f : ex2(m_used - m_new);
+        l *= raise ? alpha : 1.f;
+        if (i >= 1) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(t_lane + kColO + 32 * c, o);
+            tc_wait_ld();
+            const float f = raise ? alpha : 1.f;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] *= f;
+            tmem_st32(t_lane + kColO + 32 * c, o);
+          }
+          tc_wait_st();
+        }
+        m_used = m_new;
+      }
+      // probabilities as fp16 pairs, summed in that precision; the row is one
+      // 128-byte line in each of the two 64-token boxes of P (128-byte swizzle)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint8_t* prow = smem + kAttOffP + c * kTile + row * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = 64 * c + 8 * u + 2 * e;
+            const float p0 = x[k] == -INFINITY ? 0.f : ex2(x[k] - m_used);
+            const float p1 = x[k + 1] == -INFINITY ? 0.f : ex2(x[k + 1] - m_used);
+            const __half2 hv = __floats2half2_rn(p0, p1);
+            l += __low2float(hv) + __high2float(hv);
+            w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
+          *reinterpret_cast<uint4*>(prow + ((u ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(kBPFull));
+    }
+    // ---- epilogue: O / l, written as the bf16 output row of (query, head)
+    bool have = ok && nt > 0;
+    if (have) {
+      const bool okw = mbar_wait(bar(kBPvDone), (uint32_t)((nt - 1) & 1), abort_flag, p.status,
+                                 p.wait_limit_ns);
+      have = !__any_sync(0xffffffffu, !okw);
+    }
+    if (have) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = p.out + ((int64_t)(b * p.q_len + j) * kHeads + h) * kDV;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(t_lane + kColO + 32 * c, o);
+        tc_wait_ld();
+        if (qpos >= 0) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 v =
+                  __floats2bfloat162_rn(o[8 * u + 2 * e] * inv, o[8 * u + 2 * e + 1] * inv);
+              w[e] = *reinterpret_cast<const uint32_t*>(&v);
+            }
+            reinterpret_cast<uint4*>(dst + 32 * c)[u] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <typename Kern>
+static cudaError_t set_smem(Kern k, uint32_t bytes, bool* done) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!done[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    done[dev] = true;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_prep(const __nv_bfloat16* q, const int32_t* seqlens, __half* qh, int rows,
+                                int q_len, const RopeTable& q_tab, const AppendArgs& ap,
+                                const RopeTable& k_tab, cudaStream_t st) {
+  const int64_t q_blocks = (rows + kPrepRows - 1) / kPrepRows;
+  const int64_t a_blocks = (ap.T * kRowPieces + kPrepThreads - 1) / kPrepThreads;
+  if (q_blocks + a_blocks > (1 << 30)) return cudaErrorInvalidValue;
+  return launch_pdl(prefill_prep_kernel, dim3((unsigned)(q_blocks + a_blocks)), dim3(kPrepThreads),
+                    0, st, q, seqlens, qh, rows, q_len, q_tab, ap, k_tab);
+}
+
+cudaError_t launch_kv_expand(const CUtensorMap& pool_map, const CUtensorMap& wuk_map,
+                             const CUtensorMap& wuv_map, const PrefillParams& p, cudaStream_t st) {
+  static bool done[64] = {};
+  const cudaError_t e = set_smem(kv_expand_kernel, kExpSmem, done);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)(p.s_pad / 128), kHeads, (unsigned)p.batch);
+  return launch_pdl(kv_expand_kernel, grid, dim3(kExpThreads), kExpSmem, st, pool_map, wuk_map,
+                    wuv_map, p);
+}
+
+cudaError_t launch_prefill_attn(const CUtensorMap& q_map, const CUtensorMap& k_map,
+                                const CUtensorMap& kp_map, const CUtensorMap& v_map,
+                                const PrefillParams& p, cudaStream_t st) {
+  static bool done[64] = {};
+  const cudaError_t e = set_smem(prefill_attn_kernel, kAttSmem, done);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((p.q_len + 127) / 128), kHeads, (unsigned)p.batch);
+  return launch_pdl(prefill_attn_kernel, grid, dim3(kAttThreads), kAttSmem, st, q_map, k_map,
+                    kp_map, v_map, p);
+}
+
+}  // namespace xmla

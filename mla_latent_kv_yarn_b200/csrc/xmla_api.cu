@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "decode_chain.h"
+#include "prefill.h"
 
 namespace xmla {
 
@@ -45,6 +46,11 @@ __global__ void wait_timeout_selftest_kernel(int32_t* status, uint64_t limit_ns)
 constexpr int32_t kSplitQMinChunk = 8;
 
 struct Plan {
+  // a prompt chunk of >= kPrefillMinChunk new tokens: the non-absorbed path of
+  // prefill.cu (workspace: qh, kx, vx, kp; s_pad token rows per sequence)
+  bool prefill;
+  int64_t s_pad;
+  size_t off_qh, off_kx, off_vx, off_kp, prefill_bytes;
   bool split;   // hi/lo query (split_q) for every sequence
   bool mixed;   // hi/lo query for the sequences of <= kSplitQMaxSeqlen tokens only
   bool gemm;    // a prompt chunk: absorb and W_UV on the tensor cores (head_gemm.cu)
@@ -66,7 +72,7 @@ static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // q8: the 8-bit cache's kernel (32 rows per CTA, one f16 query row each).
 static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_sms,
                       int32_t num_splits, Plan* pl, int64_t span_pages = 0,
-                      bool allow_table = true, bool q8 = false) {
+                      bool allow_table = true, bool q8 = false, bool allow_prefill = true) {
   if (B < 1 || q_len < 1 || q_len > (q8 ? kQ8MaxQLen : kMaxQLen) || max_seqlen < q_len ||
       max_seqlen > (int64_t)0x7fffffff - kPage || num_sms < 1 || num_splits < 0 || span_pages < 0)
     return false;
@@ -108,6 +114,23 @@ static bool make_plan(int32_t B, int32_t q_len, int64_t max_seqlen, int32_t num_
   P.off_olat = align_up(P.off_utab + (P.table ? (size_t)units * 8 : 0), 1024);
   const size_t olat = P.gemm ? (size_t)B * q_len * kHeads * kDLatent * 2 : 0;
   P.bytes = align_up(P.off_olat + 2 * olat, 1024);
+  // a chunk of >= kPrefillMinChunk tokens runs the non-absorbed path (the
+  // absorbed one above stays for a chunk whose cache rows come from hidden
+  // states); the workspace covers both
+  P.prefill = false;
+  P.s_pad = (max_seqlen + 127) / 128 * 128;
+  P.prefill_bytes = 0;
+  // (the expanded rows' TMA coordinates are int32: past that bound, the absorbed path)
+  if (!q8 && allow_table && q_len >= kPrefillMinChunk &&
+      (int64_t)B * P.s_pad <= (int64_t)0x7fffffff - 128) {
+    P.off_qh = 0;
+    P.off_kx = align_up((size_t)B * q_len * kHeads * kDQ * 2, 1024);
+    P.off_vx = align_up(P.off_kx + (size_t)B * P.s_pad * kHeads * kDNope * 2, 1024);
+    P.off_kp = align_up(P.off_vx + (size_t)B * P.s_pad * kHeads * kDV * 2, 1024);
+    P.prefill_bytes = align_up(P.off_kp + (size_t)B * P.s_pad * kDRope * 2, 1024);
+    P.prefill = allow_prefill;
+    if (P.prefill_bytes > P.bytes) P.bytes = P.prefill_bytes;
+  }
   *pl = P;
   return true;
 }
@@ -164,6 +187,33 @@ static bool encode_weight(CUtensorMap* m, const void* ptr, uint64_t rows, uint64
   cuuint32_t box[2] = {64, 128};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp16 maps of the prompt-chunk path: a 3-D [rows, 32, cols] tensor with box
+// 64 columns x 1 head x 128 rows, and a 2-D [rows, cols] one with box 64 x 128,
+// 128-byte swizzle (K-major 128-row tiles, or MN-major ones read by rows).
+static bool encode_f16_3d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)kHeads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * 2 * kHeads};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool encode_f16_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -238,11 +288,52 @@ static xmla_status run_decode(const xmla_yarn_cfg* cfg, const void* q, const voi
              page_hi != INT64_MAX))
     return XMLA_ERR_INVALID_ARG;
   if (!make_plan(batch, q_len, max_seqlen, nsm, num_splits, &P, span, shard_partial == nullptr,
-                 q8))
+                 q8, pa == nullptr))
     return XMLA_ERR_SHAPE;
   if (workspace_bytes < P.bytes) return XMLA_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
   uint8_t* ws = (uint8_t*)workspace;
+  if (P.prefill) {
+    // a prompt chunk: queries as fp16 rows (and the chunk's append), K_nope / V
+    // expanded per head, then the tensor-core attention writing `out`
+    const int rows = batch * q_len;
+    PrefillParams pp;
+    pp.block_table = block_table;
+    pp.seqlens = seqlens;
+    pp.pool = (const uint16_t*)pool;
+    pp.kx = (__half*)(ws + P.off_kx);
+    pp.vx = (__half*)(ws + P.off_vx);
+    pp.kp = (__half*)(ws + P.off_kp);
+    pp.out = (__nv_bfloat16*)out;
+    pp.status = status_dev;
+    pp.num_blocks = num_blocks;
+    pp.max_seqlen = max_seqlen;
+    pp.s_pad = P.s_pad;
+    pp.wait_limit_ns = kWaitLimitNs;
+    pp.scale_log2 = softmax_scale * kLog2e;
+    pp.max_blocks = max_blocks;
+    pp.batch = batch;
+    pp.q_len = q_len;
+    __half* qh = (__half*)(ws + P.off_qh);
+    const uint64_t krows = (uint64_t)batch * P.s_pad;
+    CUtensorMap m_pool, m_wuk, m_wuv, m_q, m_k, m_v, m_kp;
+    if (!encode_rows576(&m_pool, pool, (uint64_t)num_blocks * kPage, kPage) ||
+        !encode_weight(&m_wuk, W_UK, (uint64_t)kHeads * kDNope, kDLatent) ||
+        !encode_weight(&m_wuv, W_UV, (uint64_t)kHeads * kDLatent, kDV) ||
+        !encode_f16_3d(&m_q, qh, (uint64_t)rows, kDQ) ||
+        !encode_f16_3d(&m_k, pp.kx, krows, kDNope) || !encode_f16_3d(&m_v, pp.vx, krows, kDV) ||
+        !encode_f16_2d(&m_kp, pp.kp, krows, kDRope))
+      return XMLA_ERR_CUDA;
+    const RopeTable tab = make_rope_table(cfg);
+    AppendArgs none{};
+    if (launch_prefill_prep((const __nv_bfloat16*)q, seqlens, qh, rows, q_len, tab,
+                            ap != nullptr ? *ap : none, tab, st) != cudaSuccess ||
+        launch_kv_expand(m_pool, m_wuk, m_wuv, pp, st) != cudaSuccess)
+      return XMLA_ERR_CUDA;
+    if (record_event(attn_start, st) != cudaSuccess) return XMLA_ERR_CUDA;
+    if (launch_prefill_attn(m_q, m_k, m_kp, m_v, pp, st) != cudaSuccess) return XMLA_ERR_CUDA;
+    return record_event(attn_stop, st) == cudaSuccess ? XMLA_OK : XMLA_ERR_CUDA;
+  }
   __nv_bfloat16* q_ext = (__nv_bfloat16*)(ws + P.off_qext);
   const int rows = batch * q_len;
 

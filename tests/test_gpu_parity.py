@@ -318,12 +318,19 @@ def test_short_contexts(q_len, seed):
 # attends causally to the cache up to its own position (the first ones of a
 # fresh prompt see a handful of tokens).
 PREFILL_CASES = [
-    # batch, q_len, seqlens, oracle form
+    # batch, q_len, seqlens, oracle form.  From 64 new tokens per sequence a chunk
+    # runs the non-absorbed tensor-core path (K_nope and V expanded per head, fp16
+    # products); shorter ones the absorbed split-K path.
     (1, 64, [64], "expanded"),             # a fresh 64-token prompt
     (1, 200, [1000], "expanded"),          # a chunk on an 800-token prefix
     (2, 130, [130, 700], "expanded"),      # one fresh prompt, one continued
     (1, 96, [4500], "absorbed"),           # a chunk past 4096 tokens
     (1, 1024, [1024], "absorbed"),
+    (1, 256, [256], "expanded"),           # exactly two tiles of 128 queries
+    (3, 128, [128, 1000, 300], "absorbed"),  # three sequences, different prefixes
+    (1, 64, [9000], "absorbed"),           # 64 queries over 71 key tiles
+    (2, 100, [100, 5000], "absorbed"),
+    (1, 63, [700], "absorbed"),            # one below the tensor-core path: absorbed
     (1, 16, [3000], "absorbed"),           # several splits per unit: merged before W_UV
     (2, 12, [2000, 500], "absorbed"),      # length-aware plan, merged through the unit table
 ]
@@ -336,7 +343,33 @@ def test_prefill_chunk_matches_the_oracle(batch, q_len, seqlens, form):
     inp = workloads.layer_inputs(wl, 0, "cpu")
     out, dec, _ = gc.gpu_step(wl, inp, cfg)
     assert dec.check_status() == 0
-    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, form=form), f"prefill {q_len} {seqlens}")
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg, form=form), f"prefill {q_len} {seqlens}",
+                    plain_below=True)
+
+
+@pytest.mark.parametrize("q_len,seqlens", [(70, [70]), (128, [200])])
+def test_prefill_chunk_ignores_garbage_past_sequence_end(q_len, seqlens):
+    """The pool rows past each sequence's end hold NaN: the expansion writes zeros
+    for them, so a zero probability never meets a NaN value."""
+    wl = workloads.custom(1, q_len, seqlens, seed=31 + q_len)
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    out, dec, _ = gc.gpu_step(wl, inp, cfg, pool_fill=float("nan"))
+    assert dec.check_status() == 0
+    gc.assert_close(out, gc.oracle_out(wl, inp, ocfg), f"prefill nan tail {q_len} {seqlens}")
+
+
+def test_prefill_chunk_plain_decode_call_equals_the_step():
+    """xmla_decode on a cache that already holds the chunk (no append in the call)
+    gives the step's output bit for bit."""
+    wl = workloads.custom(2, 96, [300, 96], seed=5)
+    cfg, _ = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    out, dec, st = gc.gpu_step(wl, inp, cfg)
+    again = dec.decode(cfg, st, inp.q.cuda(), xmla.xmla_softmax_scale(cfg)).clone()
+    torch.cuda.synchronize()
+    assert dec.check_status() == 0
+    assert torch.equal(out.view(torch.int16), again.view(torch.int16))
 
 
 def test_length_aware_plan_is_deterministic():
@@ -499,7 +532,7 @@ def test_workload_prefill_4k_sampled_queries():
         t = n - ql + j + 1
         ref.append(om.mla_attention_absorbed(gc.f64(inp.q[0, j:j + 1]), c[:t], kp_rot[:t], wk, wv,
                                              ocfg)[0])
-    gc.assert_close(out[:, js], {0: np.stack(ref)}, "prefill_4k sampled queries", plain_max_abs=True)
+    gc.assert_close(out[:, js], {0: np.stack(ref)}, "prefill_4k sampled queries", plain_below=True)
 
 
 @pytest.mark.parametrize("layer", [0, 39])
