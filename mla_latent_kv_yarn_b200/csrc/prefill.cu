@@ -323,37 +323,86 @@ __global__ void __launch_bounds__(kExpThreads, 1)
 
 // ---------------------------------------------------------------- attend
 
-// One CTA: 128 queries of one sequence x one head.  Tensor memory: two S
-// buffers [128 queries x 128 tokens] (columns 0 and 128) and O [128 x 128 v]
-// (columns 256..383), fp32.  Shared memory: Q (3 boxes of 64 dims), two K
-// stages (K_nope: 2 boxes, rope key: 1 box), one V stage (2 boxes of 64 v),
-// one P tile (2 boxes of 64 tokens).
-constexpr int kAttThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 softmax (a row each)
+// One CTA: 128 queries of one sequence x one head.  Tensor memory (fp32
+// columns): two S buffers [128 queries x 128 tokens] at 0 and 128, O [128 x
+// 128 v] at 256, and two P buffers [128 x 128 tokens] as fp16 pairs (64
+// columns each) at 384 and 448, the A operand of the PV product.  Shared
+// memory: Q (3 boxes of 64 dims), two K stages (K_nope: 2 boxes, rope key: 1
+// box) and two V stages (2 boxes of 64 v), all by TMA with the 128-byte
+// swizzle; and the row statistics the two softmax threads of a row exchange.
+// warp 0 TMA, warp 1 MMA, warps 2-9 softmax: a query row is shared by warps w
+// and w + 4 (the same tensor-memory lane quarter, w & 3), each taking 64 of a
+// tile's 128 tokens and 64 of the 128 v columns of O
+constexpr int kAttThreads = 320;
+constexpr int kAttSoftmax = 256;
 constexpr uint32_t kAttOffQ = 0;
 constexpr uint32_t kAttOffK = kAttOffQ + 3 * kTile;
 constexpr uint32_t kAttKStage = 3 * kTile;
 constexpr uint32_t kAttOffV = kAttOffK + 2 * kAttKStage;
-constexpr uint32_t kAttOffP = kAttOffV + 2 * kTile;
-constexpr uint32_t kAttOffBars = kAttOffP + 2 * kTile;
+constexpr uint32_t kAttVStage = 2 * kTile;
+// [slot][half][row]: the half-row maxima (float), then the ok flags (int);
+// slots 0, 1 by tile parity, slot 2 for the row sums at the end
+constexpr uint32_t kAttOffXchg = kAttOffV + 2 * kAttVStage;
+constexpr uint32_t kAttXchgSlots = 3 * 2 * 128;
+constexpr uint32_t kAttXchgBytes = 2 * kAttXchgSlots * 4;
+constexpr uint32_t kAttOffBars = kAttOffXchg + kAttXchgBytes;
 // barriers
 constexpr int kBQ = 0;
 constexpr int kBKFull = 1;    // 2
 constexpr int kBKEmpty = 3;   // 2
-constexpr int kBVFull = 5;
-constexpr int kBSFull = 6;    // 2
-constexpr int kBSFree = 8;    // 2
-constexpr int kBPFull = 10;
-constexpr int kBPvDone = 11;
-constexpr int kBDrain = 12;
-constexpr int kAttNumBars = 13;
+constexpr int kBVFull = 5;    // 2
+constexpr int kBVEmpty = 7;   // 2
+constexpr int kBSFull = 9;    // 2
+constexpr int kBSFree = 11;   // 2
+constexpr int kBPFull = 13;   // 2
+constexpr int kBPvDone = 15;  // 2
+constexpr int kBDrain = 17;
+constexpr int kAttNumBars = 18;
 constexpr uint32_t kAttOffTmem = kAttOffBars + 8 * kAttNumBars;
 constexpr uint32_t kAttOffAbort = kAttOffTmem + 4;
 constexpr uint32_t kAttSmem = kAttOffAbort + 4 + 1024;
 static_assert(kAttSmem <= 232448, "shared memory per CTA");
-constexpr uint32_t kColS = 0, kColO = 256;
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 // a row's running maximum is raised only when a score passes it by this much
 // (log2 units), so an O rescale is rare
 constexpr float kAttLazyMax = 8.0f;
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// the two warps that share a lane quarter meet here (named barrier 1 + quarter)
+__device__ __forceinline__ void pair_sync(int quarter) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16: A's rows are tensor-memory
+// lanes, two 16-bit elements per 32-bit column (the lower K index in the low half)
+__device__ __forceinline__ void tc_mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem,
+                                                  uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
 
 __global__ void __launch_bounds__(kAttThreads, 1)
     prefill_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -380,12 +429,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBKFull + i), 1);
       mbar_init(bar(kBKEmpty + i), 1);
+      mbar_init(bar(kBVFull + i), 1);
+      mbar_init(bar(kBVEmpty + i), 1);
       mbar_init(bar(kBSFull + i), 1);
-      mbar_init(bar(kBSFree + i), 128);
+      mbar_init(bar(kBSFree + i), kAttSoftmax);
+      mbar_init(bar(kBPFull + i), kAttSoftmax);
+      mbar_init(bar(kBPvDone + i), 1);
     }
-    mbar_init(bar(kBVFull), 1);
-    mbar_init(bar(kBPFull), 128);
-    mbar_init(bar(kBPvDone), 1);
     mbar_init(bar(kBDrain), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -421,50 +471,37 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       mbar_arrive_expect_tx(bar(kBQ), 3 * kTile);
       for (int k = 0; k < 3; ++k)
         tma_load_3d(base + kAttOffQ + k * kTile, &tmap_q, 64 * k, h, qrow0, bar(kBQ));
-      auto load_k = [&](int i) {
+      // K(i) and V(i) go to stage i % 2 once QK(i - 2) and PV(i - 2) are done
+      int nk = 0, nv = 0;  // tiles whose K, V copies were issued
+      for (int i = 0; i < nt; ++i) {
         const int s = i & 1;
+        const int32_t r = (int32_t)(krow0 + 128 * (int64_t)i);
         if (i >= 2 && !mbar_wait(bar(kBKEmpty + s), (uint32_t)(((i - 2) >> 1) & 1), abort_flag,
                                  p.status, p.wait_limit_ns))
-          return false;
-        const uint32_t st = base + kAttOffK + s * kAttKStage;
-        const int32_t r = (int32_t)(krow0 + 128 * (int64_t)i);
+          break;
+        const uint32_t kst = base + kAttOffK + s * kAttKStage;
         mbar_arrive_expect_tx(bar(kBKFull + s), kAttKStage);
-        tma_load_3d(st, &tmap_k, 0, h, r, bar(kBKFull + s));
-        tma_load_3d(st + kTile, &tmap_k, 64, h, r, bar(kBKFull + s));
-        tma_load_2d(st + 2 * kTile, &tmap_kp, 0, r, bar(kBKFull + s));
-        return true;
-      };
-      auto load_v = [&](int i) {
-        if (i >= 1 && !mbar_wait(bar(kBPvDone), (uint32_t)((i - 1) & 1), abort_flag, p.status,
-                                 p.wait_limit_ns))
-          return false;
-        const int32_t r = (int32_t)(krow0 + 128 * (int64_t)i);
-        mbar_arrive_expect_tx(bar(kBVFull), 2 * kTile);
-        tma_load_3d(base + kAttOffV, &tmap_v, 0, h, r, bar(kBVFull));
-        tma_load_3d(base + kAttOffV + kTile, &tmap_v, 64, h, r, bar(kBVFull));
-        return true;
-      };
-      // order: K0, K1, V0, then K(i + 1), V(i): V(i) waits for PV(i - 1), K(i + 1)
-      // only for QK(i - 1)
-      bool ok = load_k(0);
-      int k_issued = ok ? 1 : 0, v_issued = 0;
-      if (ok && nt > 1) ok = load_k(1), k_issued += ok;
-      if (ok) ok = load_v(0), v_issued += ok;
-      for (int i = 1; i < nt && ok; ++i) {
-        if (i + 1 < nt) {
-          if (!(ok = load_k(i + 1))) break;
-          ++k_issued;
-        }
-        if (!(ok = load_v(i))) break;
-        ++v_issued;
+        tma_load_3d(kst, &tmap_k, 0, h, r, bar(kBKFull + s));
+        tma_load_3d(kst + kTile, &tmap_k, 64, h, r, bar(kBKFull + s));
+        tma_load_2d(kst + 2 * kTile, &tmap_kp, 0, r, bar(kBKFull + s));
+        nk = i + 1;
+        if (i >= 2 && !mbar_wait(bar(kBVEmpty + s), (uint32_t)(((i - 2) >> 1) & 1), abort_flag,
+                                 p.status, p.wait_limit_ns))
+          break;
+        const uint32_t vst = base + kAttOffV + s * kAttVStage;
+        mbar_arrive_expect_tx(bar(kBVFull + s), kAttVStage);
+        tma_load_3d(vst, &tmap_v, 0, h, r, bar(kBVFull + s));
+        tma_load_3d(vst + kTile, &tmap_v, 64, h, r, bar(kBVFull + s));
+        nv = i + 1;
       }
       // every copy issued must land before the CTA may exit
       mbar_wait(bar(kBQ), 0, nullptr, p.status, p.wait_limit_ns);
-      for (int i = k_issued > 2 ? k_issued - 2 : 0; i < k_issued; ++i)
+      for (int i = nk > 2 ? nk - 2 : 0; i < nk; ++i)
         mbar_wait(bar(kBKFull + (i & 1)), (uint32_t)((i >> 1) & 1), nullptr, p.status,
                   p.wait_limit_ns);
-      if (v_issued > 0)
-        mbar_wait(bar(kBVFull), (uint32_t)((v_issued - 1) & 1), nullptr, p.status, p.wait_limit_ns);
+      for (int i = nv > 2 ? nv - 2 : 0; i < nv; ++i)
+        mbar_wait(bar(kBVFull + (i & 1)), (uint32_t)((i >> 1) & 1), nullptr, p.status,
+                  p.wait_limit_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -473,7 +510,6 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       constexpr uint32_t idesc_pv = idesc_f16_f32(128, 128, false, true);
       const uint64_t d_q = smem_desc_sw128(base + kAttOffQ, 16, 1024);
       const uint64_t d_k = smem_desc_sw128(base + kAttOffK, 16, 1024);
-      const uint64_t d_p = smem_desc_sw128(base + kAttOffP, 16, 1024);
       const uint64_t d_v = smem_desc_sw128(base + kAttOffV, kTile, 1024);
       auto wait = [&](int idx, uint32_t parity) {
         return mbar_wait(bar(idx), parity, abort_flag, p.status, p.wait_limit_ns);
@@ -498,135 +534,155 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       if (ok) ok = qk(0);
       for (int i = 0; i < nt && ok; ++i) {
         if (i + 1 < nt && !(ok = qk(i + 1))) break;
-        if (!(ok = wait(kBPFull, (uint32_t)(i & 1)))) break;
-        if (!(ok = wait(kBVFull, (uint32_t)(i & 1)))) break;
+        const int s = i & 1;
+        if (!(ok = wait(kBPFull + s, (uint32_t)((i >> 1) & 1)))) break;
+        if (!(ok = wait(kBVFull + s, (uint32_t)((i >> 1) & 1)))) break;
         tc_fence_after();
+        const uint64_t bv = d_v + ((s * kAttVStage) >> 4);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {  // K = 128 tokens in steps of 16
-          const uint32_t aoff = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
-          tc_mma_f16(tmem_base + kColO, d_p + aoff, d_v + ((k * 2048) >> 4), idesc_pv,
-                     (i | k) != 0 ? 1u : 0u);
-        }
-        tc_commit(bar(kBPvDone));
+        for (int k = 0; k < 8; ++k)  // K = 128 tokens in steps of 16 (8 columns of P)
+          tc_mma_f16_tmem_a(tmem_base + kColO, tmem_base + kColP + 64 * s + 8 * k,
+                            bv + ((k * 2048) >> 4), idesc_pv, (i | k) != 0 ? 1u : 0u);
+        tc_commit(bar(kBVEmpty + s));
+        tc_commit(bar(kBPvDone + s));
       }
       tc_commit(bar(kBDrain));
       mbar_wait(bar(kBDrain), 0, nullptr, p.status, p.wait_limit_ns);
     }
   } else {
-    // ------------------------------------------------------------ softmax, one query row per thread
+    // ------------------------------------------------------------ softmax, half a query row per thread
     const int quarter = warp & 3;
+    const int hf = (warp - 2) >> 2;       // tokens 64 hf .. 64 hf + 63 of a tile; v columns likewise
     const int row = 32 * quarter + lane;  // tensor-memory lane = query row of the tile
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quarter) << 16);
+    float* xmax = reinterpret_cast<float*>(smem + kAttOffXchg);
+    int* xok = reinterpret_cast<int*>(smem + kAttOffXchg + kAttXchgSlots * 4);
     const int j = j0 + row;
     // the row's last visible token (the query's own position); -1 for a padding row
     const int64_t qpos = j < j0 + jn ? seqlen - p.q_len + j : -1;
+    // tiles from here on hold tokens past some row's position: they are masked
+    const int64_t first_masked = (seqlen - p.q_len + j0 + 1) / 128;
+    const float sc = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
-    bool ok = true;
+    bool ok = true, pair_ok = true;
+    // Every exit is taken by both warps of a pair at the same point (after an
+    // exchange), so neither is left waiting at the named barrier; a failed wait
+    // only marks the thread, which finishes the tile on whatever it read.
     for (int i = 0; i < nt; ++i) {
       const int s = i & 1;
-      ok = mbar_wait(bar(kBSFull + s), (uint32_t)((i >> 1) & 1), abort_flag, p.status,
-                     p.wait_limit_ns);
+      ok &= mbar_wait(bar(kBSFull + s), (uint32_t)((i >> 1) & 1), abort_flag, p.status,
+                      p.wait_limit_ns);
       tc_fence_after();
-      float x[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float tmp[32];
-        tmem_ld32(t_lane + kColS + 128 * s + 32 * c, tmp);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) x[32 * c + k] = tmp[k];
+      float x[64];
+      {
+        float (&x0)[32] = *reinterpret_cast<float(*)[32]>(x);
+        float (&x1)[32] = *reinterpret_cast<float(*)[32]>(x + 32);
+        tmem_ld32(t_lane + kColS + 128 * s + 64 * hf, x0);
+        tmem_ld32(t_lane + kColS + 128 * s + 64 * hf + 32, x1);
       }
       tc_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(kBSFree + s));
-      const int64_t tbase = 128 * (int64_t)i;
-      float mx = -INFINITY;
+      if (i >= first_masked) {
+        const int64_t lim64 = qpos - (128 * (int64_t)i + 64 * hf);
+        const int lim = lim64 < -1 ? -1 : (lim64 > 64 ? 64 : (int)lim64);
 #pragma unroll
-      for (int k = 0; k < 128; ++k) {
-        x[k] = tbase + k <= qpos ? x[k] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[k]);
+        for (int k = 0; k < 64; ++k) x[k] = k <= lim ? x[k] : -INFINITY;
       }
-      // P and O of the previous tile are in use until its PV product completes
-      bool okp = true;
-      if (i >= 1)
-        okp = mbar_wait(bar(kBPvDone), (uint32_t)((i - 1) & 1), abort_flag, p.status,
-                        p.wait_limit_ns);
-      if (__any_sync(0xffffffffu, !ok || !okp)) {
-        ok = false;
-        break;
+      float mx;
+      {
+        float t[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          t[u] = fmax3(fmax3(x[8 * u], x[8 * u + 1], x[8 * u + 2]),
+                       fmax3(x[8 * u + 3], x[8 * u + 4], x[8 * u + 5]), fmaxf(x[8 * u + 6], x[8 * u + 7]));
+        mx = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]), fmaxf(t[6], t[7]));
       }
-      const bool raise = mx > m_used + kAttLazyMax;
+      xmax[(s * 2 + hf) * 128 + row] = mx;
+      xok[(s * 2 + hf) * 128 + row] = ok ? 1 : 0;
+      pair_sync(quarter);
+      mx = fmaxf(mx, xmax[(s * 2 + (hf ^ 1)) * 128 + row]);
+      pair_ok = ok && xok[(s * 2 + (hf ^ 1)) * 128 + row] != 0;
+      if (__any_sync(0xffffffffu, !pair_ok)) break;  // the partner warp decides alike
+      const float mxs = mx * sc;  // scores in log2 units
+      const bool raise = mxs > m_used + kAttLazyMax;
       if (__any_sync(0xffffffffu, raise)) {
-        // the warp rescales its rows of O together (tensor-memory access is per warp)
-        const float m_new = raise ? mx : m_used;
+        // the warp rescales its half rows of O together (tensor-memory access is per warp)
+        const float m_new = raise ? mxs : m_used;
         const float alpha = m_used == -INFINITY ? 0.f : ex2(m_used - m_new);
         l *= raise ? alpha : 1.f;
         if (i >= 1) {
+          // O holds PV(i - 1) once that product completes
+          ok &= mbar_wait(bar(kBPvDone + (s ^ 1)), (uint32_t)(((i - 1) >> 1) & 1), abort_flag,
+                          p.status, p.wait_limit_ns);
           tc_fence_after();
+          const float f = raise ? alpha : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 2; ++c) {
             float o[32];
-            tmem_ld32(t_lane + kColO + 32 * c, o);
+            tmem_ld32(t_lane + kColO + 64 * hf + 32 * c, o);
             tc_wait_ld();
-            const float f = raise ? alpha : 1.f;
 #pragma unroll
             for (int k = 0; k < 32; ++k) o[k] *= f;
-            tmem_st32(t_lane + kColO + 32 * c, o);
+            tmem_st32(t_lane + kColO + 64 * hf + 32 * c, o);
           }
-          tc_wait_st();
         }
         m_used = m_new;
       }
-      // probabilities as fp16 pairs, summed in that precision; the row is one
-      // 128-byte line in each of the two 64-token boxes of P (128-byte swizzle)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint8_t* prow = smem + kAttOffP + c * kTile + row * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k = 64 * c + 8 * u + 2 * e;
-            const float p0 = x[k] == -INFINITY ? 0.f : ex2(x[k] - m_used);
-            const float p1 = x[k + 1] == -INFINITY ? 0.f : ex2(x[k + 1] - m_used);
-            const __half2 hv = __floats2half2_rn(p0, p1);
-            l += __low2float(hv) + __high2float(hv);
-            w[e] = *reinterpret_cast<const uint32_t*>(&hv);
-          }
-          *reinterpret_cast<uint4*>(prow + ((u ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(kBPFull));
-    }
-    // ---- epilogue: O / l, written as the bf16 output row of (query, head)
-    bool have = ok && nt > 0;
-    if (have) {
-      const bool okw = mbar_wait(bar(kBPvDone), (uint32_t)((nt - 1) & 1), abort_flag, p.status,
-                                 p.wait_limit_ns);
-      have = !__any_sync(0xffffffffu, !okw);
-    }
-    if (have) {
+      // P buffer s was read by PV(i - 2)
+      if (i >= 2)
+        ok &= mbar_wait(bar(kBPvDone + s), (uint32_t)(((i - 2) >> 1) & 1), abort_flag, p.status,
+                        p.wait_limit_ns);
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = p.out + ((int64_t)(b * p.q_len + j) * kHeads + h) * kDV;
+      // probabilities as fp16 pairs (token 2w in the low half of column w) into
+      // the half row's 32 columns of P; l sums them before the rounding
+      const float msub = m_used == -INFINITY ? 0.f : m_used;
+      uint32_t w[32];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float p0 = ex2(fmaf(x[2 * e], sc, -msub));
+        const float p1 = ex2(fmaf(x[2 * e + 1], sc, -msub));
+        ls[e & 3] += p0 + p1;
+        const __half2 hv = __floats2half2_rn(p0, p1);
+        w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      tmem_st32u(t_lane + kColP + 64 * s + 32 * hf, w);
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBPFull + s));
+    }
+    // ---- epilogue: O / l, the pair's halves of l summed; bf16 output row of (query, head)
+    if (pair_ok && nt > 0)
+      ok &= mbar_wait(bar(kBPvDone + ((nt - 1) & 1)), (uint32_t)(((nt - 1) >> 1) & 1), abort_flag,
+                      p.status, p.wait_limit_ns);
+    // (the loop above ended for both warps of the pair at the same tile)
+    xmax[(4 + hf) * 128 + row] = l;
+    xok[(4 + hf) * 128 + row] = ok && pair_ok ? 1 : 0;
+    pair_sync(quarter);
+    const float lt = l + xmax[(4 + (hf ^ 1)) * 128 + row];
+    const bool have = nt > 0 && ok && pair_ok && xok[(4 + (hf ^ 1)) * 128 + row] != 0;
+    if (!__any_sync(0xffffffffu, !have)) {
+      tc_fence_after();
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      __nv_bfloat16* dst = p.out + ((int64_t)(b * p.q_len + j) * kHeads + h) * kDV + 64 * hf;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float o[32];
-        tmem_ld32(t_lane + kColO + 32 * c, o);
+        tmem_ld32(t_lane + kColO + 64 * hf + 32 * c, o);
         tc_wait_ld();
         if (qpos >= 0) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            uint32_t w[4];
+            uint32_t wv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const __nv_bfloat162 v =
                   __floats2bfloat162_rn(o[8 * u + 2 * e] * inv, o[8 * u + 2 * e + 1] * inv);
-              w[e] = *reinterpret_cast<const uint32_t*>(&v);
+              wv[e] = *reinterpret_cast<const uint32_t*>(&v);
             }
-            reinterpret_cast<uint4*>(dst + 32 * c)[u] = make_uint4(w[0], w[1], w[2], w[3]);
+            reinterpret_cast<uint4*>(dst + 32 * c)[u] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
           }
         }
       }
