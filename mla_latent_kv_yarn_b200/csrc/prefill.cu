@@ -329,22 +329,25 @@ __global__ void __launch_bounds__(kExpThreads, 1)
 // columns each) at 384 and 448, the A operand of the PV product.  Shared
 // memory: Q (3 boxes of 64 dims), two K stages (K_nope: 2 boxes, rope key: 1
 // box) and two V stages (2 boxes of 64 v), all by TMA with the 128-byte
-// swizzle; and the row statistics the two softmax threads of a row exchange.
-// warp 0 TMA, warp 1 MMA, warps 2-9 softmax: a query row is shared by warps w
-// and w + 4 (the same tensor-memory lane quarter, w & 3), each taking 64 of a
-// tile's 128 tokens and 64 of the 128 v columns of O
-constexpr int kAttThreads = 320;
-constexpr int kAttSoftmax = 256;
+// swizzle; and the row statistics the softmax warps hand on.
+// Warp 0 loads Q and K, warp 10 V (each as soon as its stage is free), warp 1
+// issues the MMAs, warps 2-9 are the softmax in two groups of four: group g
+// (warps 2 + 4g .. 5 + 4g) takes the key tiles i = g mod 2, through S buffer g
+// and P buffer g, one query row per thread (its lane of quarter warp & 3).  The
+// groups overlap: while one turns its scores into probabilities, the other
+// reads the next tile's; a row's running maximum passes from tile to tile
+// through shared memory, so the softmax is the one-pass online form.
+constexpr int kAttThreads = 352;
+constexpr int kAttGroup = 128;
 constexpr uint32_t kAttOffQ = 0;
 constexpr uint32_t kAttOffK = kAttOffQ + 3 * kTile;
 constexpr uint32_t kAttKStage = 3 * kTile;
 constexpr uint32_t kAttOffV = kAttOffK + 2 * kAttKStage;
 constexpr uint32_t kAttVStage = 2 * kTile;
-// [slot][half][row]: the half-row maxima (float), then the ok flags (int);
-// slots 0, 1 by tile parity, slot 2 for the row sums at the end
+// the running maximum handed from group to group [2][128], then each group's
+// (l, m, ok) at the end [2][3][128]
 constexpr uint32_t kAttOffXchg = kAttOffV + 2 * kAttVStage;
-constexpr uint32_t kAttXchgSlots = 3 * 2 * 128;
-constexpr uint32_t kAttXchgBytes = 2 * kAttXchgSlots * 4;
+constexpr uint32_t kAttXchgBytes = (2 + 6) * 128 * 4;
 constexpr uint32_t kAttOffBars = kAttOffXchg + kAttXchgBytes;
 // barriers
 constexpr int kBQ = 0;
@@ -373,9 +376,13 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// the two warps that share a lane quarter meet here (named barrier 1 + quarter)
-__device__ __forceinline__ void pair_sync(int quarter) {
-  asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+// named barriers 1..12 among the warps of one lane quarter (64 threads: the
+// one of each softmax group); the producer arrives, the consumer waits
+__device__ __forceinline__ void nbar_arrive(int id) {
+  asm volatile("bar.arrive %0, 64;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ void nbar_sync(int id) {
+  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
 }
 
 // D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16: A's rows are tensor-memory
@@ -432,8 +439,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       mbar_init(bar(kBVFull + i), 1);
       mbar_init(bar(kBVEmpty + i), 1);
       mbar_init(bar(kBSFull + i), 1);
-      mbar_init(bar(kBSFree + i), kAttSoftmax);
-      mbar_init(bar(kBPFull + i), kAttSoftmax);
+      mbar_init(bar(kBSFree + i), kAttGroup);
+      mbar_init(bar(kBPFull + i), kAttGroup);
       mbar_init(bar(kBPvDone + i), 1);
     }
     mbar_init(bar(kBDrain), 1);
@@ -471,34 +478,44 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       mbar_arrive_expect_tx(bar(kBQ), 3 * kTile);
       for (int k = 0; k < 3; ++k)
         tma_load_3d(base + kAttOffQ + k * kTile, &tmap_q, 64 * k, h, qrow0, bar(kBQ));
-      // K(i) and V(i) go to stage i % 2 once QK(i - 2) and PV(i - 2) are done
-      int nk = 0, nv = 0;  // tiles whose K, V copies were issued
+      // K(i) goes to stage i % 2 once QK(i - 2) is done
+      int nk = 0;  // tiles whose K copies were issued
       for (int i = 0; i < nt; ++i) {
         const int s = i & 1;
-        const int32_t r = (int32_t)(krow0 + 128 * (int64_t)i);
         if (i >= 2 && !mbar_wait(bar(kBKEmpty + s), (uint32_t)(((i - 2) >> 1) & 1), abort_flag,
                                  p.status, p.wait_limit_ns))
           break;
+        const int32_t r = (int32_t)(krow0 + 128 * (int64_t)i);
         const uint32_t kst = base + kAttOffK + s * kAttKStage;
         mbar_arrive_expect_tx(bar(kBKFull + s), kAttKStage);
         tma_load_3d(kst, &tmap_k, 0, h, r, bar(kBKFull + s));
         tma_load_3d(kst + kTile, &tmap_k, 64, h, r, bar(kBKFull + s));
         tma_load_2d(kst + 2 * kTile, &tmap_kp, 0, r, bar(kBKFull + s));
         nk = i + 1;
-        if (i >= 2 && !mbar_wait(bar(kBVEmpty + s), (uint32_t)(((i - 2) >> 1) & 1), abort_flag,
-                                 p.status, p.wait_limit_ns))
-          break;
-        const uint32_t vst = base + kAttOffV + s * kAttVStage;
-        mbar_arrive_expect_tx(bar(kBVFull + s), kAttVStage);
-        tma_load_3d(vst, &tmap_v, 0, h, r, bar(kBVFull + s));
-        tma_load_3d(vst + kTile, &tmap_v, 64, h, r, bar(kBVFull + s));
-        nv = i + 1;
       }
       // every copy issued must land before the CTA may exit
       mbar_wait(bar(kBQ), 0, nullptr, p.status, p.wait_limit_ns);
       for (int i = nk > 2 ? nk - 2 : 0; i < nk; ++i)
         mbar_wait(bar(kBKFull + (i & 1)), (uint32_t)((i >> 1) & 1), nullptr, p.status,
                   p.wait_limit_ns);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ V producer
+    if (lane == 0 && nt > 0) {
+      // V(i) goes to stage i % 2 once PV(i - 2) is done
+      int nv = 0;
+      for (int i = 0; i < nt; ++i) {
+        const int s = i & 1;
+        if (i >= 2 && !mbar_wait(bar(kBVEmpty + s), (uint32_t)(((i - 2) >> 1) & 1), abort_flag,
+                                 p.status, p.wait_limit_ns))
+          break;
+        const int32_t r = (int32_t)(krow0 + 128 * (int64_t)i);
+        const uint32_t vst = base + kAttOffV + s * kAttVStage;
+        mbar_arrive_expect_tx(bar(kBVFull + s), kAttVStage);
+        tma_load_3d(vst, &tmap_v, 0, h, r, bar(kBVFull + s));
+        tma_load_3d(vst + kTile, &tmap_v, 64, h, r, bar(kBVFull + s));
+        nv = i + 1;
+      }
       for (int i = nv > 2 ? nv - 2 : 0; i < nv; ++i)
         mbar_wait(bar(kBVFull + (i & 1)), (uint32_t)((i >> 1) & 1), nullptr, p.status,
                   p.wait_limit_ns);
@@ -532,8 +549,10 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       bool ok = wait(kBQ, 0);
       tc_fence_after();
       if (ok) ok = qk(0);
+      if (ok && nt > 1) ok = qk(1);
       for (int i = 0; i < nt && ok; ++i) {
-        if (i + 1 < nt && !(ok = qk(i + 1))) break;
+        // QK(i + 2) first: its S buffer is free as soon as tile i's scores are read
+        if (i + 2 < nt && !(ok = qk(i + 2))) break;
         const int s = i & 1;
         if (!(ok = wait(kBPFull + s, (uint32_t)((i >> 1) & 1)))) break;
         if (!(ok = wait(kBVFull + s, (uint32_t)((i >> 1) & 1)))) break;
@@ -550,127 +569,139 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       mbar_wait(bar(kBDrain), 0, nullptr, p.status, p.wait_limit_ns);
     }
   } else {
-    // ------------------------------------------------------------ softmax, half a query row per thread
+    // ------------------------------------------------------------ softmax, one query row per thread
+    const int g = (warp - 2) >> 2;        // key tiles i = g mod 2
     const int quarter = warp & 3;
-    const int hf = (warp - 2) >> 2;       // tokens 64 hf .. 64 hf + 63 of a tile; v columns likewise
     const int row = 32 * quarter + lane;  // tensor-memory lane = query row of the tile
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quarter) << 16);
-    float* xmax = reinterpret_cast<float*>(smem + kAttOffXchg);
-    int* xok = reinterpret_cast<int*>(smem + kAttOffXchg + kAttXchgSlots * 4);
+    float* hand = reinterpret_cast<float*>(smem + kAttOffXchg);  // [from group][row]
+    float* fin = hand + 2 * 128;                                // [group][l, m, ok][row]
     const int j = j0 + row;
     // the row's last visible token (the query's own position); -1 for a padding row
     const int64_t qpos = j < j0 + jn ? seqlen - p.q_len + j : -1;
     // tiles from here on hold tokens past some row's position: they are masked
     const int64_t first_masked = (seqlen - p.q_len + j0 + 1) / 128;
     const float sc = p.scale_log2;
-    float m_used = -INFINITY, l = 0.f;
-    bool ok = true, pair_ok = true;
-    // Every exit is taken by both warps of a pair at the same point (after an
-    // exchange), so neither is left waiting at the named barrier; a failed wait
-    // only marks the thread, which finishes the tile on whatever it read.
-    for (int i = 0; i < nt; ++i) {
-      const int s = i & 1;
-      ok &= mbar_wait(bar(kBSFull + s), (uint32_t)((i >> 1) & 1), abort_flag, p.status,
+    // m_w: the running maximum (log2 units) this group's l_w is expressed in
+    float l_w = 0.f, m_w = -INFINITY;
+    bool ok = true;
+    // No exit before the end: every handoff below has its partner in the other
+    // group, so a failed wait only marks the thread, which carries on with
+    // whatever it read (the abort flag makes the remaining waits short).
+    for (int i = g; i < nt; i += 2) {
+      ok &= mbar_wait(bar(kBSFull + g), (uint32_t)((i >> 1) & 1), abort_flag, p.status,
                       p.wait_limit_ns);
       tc_fence_after();
-      float x[64];
-      {
-        float (&x0)[32] = *reinterpret_cast<float(*)[32]>(x);
-        float (&x1)[32] = *reinterpret_cast<float(*)[32]>(x + 32);
-        tmem_ld32(t_lane + kColS + 128 * s + 64 * hf, x0);
-        tmem_ld32(t_lane + kColS + 128 * s + 64 * hf + 32, x1);
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float (&xc)[32] = *reinterpret_cast<float(*)[32]>(x + 32 * c);
+        tmem_ld32(t_lane + kColS + 128 * g + 32 * c, xc);
       }
       tc_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(kBSFree + s));
+      mbar_arrive(bar(kBSFree + g));
       if (i >= first_masked) {
-        const int64_t lim64 = qpos - (128 * (int64_t)i + 64 * hf);
-        const int lim = lim64 < -1 ? -1 : (lim64 > 64 ? 64 : (int)lim64);
+        const int64_t lim64 = qpos - 128 * (int64_t)i;
+        const int lim = lim64 < -1 ? -1 : (lim64 > 128 ? 128 : (int)lim64);
 #pragma unroll
-        for (int k = 0; k < 64; ++k) x[k] = k <= lim ? x[k] : -INFINITY;
+        for (int k = 0; k < 128; ++k) x[k] = k <= lim ? x[k] : -INFINITY;
       }
-      float mx;
+      float mxs;
       {
-        float t[8];
+        float t[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+        for (int u = 0; u < 16; ++u)
           t[u] = fmax3(fmax3(x[8 * u], x[8 * u + 1], x[8 * u + 2]),
                        fmax3(x[8 * u + 3], x[8 * u + 4], x[8 * u + 5]), fmaxf(x[8 * u + 6], x[8 * u + 7]));
-        mx = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]), fmaxf(t[6], t[7]));
+        const float a = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]), fmax3(t[6], t[7], t[8]));
+        const float b2 = fmax3(fmax3(t[9], t[10], t[11]), fmax3(t[12], t[13], t[14]), t[15]);
+        mxs = fmaxf(a, b2) * sc;  // in log2 units
       }
-      xmax[(s * 2 + hf) * 128 + row] = mx;
-      xok[(s * 2 + hf) * 128 + row] = ok ? 1 : 0;
-      pair_sync(quarter);
-      mx = fmaxf(mx, xmax[(s * 2 + (hf ^ 1)) * 128 + row]);
-      pair_ok = ok && xok[(s * 2 + (hf ^ 1)) * 128 + row] != 0;
-      if (__any_sync(0xffffffffu, !pair_ok)) break;  // the partner warp decides alike
-      const float mxs = mx * sc;  // scores in log2 units
-      const bool raise = mxs > m_used + kAttLazyMax;
-      if (__any_sync(0xffffffffu, raise)) {
-        // the warp rescales its half rows of O together (tensor-memory access is per warp)
-        const float m_new = raise ? mxs : m_used;
-        const float alpha = m_used == -INFINITY ? 0.f : ex2(m_used - m_new);
-        l *= raise ? alpha : 1.f;
-        if (i >= 1) {
-          // O holds PV(i - 1) once that product completes
-          ok &= mbar_wait(bar(kBPvDone + (s ^ 1)), (uint32_t)(((i - 1) >> 1) & 1), abort_flag,
-                          p.status, p.wait_limit_ns);
-          tc_fence_after();
-          const float f = raise ? alpha : 1.f;
+      // the running maximum after tile i - 1, from the other group
+      float m_prev = -INFINITY;
+      if (i >= 1) {
+        nbar_sync(1 + 4 * (g ^ 1) + quarter);
+        m_prev = hand[(g ^ 1) * 128 + row];
+      }
+      const bool raise = mxs > m_prev + kAttLazyMax;
+      const float m_cur = raise ? mxs : m_prev;
+      if (i + 1 < nt) {
+        hand[g * 128 + row] = m_cur;
+        nbar_arrive(1 + 4 * g + quarter);
+      }
+      if (i >= 1 && __any_sync(0xffffffffu, raise)) {
+        // O holds PV(i - 1) once that product completes; the warp rescales its
+        // rows together (tensor-memory access is per warp)
+        ok &= mbar_wait(bar(kBPvDone + (g ^ 1)), (uint32_t)(((i - 1) >> 1) & 1), abort_flag,
+                        p.status, p.wait_limit_ns);
+        tc_fence_after();
+        const float f = raise && m_prev != -INFINITY ? ex2(m_prev - m_cur) : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            float o[32];
-            tmem_ld32(t_lane + kColO + 64 * hf + 32 * c, o);
-            tc_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(t_lane + kColO + 32 * c, o);
+          tc_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] *= f;
-            tmem_st32(t_lane + kColO + 64 * hf + 32 * c, o);
-          }
+          for (int k = 0; k < 32; ++k) o[k] *= f;
+          tmem_st32(t_lane + kColO + 32 * c, o);
         }
-        m_used = m_new;
       }
-      // P buffer s was read by PV(i - 2)
+      if (m_cur != m_w) {
+        l_w = m_w == -INFINITY ? 0.f : l_w * ex2(m_w - m_cur);
+        m_w = m_cur;
+      }
+      // P buffer g was read by PV(i - 2)
       if (i >= 2)
-        ok &= mbar_wait(bar(kBPvDone + s), (uint32_t)(((i - 2) >> 1) & 1), abort_flag, p.status,
+        ok &= mbar_wait(bar(kBPvDone + g), (uint32_t)(((i - 2) >> 1) & 1), abort_flag, p.status,
                         p.wait_limit_ns);
       tc_fence_after();
       // probabilities as fp16 pairs (token 2w in the low half of column w) into
-      // the half row's 32 columns of P; l sums them before the rounding
-      const float msub = m_used == -INFINITY ? 0.f : m_used;
-      uint32_t w[32];
+      // the row's 64 columns of P buffer g; l sums them before the rounding
+      const float msub = m_cur == -INFINITY ? 0.f : m_cur;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float p0 = ex2(fmaf(x[2 * e], sc, -msub));
-        const float p1 = ex2(fmaf(x[2 * e + 1], sc, -msub));
-        ls[e & 3] += p0 + p1;
-        const __half2 hv = __floats2half2_rn(p0, p1);
-        w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = ex2(fmaf(x[64 * c + 2 * e], sc, -msub));
+          const float p1 = ex2(fmaf(x[64 * c + 2 * e + 1], sc, -msub));
+          ls[e & 3] += p0 + p1;
+          const __half2 hv = __floats2half2_rn(p0, p1);
+          w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        tmem_st32u(t_lane + kColP + 64 * g + 32 * c, w);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      tmem_st32u(t_lane + kColP + 64 * s + 32 * hf, w);
+      l_w += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(kBPFull + s));
+      mbar_arrive(bar(kBPFull + g));
     }
-    // ---- epilogue: O / l, the pair's halves of l summed; bf16 output row of (query, head)
-    if (pair_ok && nt > 0)
+    // ---- epilogue: the groups' sums brought to the final maximum; O / l as the
+    // bf16 output row of (query, head), v columns 64 g .. 64 g + 63 by group g
+    if (nt > 0)
       ok &= mbar_wait(bar(kBPvDone + ((nt - 1) & 1)), (uint32_t)(((nt - 1) >> 1) & 1), abort_flag,
                       p.status, p.wait_limit_ns);
-    // (the loop above ended for both warps of the pair at the same tile)
-    xmax[(4 + hf) * 128 + row] = l;
-    xok[(4 + hf) * 128 + row] = ok && pair_ok ? 1 : 0;
-    pair_sync(quarter);
-    const float lt = l + xmax[(4 + (hf ^ 1)) * 128 + row];
-    const bool have = nt > 0 && ok && pair_ok && xok[(4 + (hf ^ 1)) * 128 + row] != 0;
+    fin[(3 * g + 0) * 128 + row] = l_w;
+    fin[(3 * g + 1) * 128 + row] = m_w;
+    fin[(3 * g + 2) * 128 + row] = ok ? 1.f : 0.f;
+    nbar_sync(9 + quarter);
+    const float l_o = fin[(3 * (g ^ 1) + 0) * 128 + row];
+    const float m_o = fin[(3 * (g ^ 1) + 1) * 128 + row];
+    const bool have = nt > 0 && ok && fin[(3 * (g ^ 1) + 2) * 128 + row] != 0.f;
     if (!__any_sync(0xffffffffu, !have)) {
       tc_fence_after();
+      const float m_f = fmaxf(m_w, m_o);
+      float lt = 0.f;
+      if (m_w != -INFINITY) lt += l_w * ex2(m_w - m_f);
+      if (m_o != -INFINITY) lt += l_o * ex2(m_o - m_f);
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      __nv_bfloat16* dst = p.out + ((int64_t)(b * p.q_len + j) * kHeads + h) * kDV + 64 * hf;
+      __nv_bfloat16* dst = p.out + ((int64_t)(b * p.q_len + j) * kHeads + h) * kDV + 64 * g;
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         float o[32];
-        tmem_ld32(t_lane + kColO + 64 * hf + 32 * c, o);
+        tmem_ld32(t_lane + kColO + 64 * g + 32 * c, o);
         tc_wait_ld();
         if (qpos >= 0) {
 #pragma unroll
