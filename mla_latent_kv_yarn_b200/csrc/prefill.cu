@@ -370,6 +370,15 @@ constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 // (log2 units), so an O rescale is rare
 constexpr float kAttLazyMax = 8.0f;
 
+// The softmax waits end in __syncwarp: lanes that leave the polling loop at
+// different iterations meet again before the warp-wide tcgen05.ld / st.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               int32_t* status, uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort, status, limit_ns);
+  __syncwarp();
+  return ok;
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -589,7 +598,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     // group, so a failed wait only marks the thread, which carries on with
     // whatever it read (the abort flag makes the remaining waits short).
     for (int i = g; i < nt; i += 2) {
-      ok &= mbar_wait(bar(kBSFull + g), (uint32_t)((i >> 1) & 1), abort_flag, p.status,
+      ok &= mbar_wait_warp(bar(kBSFull + g), (uint32_t)((i >> 1) & 1), abort_flag, p.status,
                       p.wait_limit_ns);
       tc_fence_after();
       float x[128];
@@ -633,7 +642,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       if (i >= 1 && __any_sync(0xffffffffu, raise)) {
         // O holds PV(i - 1) once that product completes; the warp rescales its
         // rows together (tensor-memory access is per warp)
-        ok &= mbar_wait(bar(kBPvDone + (g ^ 1)), (uint32_t)(((i - 1) >> 1) & 1), abort_flag,
+        ok &= mbar_wait_warp(bar(kBPvDone + (g ^ 1)), (uint32_t)(((i - 1) >> 1) & 1), abort_flag,
                         p.status, p.wait_limit_ns);
         tc_fence_after();
         const float f = raise && m_prev != -INFINITY ? ex2(m_prev - m_cur) : 1.f;
@@ -653,7 +662,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       }
       // P buffer g was read by PV(i - 2)
       if (i >= 2)
-        ok &= mbar_wait(bar(kBPvDone + g), (uint32_t)(((i - 2) >> 1) & 1), abort_flag, p.status,
+        ok &= mbar_wait_warp(bar(kBPvDone + g), (uint32_t)(((i - 2) >> 1) & 1), abort_flag, p.status,
                         p.wait_limit_ns);
       tc_fence_after();
       // probabilities as fp16 pairs (token 2w in the low half of column w) into
@@ -681,7 +690,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     // ---- epilogue: the groups' sums brought to the final maximum; O / l as the
     // bf16 output row of (query, head), v columns 64 g .. 64 g + 63 by group g
     if (nt > 0)
-      ok &= mbar_wait(bar(kBPvDone + ((nt - 1) & 1)), (uint32_t)(((nt - 1) >> 1) & 1), abort_flag,
+      ok &= mbar_wait_warp(bar(kBPvDone + ((nt - 1) & 1)), (uint32_t)(((nt - 1) >> 1) & 1), abort_flag,
                       p.status, p.wait_limit_ns);
     fin[(3 * g + 0) * 128 + row] = l_w;
     fin[(3 * g + 1) * 128 + row] = m_w;
