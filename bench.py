@@ -61,7 +61,7 @@ def parse_args():
                          "(torchrun) each rank holds one shard and the partials are all-gathered "
                          "over NCCL; on one GPU, rank 0's share is timed (its shard, the gathered "
                          "partials' combine; the all-gather becomes a local copy)")
-    ap.add_argument("--workloads", default="decode_4k,step_40l_b32,verify_q4_b8,decode_512k_b4",
+    ap.add_argument("--workloads", default="decode_4k,step_40l_b32,verify_q4_b8,decode_512k_b4,prefill_4k",
                     help="other workloads measured in the same run (one GPU; step and split-K "
                          "kernel times and roofline fractions under the line's 'workloads' key); "
                          "empty to skip")
@@ -269,22 +269,24 @@ def run_reference(args, wl):
 
 # ------------------------------------------------------------------ GPU arm
 
-# the translation unit of the split-K kernel: its source and the headers it includes
+# the translation unit of the timed kernel: its source and the headers it includes
+# (the split-K kernel, or a prompt chunk's attention kernel)
 KERNEL_SOURCES = ["mla_decode.cu", "split_kv.h", "xmla_device.cuh"]
+PREFILL_SOURCES = ["prefill.cu", "prefill.h", "xmla_device.cuh"]
 
 
-def kernel_sources_sha() -> str:
+def kernel_sources_sha(names=None) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in names or KERNEL_SOURCES:
         with open(os.path.join(ROOT, "mla_latent_kv_yarn_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def traffic_record(kernel_src_sha: str, name: str):
-    """DRAM bytes per launch of the split-K kernel from a committed ncu summary,
+def traffic_record(kernel_src_sha: str, name: str, kernel: str = "mla_decode_kernel"):
+    """DRAM bytes per launch of the timed kernel from a committed ncu summary,
     valid only while the kernel source is unchanged."""
-    p = os.path.join(ROOT, "profiles", f"mla_decode_kernel_{name}_dram.json")
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{name}_dram.json")
     try:
         with open(p) as f:
             d = json.load(f)
@@ -608,8 +610,10 @@ def run_xmla(args, wl):
     flops_layer = pair_flops(wl) * 32 * pairs
     attn_mean_ms = statistics.mean(attn_ms)
     achieved = cache_bytes_layer / (attn_mean_ms * 1e-3) / 1e9
-    ksha = kernel_sources_sha()
-    traffic = None if q8 else traffic_record(ksha, wl.name)
+    if wl.q_len >= PREFILL_MIN_CHUNK:
+        traffic = traffic_record(kernel_sources_sha(PREFILL_SOURCES), wl.name, "prefill_attn_kernel")
+    else:
+        traffic = None if q8 else traffic_record(kernel_sources_sha(), wl.name)
     # per layer and step: prologue (append or producer + q absorb), split-K
     # attention, combine; on the 8-bit cache the append is a kernel of its own; a
     # prompt chunk: query prep (+ append), K/V expansion, attention
