@@ -434,10 +434,12 @@ __global__ void __launch_bounds__(kAttThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kAttOffAbort);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // the last query tiles see the most tokens: they run first
-  const int qt = (int)(gridDim.x - 1 - blockIdx.x);
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
+  // Blocks start in the order x, y, z: every head and sequence of the last
+  // query tile (the most tokens) first, then the tile before it, and so on,
+  // so the long units start first across the whole grid.
+  const int qt = (int)(gridDim.z - 1 - blockIdx.z);
+  const int h = blockIdx.x;
+  const int b = blockIdx.y;
   const int j0 = qt * 128;
 
   if (threadIdx.x == 0) {
@@ -779,7 +781,7 @@ cudaError_t launch_prefill_attn(const CUtensorMap& q_map, const CUtensorMap& k_m
   static bool done[64] = {};
   const cudaError_t e = set_smem(prefill_attn_kernel, kAttSmem, done);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((p.q_len + 127) / 128), kHeads, (unsigned)p.batch);
+  const dim3 grid(kHeads, (unsigned)p.batch, (unsigned)((p.q_len + 127) / 128));
   return launch_pdl(prefill_attn_kernel, grid, dim3(kAttThreads), kAttSmem, st, q_map, k_map,
                     kp_map, v_map, p);
 }
