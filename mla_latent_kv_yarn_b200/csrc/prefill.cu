@@ -96,8 +96,8 @@ __global__ void __launch_bounds__(kPrepThreads)
       cs[rr][i][0] = c * q_tab.magnitude;
       cs[rr][i][1] = s * q_tab.magnitude;
     }
-    __syncthreads();
-    // q_nope: 16 pieces of 8 values per (row, head)
+    // q_nope: 16 pieces of 8 values per (row, head), converted while the
+    // angles are formed
     for (int e = t; e < nr * kHeads * 16; e += kPrepThreads) {
       const int64_t rh = (int64_t)r_lo * kHeads + e / 16;
       const int u = e % 16;
@@ -109,16 +109,34 @@ __global__ void __launch_bounds__(kPrepThreads)
       for (int k = 0; k < 4; ++k) ow[k] = pack_half2(__low2float(b2[k]), __high2float(b2[k]));
       *reinterpret_cast<uint4*>(qh + rh * kDQ + 8 * u) = o;
     }
-    // rotated q_pe: pair (i, i + 32) of every (row, head)
-    for (int e = t; e < nr * kHeads * kPairs; e += kPrepThreads) {
-      const int rr = e / (kHeads * kPairs), i = e % kPairs;
-      const int64_t rh = (int64_t)(r_lo + rr) * kHeads + (e / kPairs) % kHeads;
+    __syncthreads();
+    // rotated q_pe: pairs (i, i + 32) for four consecutive i per thread
+    for (int e = t; e < nr * kHeads * (kPairs / 4); e += kPrepThreads) {
+      const int rr = e / (kHeads * (kPairs / 4));
+      const int i0 = 4 * (e % (kPairs / 4));
+      const int64_t rh = (int64_t)(r_lo + rr) * kHeads + (e / (kPairs / 4)) % kHeads;
       const __nv_bfloat16* x = q + rh * kDQ + kDNope;
-      const double x1 = (double)__bfloat162float(x[i]), x2 = (double)__bfloat162float(x[i + kPairs]);
-      const double c = cs[rr][i][0], s = cs[rr][i][1];
+      const uint2 lo = *reinterpret_cast<const uint2*>(x + i0);
+      const uint2 hi = *reinterpret_cast<const uint2*>(x + i0 + kPairs);
+      const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lo);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hi);
+      uint32_t o1[2], o2[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const double xa0 = (double)__low2float(l2[k]), xa1 = (double)__high2float(l2[k]);
+        const double xb0 = (double)__low2float(h2[k]), xb1 = (double)__high2float(h2[k]);
+        const double c0 = cs[rr][i0 + 2 * k][0], s0 = cs[rr][i0 + 2 * k][1];
+        const double c1 = cs[rr][i0 + 2 * k + 1][0], s1 = cs[rr][i0 + 2 * k + 1][1];
+        const __half2 ra = __halves2half2(__double2half(xa0 * c0 - xb0 * s0),
+                                          __double2half(xa1 * c1 - xb1 * s1));
+        const __half2 rb = __halves2half2(__double2half(xb0 * c0 + xa0 * s0),
+                                          __double2half(xb1 * c1 + xa1 * s1));
+        o1[k] = *reinterpret_cast<const uint32_t*>(&ra);
+        o2[k] = *reinterpret_cast<const uint32_t*>(&rb);
+      }
       __half* o = qh + rh * kDQ + kDNope;
-      o[i] = __double2half(x1 * c - x2 * s);
-      o[i + kPairs] = __double2half(x2 * c + x1 * s);
+      *reinterpret_cast<uint2*>(o + i0) = make_uint2(o1[0], o1[1]);
+      *reinterpret_cast<uint2*>(o + i0 + kPairs) = make_uint2(o2[0], o2[1]);
     }
     return;
   }
