@@ -115,3 +115,21 @@ def test_row_counts_beyond_int32_are_rejected(x):
     # the shard combine checks the same bound before touching any pointer
     fake = ctypes.c_void_p(256)
     assert L.xmla_combine_shards(fake, 2, fake, 1 << 16, 1024, fake, None) == 2
+
+
+def test_prompt_chunk_workspace_covers_the_non_absorbed_path(x):
+    # From 64 new tokens a chunk runs the non-absorbed form: the workspace holds
+    # the fp16 queries [rows, 32, 192], K_nope and V [B * s_pad, 32, 128] each and
+    # the rope key [B * s_pad, 64] (s_pad = max_seqlen rounded up to 128), each
+    # piece 1 KiB aligned.  Below 64 tokens the absorbed form's smaller plan.
+    def prefill_bytes(batch, q_len, max_seqlen):
+        up = lambda v: (v + 1023) // 1024 * 1024
+        s_pad = (max_seqlen + 127) // 128 * 128
+        kx = up(batch * q_len * 32 * 192 * 2)
+        vx = up(kx + batch * s_pad * 32 * 128 * 2)
+        kp = up(vx + batch * s_pad * 32 * 128 * 2)
+        return up(kp + batch * s_pad * 64 * 2)
+    for batch, q_len, n in [(1, 64, 4096), (1, 4096, 4096), (3, 100, 5000), (2, 128, 129)]:
+        assert x.xmla_decode_workspace_size(batch, q_len, n, 148) >= prefill_bytes(batch, q_len, n)
+    # one token fewer: the absorbed plan, which needs no expanded K/V
+    assert x.xmla_decode_workspace_size(1, 63, 4096, 148) < prefill_bytes(1, 64, 4096)
