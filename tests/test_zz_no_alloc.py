@@ -49,6 +49,28 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls():
         assert torch.equal(out, ref)
 
 
+def test_noalloc_prompt_chunk_matches_workspace_decode():
+    # a 128-token chunk runs the non-absorbed path (about 14 MB of workspace)
+    wl = workloads.custom(1, 128, [700], seed=43)
+    cfg, ocfg = gc.cfgs()
+    inp = workloads.layer_inputs(wl, 0, "cpu")
+    _, dec, st = gc.gpu_step(wl, inp, cfg)
+    q = inp.q.cuda()
+    scale = xmla.xmla_softmax_scale(cfg, 192)
+    ref = dec.decode(cfg, st, q, scale).clone()
+    torch.cuda.synchronize()
+    assert dec.check_status() == 0
+    assert xmla.xmla_decode_workspace_size(1, 128, 700, dec.sms, 0) <= (32 << 20)
+    out = torch.full_like(ref, float("nan"))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    xmla.xmla_decode_noalloc(cfg, q, st.W_UK, st.W_UV, st.pool, st.num_blocks, st.block_table,
+                             st.max_blocks, st.seqlens, wl.batch, wl.q_len, wl.max_seqlen,
+                             scale, 0, status, out)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(out, ref)
+
+
 def test_noalloc_decode_rejects_sizes_beyond_its_scratch():
     cfg, _ = gc.cfgs()
     # 256 sequences x 8 queries at 1M context need far more than the fixed scratch
