@@ -67,7 +67,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 // ---------------------------------------------------------------- prep
 
 constexpr int kPrepThreads = 256;
-constexpr int kPrepRows = 4;  // query rows (all 32 heads) per block
+constexpr int kPrepRows = 2;  // query rows (all 32 heads) per block
 
 // Blocks [0, ceil(rows / kPrepRows)): qh[r, h] = [q_nope | rope(q_pe, pos_r)]
 // as fp16, pos_r = seqlens[b] - q_len + j for r = b * q_len + j (the angle in
